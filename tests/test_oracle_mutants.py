@@ -1,0 +1,74 @@
+"""Planted mistakes in copies of the oracle must each fail at least one pin.
+
+Every case compiles a copy of oracle/attn_oracle.c with one plausible slip (a dropped term, a
+wrong sign, a wrong index, an off-by-one, a transposed operand) into a temporary library and
+runs the whole pin suite against it on the CPU. The built oracle itself is never modified.
+"""
+import os
+import subprocess
+import tempfile
+
+import pytest
+
+import oracle
+from tests import oracle_pins
+
+SRC = os.path.join(os.path.dirname(oracle.__file__), "attn_oracle.c")
+
+# (name, original text, replacement, which occurrence)
+MUTANTS = [
+    ("dropped_scale", "s[j] = scale * acc;", "s[j] = acc;", 0),
+    ("gqa_index_modulo", "h / group, nk, Nq, Nkv, Sq, Skv, D,\n                 scale, s, out + oo",
+     "h % Nkv, nk, Nq, Nkv, Sq, Skv, D,\n                 scale, s, out + oo", 0),
+    ("keys_from_query_sequence", "ld(k, offs(layout, b, tk0, j, g, d", "ld(k, offs(layout, b, tq0, j, g, d", 0),
+    ("values_use_key_head_of_query", "ld(v, offs(layout, b, tk0, j, g, d", "ld(v, offs(layout, b, tk0, j, h % Nkv, d", 0),
+    ("causal_off_by_one", "return last + 1 < sk ? last + 1 : sk;", "return last < sk ? last : sk;", 0),
+    ("bottomright_sign", "i + sk - sq", "i + sq - sk", 0),
+    ("max_not_subtracted", "s[j] = exp(s[j] - mx);", "s[j] = exp(s[j]);", 0),
+    ("dropped_normalisation", "for (d = 0; d < D; ++d) o[d] /= sum;\n  *m = mx;",
+     "for (d = 0; d < D; ++d) o[d] /= 1.0;\n  *m = mx;", 0),
+    ("sequence_search_off_by_one", "while (cu_q[b] <= tok) ++b; /* sequence", "while (cu_q[b] < tok) ++b; /* sequence", 0),
+    ("stats_head_major", "(tq0 + i) * Nq + h;", "(tq0 + i) + h * Sq;", 0),
+    ("csr_scale_without_sqrt", "1.0 / sqrt((double)D)", "1.0 / (double)D", 0),
+    ("csr_first_slice_only", "base = bhi * (int64_t)S * D;", "base = 0;", 0),
+    ("csr_query_transposed", "ld(q, rowq + d, et) * ld(k, base + j * D + d, et)",
+     "ld(q, base + j * D + d, et) * ld(k, rowq + d, et)", 0),
+    ("csr_normalisation_dropped", "for (d = 0; d < D; ++d) o[d] /= sum;\n    }\n    free(s);",
+     "for (d = 0; d < D; ++d) o[d] /= 1.0;\n    }\n    free(s);", 0),
+    ("merge_exp_sign", "prev_sum[x] * exp(pm - m)", "prev_sum[x] * exp(m - pm)", 0),
+    ("merge_uses_lane_1", "po = l[0] != 0.0 ? ps_scaled[0] / l[0] : 0.0;",
+     "po = l[1] != 0.0 ? ps_scaled[1] / l[1] : 0.0;", 0),
+    ("merge_bsh_indexing", "((s * B + b) * N + n) * (int64_t)D + d", "((b * S + s) * N + n) * (int64_t)D + d", 0),
+    ("merge_swapped_sides", "ld(prev_out, x, et) * po + ld(cur_out, x, et) * co",
+     "ld(prev_out, x, et) * co + ld(cur_out, x, et) * po", 0),
+    ("merge_sum_not_rescaled", "cs_scaled[lane] = cur_sum[x] * exp(cm - m);", "cs_scaled[lane] = cur_sum[x];", 0),
+    ("bf16_truncates", "nearbyint(m * 256.0)", "floor(m * 256.0)", 0),
+]
+
+
+def _mutate(text, old, new, nth):
+    pos = -1
+    for _ in range(nth + 1):
+        pos = text.find(old, pos + 1)
+        assert pos >= 0, f"mutation anchor not found: {old!r}"
+    return text[:pos] + new + text[pos + len(old):]
+
+
+@pytest.mark.parametrize("name,old,new,nth", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_planted_mistake_is_caught(name, old, new, nth, tmp_path):
+    src = open(SRC).read()
+    mutated = _mutate(src, old, new, nth)
+    assert mutated != src
+    c = tmp_path / "mutant.c"
+    so = tmp_path / "mutant.so"
+    c.write_text(mutated)
+    subprocess.run(["gcc", "-O1", "-std=c99", "-fPIC", "-shared", "-o", str(so), str(c), "-lm"],
+                   check=True)
+    failed = []
+    with oracle.using(str(so)):
+        for pin in oracle_pins.ALL_PINS:
+            try:
+                pin()
+            except Exception:  # an assertion, or the mutant rejecting valid input
+                failed.append(pin.__name__)
+    assert failed, f"mutant {name} passed every pin"
