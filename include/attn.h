@@ -1,0 +1,166 @@
+/*
+ * attn.h -- C ABI of libattn.so: scaled-dot-product attention forward on NVIDIA B200 (sm_100a).
+ *
+ * Three operations, each a single asynchronous launch on the caller's CUDA stream:
+ *
+ *   attn_fwd         O = softmax(scale * Q K^T + mask) V, with per-row softmax max and sum.
+ *   attn_sparse_csr  the same softmax restricted to the entries of a CSR pattern (fp32).
+ *   attn_merge       merge of two partial attention results from their max/sum statistics.
+ *
+ * Conventions shared by every call
+ *   - All tensor pointers are DEVICE pointers owned by the caller. The library allocates no
+ *     device memory, keeps no reference to any argument after the call returns, and never
+ *     synchronises the stream (except attn_get_last_error, which says so).
+ *   - Tensors are dense and contiguous in the layout stated for each argument (row-major,
+ *     last index fastest).
+ *   - `stream` is a cudaStream_t passed as void*; NULL means the legacy default stream.
+ *   - Shape and argument errors are found on the host before anything is launched and are
+ *     returned as an attn_status; nothing is written in that case.
+ *   - Errors that depend on device data (cumulative lengths that are not monotone or do not
+ *     end at the total, CSR columns out of range, a row pointer that decreases, a pipeline
+ *     wait that timed out) are recorded in a per-device status word that
+ *     attn_get_last_error() reads. The kernel skips the offending unit of work (its outputs
+ *     are left as zeros where that is stated below) and never traps or aborts.
+ *   - Results are deterministic: the same inputs give bitwise-identical outputs (no atomics
+ *     take part in any result).
+ *   - Every function is thread-safe; calls on different streams may overlap.
+ *
+ * Softmax statistics (all calls): softmax_max is max_j s_ij, with s_ij = scale * q_i . k_j, in
+ * natural-log units; softmax_sum is sum_j exp(s_ij - softmax_max). A row that sees no key has
+ * output 0, softmax_max = -inf and softmax_sum = 0.
+ */
+#ifndef SDPA_B200_ATTN_H
+#define SDPA_B200_ATTN_H
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define ATTN_API __attribute__((visibility("default")))
+#else
+#define ATTN_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  ATTN_OK = 0,
+  ATTN_ERR_INVALID = 1,     /* bad shape, null pointer, inconsistent sizes              */
+  ATTN_ERR_UNSUPPORTED = 2, /* valid request this build does not run (e.g. bf16, D=96)  */
+  ATTN_ERR_CUDA = 3,        /* a CUDA runtime call failed (launch, device query)        */
+  ATTN_ERR_DATA = 4,        /* device-side: bad cumulative lengths or CSR indices       */
+  ATTN_ERR_TIMEOUT = 5      /* device-side: a pipeline wait exceeded its bound          */
+} attn_status;
+
+typedef enum { ATTN_BF16 = 0, ATTN_F32 = 1 } attn_dtype;
+
+typedef enum { ATTN_BHSD = 0, ATTN_TND = 1 } attn_layout;
+
+typedef enum {
+  ATTN_MASK_NONE = 0,
+  ATTN_MASK_CAUSAL_TOPLEFT = 1,    /* key j visible to query i iff j <= i                  */
+  ATTN_MASK_CAUSAL_BOTTOMRIGHT = 2 /* key j visible iff j <= i + Skv_b - Sq_b (per sequence) */
+} attn_mask;
+
+/*
+ * attn_fwd -- fused attention forward (FlashAttention-style tiling with an online softmax).
+ *
+ * Defined by: "paddle.nn.functional.sparse_attention" (Paddle 2.3 API doc), formula
+ * result = softmax(Q K^T / sqrt(d)) V, here with a general `scale`; "aclnnFlashAttentionVarLenScore"
+ * (CANN 8.5 API doc), 功能说明 (function) and 约束说明 (constraints): the packed TND layout,
+ * cumulative sequence lengths, GQA/MQA head ratios, lower-triangular masks and the shape limits.
+ *
+ * Layouts (layout = ATTN_BHSD):
+ *   q   [B, Nq,  Sq,  D]     k, v [B, Nkv, Skv, D]     out [B, Nq, Sq, D]
+ *   softmax_max, softmax_sum  float32 [B, Nq, Sq]
+ * Layouts (layout = ATTN_TND, packed variable-length batch):
+ *   q   [Tq, Nq, D]          k, v [Tkv, Nkv, D]        out [Tq, Nq, D]
+ *   softmax_max, softmax_sum  float32 [Tq, Nq]
+ *   Sq and Skv are the totals Tq and Tkv. cu_seqlens_q / cu_seqlens_kv are device int32
+ *   arrays of B entries holding cumulative lengths WITHOUT a leading zero: sequence b
+ *   occupies tokens [cu[b-1], cu[b]) with cu[-1] = 0, and cu[B-1] must equal the total.
+ *   Lengths [2,2,0,2,2] are passed as [2,4,4,6,8]; zero-length sequences are allowed.
+ * GQA/MQA: query head h reads key/value head h / (Nq / Nkv); Nq must be a multiple of Nkv.
+ * dtype: ATTN_BF16 (q, k, v, out bfloat16; fp32 accumulation; D = 64 or 128) or
+ *        ATTN_F32 (float32 throughout, CUDA-core FMA; 1 <= D <= 256).
+ * softmax_max / softmax_sum may both be NULL to skip the statistics.
+ * Limits (from the constraints): 1 <= Nq <= 256, D <= 768 (larger D is ATTN_ERR_INVALID;
+ * sizes this build does not run are ATTN_ERR_UNSUPPORTED), Tq, Tkv <= 1M tokens and
+ * B <= 2048 for TND. Empty problems (B = 0, Sq = 0 or a total of 0 tokens) return ATTN_OK
+ * without a launch. For ATTN_BF16, q, k, v and out must be 16-byte aligned.
+ * Data errors: cumulative lengths that decrease or do not end at the totals set ATTN_ERR_DATA
+ * in the status word; the affected outputs are not written.
+ */
+ATTN_API int attn_fwd(const void* q, const void* k, const void* v,
+             const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_kv,
+             int B, int Sq, int Skv, int Nq, int Nkv, int D,
+             float scale, int mask_mode, int dtype, int layout,
+             void* out, float* softmax_max, float* softmax_sum, void* stream);
+
+/*
+ * attn_sparse_csr -- CSR-sparse attention forward, float32.
+ *
+ * Defined by: "paddle.nn.functional.sparse_attention" (Paddle 2.3 API doc), formula and
+ * 参数 (parameters): for every (b, h, i), the softmax of q_i . k_j / sqrt(D) runs over the
+ * stored entries c of row i only, j = columns[b, h, c], and the output is the weighted sum of
+ * the v_j. The offset array is read as a row pointer (the page's worked example is one).
+ *
+ *   q, k, v, out   float32 [B, H, S, D]
+ *   csr_offset     int32 [B, H, S+1]: per (b, h) row pointer, offset[0] = 0, non-decreasing,
+ *                  offset[S] <= nnz_cap
+ *   csr_columns    int32 [B, H, nnz_cap]: column of each stored entry, 0 <= j < S; order
+ *                  within a row is free and a repeated column counts once per entry
+ * An empty row gives an output row of zeros. 1 <= D <= 256.
+ * Data errors: a column outside [0, S), or a row pointer that starts above 0, decreases or
+ * passes nnz_cap, set ATTN_ERR_DATA; the affected rows are written as zeros.
+ */
+ATTN_API int attn_sparse_csr(const float* q, const float* k, const float* v,
+                    const int32_t* csr_offset, const int32_t* csr_columns,
+                    int B, int H, int S, int D, int64_t nnz_cap,
+                    float* out, void* stream);
+
+/*
+ * attn_merge -- merge two partial attention results (the ring-attention update).
+ *
+ * Defined by: "npu_ring_attention_update" (MindSpeed op doc), 小算子等价计算逻辑 (equivalent
+ * small-op logic) and 前向接口 (forward interface). For every statistic lane (8 per row):
+ *     m = max(pm, cm); ps' = ps * exp(pm - m); cs' = cs * exp(cm - m); l = ps' + cs'
+ * and out = prev_out * (ps'/l) + cur_out * (cs'/l) with the lane-0 values of each row,
+ * computed in float32 and rounded once (to nearest even) to the output type.
+ *
+ * layout = ATTN_BHSD means the page's "SBH" layout:
+ *   prev_out, cur_out, out     [S, B, N*D] of `dtype` (ATTN_BF16 or ATTN_F32)
+ *   prev_/cur_/out_ max, sum   float32 [B, N, S, 8]
+ * layout = ATTN_TND is not run by this build (ATTN_ERR_UNSUPPORTED); actual_seq_qlen is
+ * reserved for it and must be NULL.
+ * A lane whose two maxima are both -inf (two empty partials) gives m = -inf, l = 0 and, on
+ * lane 0, an output row of zeros; where the lane-0 l is 0 the output scales are 0.
+ * Outputs may alias the prev_* inputs (in-place accumulation); no other overlap is allowed.
+ */
+ATTN_API int attn_merge(const void* prev_out, const float* prev_max, const float* prev_sum,
+               const void* cur_out, const float* cur_max, const float* cur_sum,
+               int S, int B, int N, int D, int dtype, int layout,
+               const int64_t* actual_seq_qlen,
+               void* out, float* out_max, float* out_sum, void* stream);
+
+/*
+ * attn_get_last_error -- read and clear the calling device's status word.
+ * Synchronises `stream`, then returns in *device_status the first device-side error
+ * (ATTN_ERR_DATA or ATTN_ERR_TIMEOUT) recorded by any launch on the current device since the
+ * previous read, or ATTN_OK. The return value is ATTN_OK, or ATTN_ERR_CUDA if the
+ * synchronisation or the read failed. The word is per device, shared by all streams.
+ */
+ATTN_API int attn_get_last_error(void* stream, int* device_status);
+
+/* Static description of a status code. */
+ATTN_API const char* attn_status_string(int status);
+
+/* ABI version of this header: (major << 16) | minor. */
+ATTN_API int attn_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SDPA_B200_ATTN_H */

@@ -1,0 +1,138 @@
+"""Python binding of libattn.so: scaled-dot-product attention forward on B200 (sm_100a).
+
+The three operations are the C-ABI calls declared in ``include/attn.h``; the functions here
+carry the same names and only marshal arguments (tensor data pointers, sizes, the current
+CUDA stream) into them. Every step of the computation runs in the library's CUDA kernels.
+There is no CPU path: if ``libattn.so`` is missing the first call raises.
+
+PyTorch is used for device memory and streams only: pass CUDA tensors (contiguous, in the
+layouts the header states) and preallocated outputs.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+from typing import Optional
+
+__all__ = [
+    "attn_fwd", "attn_sparse_csr", "attn_merge", "attn_get_last_error", "AttnError",
+    "ATTN_BF16", "ATTN_F32", "ATTN_BHSD", "ATTN_TND", "ATTN_MASK_NONE",
+    "ATTN_MASK_CAUSAL_TOPLEFT", "ATTN_MASK_CAUSAL_BOTTOMRIGHT", "lib_path", "load_library",
+]
+
+ATTN_OK, ATTN_ERR_INVALID, ATTN_ERR_UNSUPPORTED, ATTN_ERR_CUDA, ATTN_ERR_DATA, ATTN_ERR_TIMEOUT = range(6)
+ATTN_BF16, ATTN_F32 = 0, 1
+ATTN_BHSD, ATTN_TND = 0, 1
+ATTN_MASK_NONE, ATTN_MASK_CAUSAL_TOPLEFT, ATTN_MASK_CAUSAL_BOTTOMRIGHT = 0, 1, 2
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_lock = threading.Lock()
+_lib = None
+
+
+class AttnError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {_status_string(status)} (status {status})")
+
+
+def lib_path() -> str:
+    return os.path.join(_HERE, "libattn.so")
+
+
+def load_library():
+    """Load libattn.so (once). Raises if it has not been built."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        path = lib_path()
+        if not os.path.exists(path):
+            raise RuntimeError(f"{path} is missing: build it with "
+                               "`python -m scaled_dot_product_16_b200.build`")
+        lib = ctypes.CDLL(path)
+        P, I, I64, F = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float
+        lib.attn_fwd.argtypes = [P, P, P, P, P, I, I, I, I, I, I, F, I, I, I, P, P, P, P]
+        lib.attn_fwd.restype = I
+        lib.attn_sparse_csr.argtypes = [P, P, P, P, P, I, I, I, I, I64, P, P]
+        lib.attn_sparse_csr.restype = I
+        lib.attn_merge.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, P, P, P, P, P]
+        lib.attn_merge.restype = I
+        lib.attn_get_last_error.argtypes = [P, ctypes.POINTER(I)]
+        lib.attn_get_last_error.restype = I
+        lib.attn_status_string.argtypes = [I]
+        lib.attn_status_string.restype = ctypes.c_char_p
+        lib.attn_abi_version.argtypes = []
+        lib.attn_abi_version.restype = I
+        _lib = lib
+        return lib
+
+
+def _status_string(status: int) -> str:
+    try:
+        return load_library().attn_status_string(int(status)).decode()
+    except Exception:  # pragma: no cover - only for messages
+        return "unknown"
+
+
+def _ptr(x) -> Optional[int]:
+    """Data pointer of a tensor (or an int address, or None)."""
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    return int(x.data_ptr())
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        import torch
+        return int(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, int):
+        return stream
+    return int(stream.cuda_stream)
+
+
+def _check(status: int, what: str) -> None:
+    if status != ATTN_OK:
+        raise AttnError(status, what)
+
+
+def attn_fwd(q, k, v, *, cu_seqlens_q=None, cu_seqlens_kv=None, B: int, Sq: int, Skv: int,
+             Nq: int, Nkv: int, D: int, scale: float, mask_mode: int, dtype: int, layout: int,
+             out, softmax_max=None, softmax_sum=None, stream=None) -> None:
+    """Fused attention forward (see ``attn_fwd`` in include/attn.h for layouts and limits)."""
+    lib = load_library()
+    _check(lib.attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens_q), _ptr(cu_seqlens_kv),
+                        int(B), int(Sq), int(Skv), int(Nq), int(Nkv), int(D), float(scale),
+                        int(mask_mode), int(dtype), int(layout), _ptr(out), _ptr(softmax_max),
+                        _ptr(softmax_sum), _stream(stream)), "attn_fwd")
+
+
+def attn_sparse_csr(q, k, v, csr_offset, csr_columns, *, B: int, H: int, S: int, D: int,
+                    nnz_cap: int, out, stream=None) -> None:
+    """CSR-sparse attention forward in float32 (see ``attn_sparse_csr`` in include/attn.h)."""
+    lib = load_library()
+    _check(lib.attn_sparse_csr(_ptr(q), _ptr(k), _ptr(v), _ptr(csr_offset), _ptr(csr_columns),
+                               int(B), int(H), int(S), int(D), int(nnz_cap), _ptr(out),
+                               _stream(stream)), "attn_sparse_csr")
+
+
+def attn_merge(prev_out, prev_max, prev_sum, cur_out, cur_max, cur_sum, *, S: int, B: int, N: int,
+               D: int, dtype: int, out, out_max, out_sum, layout: int = ATTN_BHSD,
+               actual_seq_qlen=None, stream=None) -> None:
+    """Merge two partial attention results (see ``attn_merge`` in include/attn.h)."""
+    lib = load_library()
+    _check(lib.attn_merge(_ptr(prev_out), _ptr(prev_max), _ptr(prev_sum), _ptr(cur_out),
+                          _ptr(cur_max), _ptr(cur_sum), int(S), int(B), int(N), int(D), int(dtype),
+                          int(layout), _ptr(actual_seq_qlen), _ptr(out), _ptr(out_max),
+                          _ptr(out_sum), _stream(stream)), "attn_merge")
+
+
+def attn_get_last_error(stream=None) -> int:
+    """Synchronise the stream and return (and clear) the device status word."""
+    lib = load_library()
+    st = ctypes.c_int(0)
+    _check(lib.attn_get_last_error(_stream(stream), ctypes.byref(st)), "attn_get_last_error")
+    return int(st.value)

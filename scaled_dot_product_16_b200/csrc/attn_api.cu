@@ -1,0 +1,200 @@
+// attn_api.cu -- the C ABI of libattn.so: argument checks, the device status word, dispatch.
+//
+// Argument limits follow the constraints of "aclnnFlashAttentionVarLenScore" (CANN 8.5 API
+// doc, 约束说明): Nq/Nkv a nonzero integer with 1 <= Nq <= 256, head dim at most 768, at most
+// 1M packed tokens and 2K cumulative-length entries. The host never reads device data, so
+// data-dependent checks happen in the kernels, which record them in the status word below.
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <math.h>
+
+#include <mutex>
+
+#include "attn.h"
+#include "launch.h"
+
+namespace {
+
+// One status word per device; kernels record the first device-side error here.
+__device__ int g_status_word;
+
+constexpr int kMaxDevices = 64;
+std::mutex g_mu;
+int* g_status_ptr[kMaxDevices] = {};
+int g_num_sms[kMaxDevices] = {};
+
+// Device address of this device's status word and its SM count (looked up once per device).
+int device_state(int** status, int* num_sms) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return ATTN_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (g_status_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_status_word) != cudaSuccess) return ATTN_ERR_CUDA;
+    int sms = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return ATTN_ERR_CUDA;
+    g_status_ptr[dev] = static_cast<int*>(p);
+    g_num_sms[dev] = sms;
+  }
+  *status = g_status_ptr[dev];
+  *num_sms = g_num_sms[dev];
+  return ATTN_OK;
+}
+
+constexpr int64_t kMaxTokens = 1 << 20;  // "1M"
+constexpr int kMaxCu = 2048;             // "2K" cumulative-length entries
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace
+
+extern "C" {
+
+int attn_abi_version(void) { return (1 << 16) | 0; }
+
+const char* attn_status_string(int s) {
+  switch (s) {
+    case ATTN_OK: return "ok";
+    case ATTN_ERR_INVALID: return "invalid argument";
+    case ATTN_ERR_UNSUPPORTED: return "unsupported by this build";
+    case ATTN_ERR_CUDA: return "CUDA runtime error";
+    case ATTN_ERR_DATA: return "bad device data (cumulative lengths or CSR indices)";
+    case ATTN_ERR_TIMEOUT: return "pipeline wait timed out";
+    default: return "unknown status";
+  }
+}
+
+int attn_fwd(const void* q, const void* k, const void* v, const int32_t* cu_seqlens_q,
+             const int32_t* cu_seqlens_kv, int B, int Sq, int Skv, int Nq, int Nkv, int D,
+             float scale, int mask_mode, int dtype, int layout, void* out, float* softmax_max,
+             float* softmax_sum, void* stream) {
+  if (layout != ATTN_BHSD && layout != ATTN_TND) return ATTN_ERR_INVALID;
+  if (dtype != ATTN_BF16 && dtype != ATTN_F32) return ATTN_ERR_INVALID;
+  if (mask_mode < ATTN_MASK_NONE || mask_mode > ATTN_MASK_CAUSAL_BOTTOMRIGHT) return ATTN_ERR_INVALID;
+  if (B < 0 || Sq < 0 || Skv < 0) return ATTN_ERR_INVALID;
+  if (Nq < 1 || Nq > 256 || Nkv < 1 || Nq % Nkv != 0) return ATTN_ERR_INVALID;
+  if (D < 1 || D > 768) return ATTN_ERR_INVALID;
+  if (!(scale > 0.f) || scale == INFINITY) return ATTN_ERR_INVALID;  // finite and positive
+  if ((softmax_max == nullptr) != (softmax_sum == nullptr)) return ATTN_ERR_INVALID;
+  if (layout == ATTN_TND) {
+    if (B > kMaxCu || Sq > kMaxTokens || Skv > kMaxTokens) return ATTN_ERR_INVALID;
+    if (B > 0 && (cu_seqlens_q == nullptr || cu_seqlens_kv == nullptr)) return ATTN_ERR_INVALID;
+  } else if (cu_seqlens_q != nullptr || cu_seqlens_kv != nullptr) {
+    return ATTN_ERR_INVALID;
+  }
+  const bool empty_q = B == 0 || Sq == 0;
+  if (empty_q) return ATTN_OK;
+  if (q == nullptr || out == nullptr) return ATTN_ERR_INVALID;
+  if (Skv > 0 && (k == nullptr || v == nullptr)) return ATTN_ERR_INVALID;
+  if (dtype == ATTN_F32 && D > 256) return ATTN_ERR_UNSUPPORTED;
+  if (dtype == ATTN_BF16) {
+    if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return ATTN_ERR_INVALID;
+  }
+
+  sdpa::FwdArgs a{};
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.cu_q = cu_seqlens_q;
+  a.cu_kv = cu_seqlens_kv;
+  a.B = B;
+  a.Sq = Sq;
+  a.Skv = Skv;
+  a.Nq = Nq;
+  a.Nkv = Nkv;
+  a.D = D;
+  a.scale = scale;
+  a.mask_mode = mask_mode;
+  a.layout = layout;
+  a.out = out;
+  a.smax = softmax_max;
+  a.ssum = softmax_sum;
+  int rc = device_state(&a.status, &a.num_sms);
+  if (rc != ATTN_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const cudaError_t e = dtype == ATTN_F32 ? sdpa::launch_fwd_f32(a, st) : sdpa::launch_fwd_bf16(a, st);
+  return e == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+int attn_sparse_csr(const float* q, const float* k, const float* v, const int32_t* csr_offset,
+                    const int32_t* csr_columns, int B, int H, int S, int D, int64_t nnz_cap,
+                    float* out, void* stream) {
+  if (B < 0 || H < 0 || S < 0 || nnz_cap < 0) return ATTN_ERR_INVALID;
+  if (D < 1) return ATTN_ERR_INVALID;
+  if ((int64_t)B * H * S == 0) return ATTN_OK;
+  if (q == nullptr || k == nullptr || v == nullptr || out == nullptr || csr_offset == nullptr)
+    return ATTN_ERR_INVALID;
+  if (nnz_cap > 0 && csr_columns == nullptr) return ATTN_ERR_INVALID;
+  if (D > 256) return ATTN_ERR_UNSUPPORTED;
+  sdpa::CsrArgs a{};
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.offset = csr_offset;
+  a.columns = csr_columns;
+  a.B = B;
+  a.H = H;
+  a.S = S;
+  a.D = D;
+  a.nnz_cap = nnz_cap;
+  a.out = out;
+  int sms = 0;
+  int rc = device_state(&a.status, &sms);
+  if (rc != ATTN_OK) return rc;
+  const cudaError_t e = sdpa::launch_sparse_csr(a, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+int attn_merge(const void* prev_out, const float* prev_max, const float* prev_sum,
+               const void* cur_out, const float* cur_max, const float* cur_sum, int S, int B,
+               int N, int D, int dtype, int layout, const int64_t* actual_seq_qlen, void* out,
+               float* out_max, float* out_sum, void* stream) {
+  if (dtype != ATTN_BF16 && dtype != ATTN_F32) return ATTN_ERR_INVALID;
+  if (layout != ATTN_BHSD && layout != ATTN_TND) return ATTN_ERR_INVALID;
+  if (S < 0 || B < 0 || N < 1 || D < 1) return ATTN_ERR_INVALID;
+  if (layout == ATTN_TND) return ATTN_ERR_UNSUPPORTED;
+  if (actual_seq_qlen != nullptr) return ATTN_ERR_INVALID;
+  if ((int64_t)S * B == 0) return ATTN_OK;
+  if ((int64_t)B * N > 0x7fffffffLL || S > 65535LL * 32) return ATTN_ERR_UNSUPPORTED;
+  if (!prev_out || !prev_max || !prev_sum || !cur_out || !cur_max || !cur_sum || !out ||
+      !out_max || !out_sum)
+    return ATTN_ERR_INVALID;
+  sdpa::MergeArgs a{};
+  a.prev_out = prev_out;
+  a.prev_max = prev_max;
+  a.prev_sum = prev_sum;
+  a.cur_out = cur_out;
+  a.cur_max = cur_max;
+  a.cur_sum = cur_sum;
+  a.S = S;
+  a.B = B;
+  a.N = N;
+  a.D = D;
+  a.dtype = dtype;
+  a.out = out;
+  a.out_max = out_max;
+  a.out_sum = out_sum;
+  const cudaError_t e = sdpa::launch_merge(a, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+int attn_get_last_error(void* stream, int* device_status) {
+  if (device_status == nullptr) return ATTN_ERR_INVALID;
+  int* word = nullptr;
+  int sms = 0;
+  int rc = device_state(&word, &sms);
+  if (rc != ATTN_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int host = 0;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return ATTN_ERR_CUDA;
+  if (cudaMemcpy(&host, word, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return ATTN_ERR_CUDA;
+  if (cudaMemset(word, 0, sizeof(int)) != cudaSuccess) return ATTN_ERR_CUDA;
+  *device_status = host;
+  return ATTN_OK;
+}
+
+}  // extern "C"

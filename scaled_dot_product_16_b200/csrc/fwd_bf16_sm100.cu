@@ -1,0 +1,545 @@
+// fwd_bf16_sm100.cu -- fused attention forward for bf16 on B200 (sm_100a).
+//
+// O = softmax(scale * Q K^T + mask) V with per-row softmax max / sum, for dense BHSD or packed
+// TND batches with GQA/MQA head ratios and causal masks ("aclnnFlashAttentionVarLenScore",
+// CANN 8.5 API doc, 功能说明 and 约束说明; the formula of "paddle.nn.functional.sparse_attention").
+// The pages name the FlashAttention algorithm (tiles of Q against streamed K/V tiles with an
+// online softmax) but give no kernel; this is a from-scratch sm_100a design:
+//
+//   * one block owns 256 query rows of one (sequence, head), as two 128-row tiles Q0 and Q1;
+//   * K and V tiles (128 keys x D) stream through a ring of shared-memory stages, loaded by
+//     TMA with 128-byte swizzle (one issuing thread, no multicast);
+//   * one thread issues every tcgen05.mma: S_q = Q_q K_j^T (both operands in shared memory,
+//     fp32 accumulator in tensor memory) and O_q += P_q V_j (P read from tensor memory);
+//   * two softmax warpgroups (one per Q tile, one thread per row = one TMEM lane) read S with
+//     tcgen05.ld, apply the mask, keep the running max / sum, write P = exp2(...) as bf16 back
+//     into the first half of S's TMEM columns, and at the end normalise O and store it;
+//   * while one warpgroup is in its softmax, the tensor core runs the other tile's MMAs;
+//   * the running max is updated lazily: only when a row's maximum grows by more than 2^8 are
+//     O and the sum rescaled (exact, because the same max is used for P, the sum and O);
+//   * key tiles entirely above the causal diagonal are never loaded or multiplied, the
+//     diagonal and ragged tiles are masked element by element, rows past a sequence's end are
+//     never stored, and zero-length sequences produce no work.
+//
+// Roles (320 threads): warps 0-3 softmax Q0, warps 4-7 softmax Q1, warp 8 MMA issue,
+// warp 9 TMA producer. TMEM: S0 [0,128) S1 [128,256) O0 [256,256+D) O1 [256+D,256+2D).
+//
+// Every mbarrier wait is bounded in time: if a wait runs out the block records
+// ATTN_ERR_TIMEOUT, stops issuing work, drains what it started and frees its TMEM.
+#include <cuda.h>
+#include <math.h>
+
+#include <mutex>
+
+#include "common.cuh"
+#include "launch.h"
+#include "sm100.cuh"
+
+namespace sdpa {
+namespace {
+
+using namespace sm100;
+
+constexpr int kBM = 128;          // rows per Q tile (= TMEM lanes)
+constexpr int kBN = 128;          // keys per K/V tile
+constexpr int kRowsPerBlock = 2 * kBM;
+constexpr int kThreads = 320;
+constexpr int kMmaWarp = 8;
+constexpr int kTmaWarp = 9;
+constexpr uint32_t kTmemCols = 512;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale when the max grows by > 2^8
+constexpr uint64_t kWaitLimitNs = 200ull * 1000ull * 1000ull;  // 200 ms per barrier wait
+
+template <int HD>
+struct Cfg {
+  static constexpr int kBoxes = HD / 64;                 // 64-element (128-byte) TMA boxes
+  static constexpr int kTileBytes = kBM * HD * 2;        // one Q, K or V tile
+  static constexpr int kStages = HD == 128 ? 4 : 6;      // K/V ring depth
+  static constexpr int kQOff = 0;
+  static constexpr int kKVOff = 2 * kTileBytes;
+  static constexpr int kBarOff = kKVOff + kStages * kTileBytes;
+  static constexpr int kSmemBytes = kBarOff + 256 + 1024;  // barriers + 1 KB for alignment
+  static constexpr uint32_t kIdescQK = idesc_bf16_f32(kBM, kBN, 0, 0);
+  static constexpr uint32_t kIdescPV = idesc_bf16_f32(kBM, HD, 0, 1);
+};
+
+struct Barriers {
+  uint64_t kv_full[8];
+  uint64_t kv_empty[8];
+  uint64_t q_full;
+  uint64_t s_full[2];
+  uint64_t p_ready[2];
+  uint64_t o_done[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort;
+};
+
+// Bounded wait on an mbarrier phase. Returns false (after recording a timeout, or when another
+// role of this block already gave up) instead of waiting forever.
+// With heed_abort = false (used when draining work already issued) only the time bound applies.
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort,
+                                         int* status, bool heed_abort = true) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 255u) == 0) {
+      if (heed_abort && *abort) return false;
+      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+        *abort = 1;
+        report(status, ATTN_ERR_TIMEOUT);
+        return false;
+      }
+    }
+  }
+}
+
+struct Work {
+  int b, h, g;      // sequence, query head, key/value head
+  int q0, sq;       // first query token and query length of the sequence
+  int k0, sk;       // same for keys
+  int row0;         // first row (within the sequence) of this block's 256 rows
+};
+
+template <int HD>
+__global__ void __launch_bounds__(kThreads, 1)
+    fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v, FwdArgs a, int units_per_seq,
+                    float scale_log2) {
+  using C = Cfg<HD>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Barriers* bars = reinterpret_cast<Barriers*>(smem + C::kBarOff);
+  __shared__ int s_work[4];
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  // ---- work unit: (sequence b, 256-row block) of query head h -----------------------------
+  // Block ids run head-fastest; within a head the heaviest (last) row blocks come first.
+  const int h = (int)(blockIdx.x % (unsigned)a.Nq);
+  const int y = (int)(blockIdx.x / (unsigned)a.Nq);
+  if (warp == 0) {
+    int b = 0, u = 0, ok = 1;
+    if (a.layout == ATTN_BHSD) {
+      const int level = y / a.B;  // 0 = last row block of every sequence
+      b = y - level * a.B;
+      u = units_per_seq - 1 - level;
+      ok = u >= 0;
+    } else {
+      bool bad;
+      int t;
+      ok = warp_find_tile(a.cu_q, a.B, a.Sq, kRowsPerBlock, y, &b, &t, a.status, &bad);
+      if (ok) {
+        int qs, ql;
+        seq_span(a.cu_q, b, &qs, &ql);
+        u = (ql + kRowsPerBlock - 1) / kRowsPerBlock - 1 - t;
+      } else if (!bad && h == 0) {
+        int sb, st;
+        bool bad2;  // a block past the last unit validates the key-side lengths
+        warp_find_tile(a.cu_kv, a.B, a.Skv, 1 << 30, 1 << 30, &sb, &st, a.status, &bad2);
+      }
+    }
+    if (lane == 0) {
+      s_work[0] = ok;
+      s_work[1] = b;
+      s_work[2] = u;
+    }
+  }
+  __syncthreads();
+  if (!s_work[0]) return;
+
+  Work w;
+  w.b = s_work[1];
+  w.h = h;
+  w.g = h / (a.Nq / a.Nkv);
+  w.row0 = s_work[2] * kRowsPerBlock;
+  if (a.layout == ATTN_BHSD) {
+    w.q0 = 0;
+    w.sq = a.Sq;
+    w.k0 = 0;
+    w.sk = a.Skv;
+  } else {
+    seq_span(a.cu_q, w.b, &w.q0, &w.sq);
+    seq_span(a.cu_kv, w.b, &w.k0, &w.sk);
+    if (w.k0 < 0 || w.sk < 0 || w.k0 + w.sk > a.Skv) {
+      if (threadIdx.x == 0) report(a.status, ATTN_ERR_DATA);
+      return;
+    }
+  }
+  // rows and key tiles of each Q tile
+  const int rows0 = min(kBM, w.sq - w.row0);
+  const int rows1 = min(kBM, w.sq - w.row0 - kBM);  // <= 0: no second tile
+  const bool has1 = rows1 > 0;
+  const int kv_end0 = visible_end(a.mask_mode, w.row0 + rows0 - 1, w.sq, w.sk);
+  const int kv_end1 = has1 ? visible_end(a.mask_mode, w.row0 + kBM + rows1 - 1, w.sq, w.sk) : 0;
+  const int n0 = (kv_end0 + kBN - 1) / kBN;
+  const int n1 = has1 ? (kv_end1 + kBN - 1) / kBN : n0;  // tiles loaded (n1 >= n0)
+
+  const uint32_t bar_base = smem_u32(bars);
+  auto bar_addr = [&](const uint64_t* p) { return smem_u32(p); };
+  (void)bar_base;
+
+  // ---- setup: barriers, TMEM -------------------------------------------------------------
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(bar_addr(&bars->kv_full[s]), 1);
+      mbar_init(bar_addr(&bars->kv_empty[s]), 1);
+    }
+    mbar_init(bar_addr(&bars->q_full), 1);
+    mbar_init(bar_addr(&bars->drain), 1);
+    for (int q = 0; q < 2; ++q) {
+      mbar_init(bar_addr(&bars->s_full[q]), 1);
+      mbar_init(bar_addr(&bars->p_ready[q]), kBM);
+      mbar_init(bar_addr(&bars->o_done[q]), 1);
+    }
+    bars->abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(&bars->tmem_base), kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+  volatile int* abort = &bars->abort;
+
+  const uint32_t sQ = smem_u32(smem + C::kQOff);
+  const uint32_t sKV = smem_u32(smem + C::kKVOff);
+
+  if (warp == kTmaWarp) {
+    // =============================== TMA producer =======================================
+    if (lane == 0) {
+      const bool bhsd = a.layout == ATTN_BHSD;
+      const int qhead = bhsd ? w.b * a.Nq + w.h : w.h;
+      const int khead = bhsd ? w.b * a.Nkv + w.g : w.g;
+      auto load_tile = [&](const CUtensorMap* map, uint32_t dst, uint32_t bar, int tok, int head) {
+        for (int x = 0; x < C::kBoxes; ++x) {
+          if (bhsd)
+            tma_load_3d(dst + x * (kBM * 128), map, bar, x * 64, tok, head);
+          else
+            tma_load_3d(dst + x * (kBM * 128), map, bar, x * 64, head, tok);
+        }
+      };
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      const uint32_t qbar = bar_addr(&bars->q_full);
+      mbar_arrive_expect_tx(qbar, (has1 ? 2 : 1) * C::kTileBytes);
+      load_tile(&tm_q, sQ, qbar, w.q0 + w.row0, qhead);
+      if (has1) load_tile(&tm_q, sQ + C::kTileBytes, qbar, w.q0 + w.row0 + kBM, qhead);
+      // K0, V0, K1, V1, ... through the ring
+      int issued = 0;
+      for (int i = 0; i < 2 * n1; ++i, ++issued) {
+        const int s = i % C::kStages, r = i / C::kStages;
+        if (r > 0 && !wait_bar(bar_addr(&bars->kv_empty[s]), (r - 1) & 1, abort, a.status)) break;
+        const uint32_t fb = bar_addr(&bars->kv_full[s]);
+        mbar_arrive_expect_tx(fb, C::kTileBytes);
+        const int j = i >> 1;
+        load_tile((i & 1) ? &tm_v : &tm_k, sKV + s * C::kTileBytes, fb, w.k0 + j * kBN, khead);
+      }
+      // drain: every stage this thread filled must have landed before the block exits
+      for (int i = max(0, issued - C::kStages); i < issued; ++i) {
+        const int s = i % C::kStages, r = i / C::kStages;
+        wait_bar(bar_addr(&bars->kv_full[s]), r & 1, abort, a.status, false);
+      }
+      wait_bar(bar_addr(&bars->q_full), 0, abort, a.status, false);
+    }
+  } else if (warp == kMmaWarp) {
+    // =============================== MMA issue ==========================================
+    if (lane == 0) {
+      const uint32_t S0 = tmem, S1 = tmem + 128, O0 = tmem + 256, O1 = tmem + 256 + HD;
+      auto full = [&](int i) {
+        return wait_bar(bar_addr(&bars->kv_full[i % C::kStages]), (i / C::kStages) & 1, abort,
+                        a.status);
+      };
+      auto release = [&](int i) { mma_commit(bar_addr(&bars->kv_empty[i % C::kStages])); };
+      auto kv_smem = [&](int i) { return sKV + (i % C::kStages) * C::kTileBytes; };
+      auto issue_qk = [&](uint32_t d, uint32_t q_smem, uint32_t k_smem) {
+#pragma unroll
+        for (int kk = 0; kk < HD / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * (kBM * 128) + (kk & 3) * 32;
+          mma_ss(d, smem_desc_sw128(q_smem + off, 16, 1024), smem_desc_sw128(k_smem + off, 16, 1024),
+                 C::kIdescQK, kk > 0);
+        }
+      };
+      auto issue_pv = [&](uint32_t d, uint32_t p_tmem, uint32_t v_smem, bool acc) {
+#pragma unroll
+        for (int kk = 0; kk < kBN / 16; ++kk) {
+          mma_ts(d, p_tmem + kk * 8, smem_desc_sw128(v_smem + kk * 2048, kBN * 128, 1024),
+                 C::kIdescPV, (acc || kk > 0) ? 1u : 0u);
+        }
+      };
+      bool ok = true;
+      if (n1 > 0) {
+        ok = wait_bar(bar_addr(&bars->q_full), 0, abort, a.status);
+        if (ok) ok = full(0);
+      }
+      if (ok && n1 > 0) {
+        tc_fence_after();
+        if (n0 > 0) {
+          issue_qk(S0, sQ, kv_smem(0));
+          mma_commit(bar_addr(&bars->s_full[0]));
+        }
+        if (has1) {
+          issue_qk(S1, sQ + C::kTileBytes, kv_smem(0));
+          mma_commit(bar_addr(&bars->s_full[1]));
+        }
+        release(0);
+      }
+      for (int j = 0; ok && j < n1; ++j) {
+        const int iv = 2 * j + 1, ik = 2 * j + 2;
+        if (!(ok = full(iv))) break;
+        tc_fence_after();
+        if (j < n0) {
+          if (!(ok = wait_bar(bar_addr(&bars->p_ready[0]), j & 1, abort, a.status))) break;
+          tc_fence_after();
+          issue_pv(O0, S0, kv_smem(iv), j > 0);
+          if (j == n0 - 1) mma_commit(bar_addr(&bars->o_done[0]));
+        }
+        const bool next = j + 1 < n1;
+        if (next) {
+          if (!(ok = full(ik))) break;
+          tc_fence_after();
+          if (j + 1 < n0) {
+            issue_qk(S0, sQ, kv_smem(ik));
+            mma_commit(bar_addr(&bars->s_full[0]));
+          }
+        }
+        if (has1) {
+          if (!(ok = wait_bar(bar_addr(&bars->p_ready[1]), j & 1, abort, a.status))) break;
+          tc_fence_after();
+          issue_pv(O1, S1, kv_smem(iv), j > 0);
+          if (j == n1 - 1) mma_commit(bar_addr(&bars->o_done[1]));
+        }
+        release(iv);
+        if (next) {
+          if (has1) {
+            issue_qk(S1, sQ + C::kTileBytes, kv_smem(ik));
+            mma_commit(bar_addr(&bars->s_full[1]));
+          }
+          release(ik);
+        }
+      }
+      if (!ok) *abort = 1;
+      // every MMA and commit issued above must have completed before TMEM is freed
+      mma_commit(bar_addr(&bars->drain));
+      wait_bar(bar_addr(&bars->drain), 0, abort, a.status, false);
+    }
+  } else {
+    // =============================== softmax + epilogue ================================
+    const int q = warp >> 2;                       // Q tile of this warpgroup
+    const int quarter = warp & 3;                  // TMEM lane quarter of this warp
+    const int r = quarter * 32 + lane;             // row within the Q tile = TMEM lane
+    const int n = q == 0 ? n0 : (has1 ? n1 : 0);
+    const int rows = q == 0 ? rows0 : rows1;
+    const int i = w.row0 + q * kBM + r;            // row within the sequence
+    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    const uint32_t S = tmem + lane_off + q * 128;
+    const uint32_t O = tmem + lane_off + 256 + q * HD;
+    const int lim = i < w.sq ? visible_end(a.mask_mode, i, w.sq, w.sk) : w.sk;
+
+    float m = -INFINITY;        // running max used for P (log2 units, lazily updated)
+    float mraw = -INFINITY;     // true max of the raw scores q.k
+    float l = 0.f;
+    bool ok = true;
+    if (q == 0 || has1) {
+      for (int j = 0; j < n; ++j) {
+        ok = __all_sync(0xffffffffu, wait_bar(bar_addr(&bars->s_full[q]), j & 1, abort, a.status));
+        if (!ok) break;
+        tc_fence_after();
+        float s[4][32];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_ld32f(S + c * 32, s[c]);
+        tmem_wait_ld();
+        const int kbase = j * kBN;
+        if (kbase + kBN > lim) {
+#pragma unroll
+          for (int c = 0; c < kBN; ++c)
+            if (kbase + c >= lim) s[c >> 5][c & 31] = -INFINITY;
+        }
+        float mx[8];
+#pragma unroll
+        for (int x = 0; x < 8; ++x) mx[x] = s[x >> 1][(x & 1) * 16];
+#pragma unroll
+        for (int c = 0; c < kBN; ++c)
+          if ((c & 15) != 0) mx[c >> 4] = fmaxf(mx[c >> 4], s[c >> 5][c & 31]);
+        const float tmax = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                                 fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+        mraw = fmaxf(mraw, tmax);
+        const float tmax2 = tmax * scale_log2;
+        bool bump = tmax2 > m + kRescaleThreshold;  // also true for the first finite max
+        float corr = 1.f;
+        if (bump) {
+          corr = (m == -INFINITY) ? 0.f : ex2(m - tmax2);
+          m = tmax2;
+          l *= corr;
+        }
+        const float muse = m == -INFINITY ? 0.f : m;
+        float rs[4] = {0.f, 0.f, 0.f, 0.f};
+        uint32_t pk[2][32];
+#pragma unroll
+        for (int c = 0; c < kBN; c += 2) {
+          const float p0 = ex2(fmaf(s[c >> 5][c & 31], scale_log2, -muse));
+          const float p1 = ex2(fmaf(s[c >> 5][(c + 1) & 31], scale_log2, -muse));
+          rs[(c >> 1) & 3] += p0 + p1;
+          pk[c >> 6][(c >> 1) & 31] = pack_bf16x2(p0, p1);
+        }
+        l += (rs[0] + rs[1]) + (rs[2] + rs[3]);
+        // rescale O (complete up to tile j-1: the S_j commit covers every earlier MMA)
+        if (__any_sync(0xffffffffu, bump && j > 0)) {
+          const float f = (bump && j > 0) ? corr : 1.f;
+#pragma unroll
+          for (int c = 0; c < HD / 32; ++c) {
+            uint32_t o[32];
+            tmem_ld32(O + c * 32, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int x = 0; x < 32; ++x) o[x] = __float_as_uint(__uint_as_float(o[x]) * f);
+            tmem_st32(O + c * 32, o);
+          }
+        }
+        tmem_st32(S, pk[0]);
+        tmem_st32(S + 32, pk[1]);
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar_addr(&bars->p_ready[q]));
+      }
+    }
+    // ---- epilogue: O / l -> bf16, statistics ------------------------------------------------
+    const bool have_o = ok && n > 0 && (q == 0 || has1);
+    if (have_o) ok = __all_sync(0xffffffffu, wait_bar(bar_addr(&bars->o_done[q]), 0, abort, a.status));
+    tc_fence_after();
+    if (q == 0 || has1) {
+      const bool store = r < rows;
+      const bool bhsd = a.layout == ATTN_BHSD;
+      __nv_bfloat16* out = static_cast<__nv_bfloat16*>(a.out);
+      const int64_t orow = bhsd ? (((int64_t)w.b * a.Nq + w.h) * a.Sq + i) * HD
+                                : ((int64_t)(w.q0 + i) * a.Nq + w.h) * HD;
+      const float inv = (l > 0.f && ok) ? 1.f / l : 0.f;
+#pragma unroll
+      for (int c = 0; c < HD / 32; ++c) {
+        uint32_t o[32];
+        if (have_o && ok) {
+          tmem_ld32(O + c * 32, o);
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int x = 0; x < 32; ++x) o[x] = 0u;
+        }
+        if (store) {
+          uint32_t pkd[16];
+#pragma unroll
+          for (int x = 0; x < 16; ++x)
+            pkd[x] = pack_bf16x2(inv == 0.f ? 0.f : __uint_as_float(o[2 * x]) * inv,
+                                 inv == 0.f ? 0.f : __uint_as_float(o[2 * x + 1]) * inv);
+          uint4* dst = reinterpret_cast<uint4*>(out + orow + c * 32);
+#pragma unroll
+          for (int x = 0; x < 4; ++x)
+            dst[x] = make_uint4(pkd[4 * x], pkd[4 * x + 1], pkd[4 * x + 2], pkd[4 * x + 3]);
+        }
+      }
+      if (store && a.smax != nullptr) {
+        const int64_t so = bhsd ? ((int64_t)w.b * a.Nq + w.h) * a.Sq + i
+                                : (int64_t)(w.q0 + i) * a.Nq + w.h;
+        const bool any = l > 0.f && ok;
+        a.smax[so] = any ? mraw * a.scale : -INFINITY;
+        a.ssum[so] = any ? l * ex2(m - mraw * scale_log2) : 0.f;
+      }
+    }
+  }
+
+  // ---- teardown ----------------------------------------------------------------------------
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// ------------------------------------------------------------------------------------------------
+// host side: tensor maps and launch
+// ------------------------------------------------------------------------------------------------
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 3-D map over a bf16 tensor viewed as (D, dim1, dim2), box (64, box1, box2), 128-byte swizzle.
+bool make_map(CUtensorMap* m, const void* base, uint64_t D, uint64_t dim1, uint64_t dim2,
+              uint64_t stride1_bytes, uint64_t stride2_bytes, uint32_t box1, uint32_t box2) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[3] = {D, dim1, dim2};
+  const cuuint64_t strides[2] = {stride1_bytes, stride2_bytes};
+  const cuuint32_t box[3] = {64, box1, box2};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int HD>
+cudaError_t launch_hd(const FwdArgs& a, cudaStream_t st) {
+  using C = Cfg<HD>;
+  CUtensorMap tq, tk, tv;
+  const uint64_t D = HD;
+  bool ok;
+  if (a.layout == ATTN_BHSD) {
+    // (d, s, b*h): rows of a head are contiguous
+    ok = make_map(&tq, a.q, D, a.Sq, (uint64_t)a.B * a.Nq, D * 2, (uint64_t)a.Sq * D * 2, kBM, 1) &&
+         make_map(&tk, a.k, D, a.Skv, (uint64_t)a.B * a.Nkv, D * 2, (uint64_t)a.Skv * D * 2, kBN, 1) &&
+         make_map(&tv, a.v, D, a.Skv, (uint64_t)a.B * a.Nkv, D * 2, (uint64_t)a.Skv * D * 2, kBN, 1);
+  } else {
+    // (d, head, token): a tile is 128 tokens of one head
+    const uint64_t tq_rows = a.Sq > 0 ? a.Sq : 1, tk_rows = a.Skv > 0 ? a.Skv : 1;
+    ok = make_map(&tq, a.q, D, a.Nq, tq_rows, D * 2, (uint64_t)a.Nq * D * 2, 1, kBM) &&
+         make_map(&tk, a.k, D, a.Nkv, tk_rows, D * 2, (uint64_t)a.Nkv * D * 2, 1, kBN) &&
+         make_map(&tv, a.v, D, a.Nkv, tk_rows, D * 2, (uint64_t)a.Nkv * D * 2, 1, kBN);
+  }
+  if (!ok) return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(fwd_bf16_kernel<HD>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+  if (e != cudaSuccess) return e;
+  int units_per_seq = 0;
+  int64_t units;
+  if (a.layout == ATTN_BHSD) {
+    units_per_seq = (a.Sq + kRowsPerBlock - 1) / kRowsPerBlock;
+    units = (int64_t)a.B * units_per_seq;
+  } else {
+    units = (a.Sq + kRowsPerBlock - 1) / kRowsPerBlock + a.B;
+  }
+  const int64_t blocks = units * a.Nq;
+  if (blocks <= 0) return cudaSuccess;
+  if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+  const float scale_log2 = a.scale * 1.4426950408889634f;
+  fwd_bf16_kernel<HD><<<(unsigned)blocks, kThreads, C::kSmemBytes, st>>>(tq, tk, tv, a,
+                                                                           units_per_seq, scale_log2);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_fwd_bf16(const FwdArgs& a, cudaStream_t st) {
+  if (a.D == 128) return launch_hd<128>(a, st);
+  return launch_hd<64>(a, st);
+}
+
+}  // namespace sdpa

@@ -1,0 +1,55 @@
+// launch.h -- internal launch entry points of libattn.so (not part of the C ABI).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace sdpa {
+
+struct FwdArgs {
+  const void* q;
+  const void* k;
+  const void* v;
+  const int32_t* cu_q;   // TND only
+  const int32_t* cu_kv;  // TND only
+  int B, Sq, Skv, Nq, Nkv, D;
+  float scale;
+  int mask_mode, layout;
+  void* out;
+  float* smax;  // may be null (with ssum)
+  float* ssum;
+  int* status;  // device status word
+  int num_sms;
+};
+
+struct CsrArgs {
+  const float* q;
+  const float* k;
+  const float* v;
+  const int32_t* offset;
+  const int32_t* columns;
+  int B, H, S, D;
+  int64_t nnz_cap;
+  float* out;
+  int* status;
+};
+
+struct MergeArgs {
+  const void* prev_out;
+  const float* prev_max;
+  const float* prev_sum;
+  const void* cur_out;
+  const float* cur_max;
+  const float* cur_sum;
+  int S, B, N, D, dtype;
+  void* out;
+  float* out_max;
+  float* out_sum;
+};
+
+cudaError_t launch_merge(const MergeArgs& a, cudaStream_t st);
+cudaError_t launch_fwd_f32(const FwdArgs& a, cudaStream_t st);
+cudaError_t launch_fwd_bf16(const FwdArgs& a, cudaStream_t st);
+cudaError_t launch_sparse_csr(const CsrArgs& a, cudaStream_t st);
+
+}  // namespace sdpa

@@ -1,0 +1,189 @@
+// merge.cu -- merge of two partial attention results from their softmax statistics.
+//
+// "npu_ring_attention_update" (MindSpeed op doc), 小算子等价计算逻辑: per statistic lane,
+//   m = max(pm, cm), ps' = ps * exp(pm - m), cs' = cs * exp(cm - m), l = ps' + cs',
+// and out = prev * (ps'_0 / l_0) + cur * (cs'_0 / l_0) with lane 0 of each (b, n, s) row.
+//
+// SBH layout: outputs [S, B, N*D]; statistics [B, N, S, 8] fp32.
+//
+// The kernel is HBM-bound (about 1 GB moved per call at S=8192, B=4, N=32, D=128), so the
+// design is about access shape only:
+//   * one block owns ROWS consecutive s of one (b, n): its statistics are ROWS*8 contiguous
+//     floats per array (one coalesced load per thread), and every output row is D
+//     contiguous elements (D*2 = 256 B for bf16, D = 128);
+//   * every thread issues all of its 16-byte loads of the block before any math, so a
+//     block keeps ROWS*D*2*sizeof(T) bytes in flight;
+//   * no shared-memory traffic except the ROWS pairs of lane-0 scales.
+#include "common.cuh"
+#include "launch.h"
+
+namespace sdpa {
+namespace {
+
+constexpr int kRows = 32;     // s rows per block
+constexpr int kThreads = 256;
+
+template <typename T>
+struct Vec16;
+template <>
+struct Vec16<__nv_bfloat16> {
+  static constexpr int n = 8;
+};
+template <>
+struct Vec16<float> {
+  static constexpr int n = 4;
+};
+
+__device__ __forceinline__ void unpack(const uint4& u, float* f, __nv_bfloat16*) {
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 t = __bfloat1622float2(h[i]);
+    f[2 * i] = t.x;
+    f[2 * i + 1] = t.y;
+  }
+}
+__device__ __forceinline__ void unpack(const uint4& u, float* f, float*) {
+  f[0] = __uint_as_float(u.x);
+  f[1] = __uint_as_float(u.y);
+  f[2] = __uint_as_float(u.z);
+  f[3] = __uint_as_float(u.w);
+}
+__device__ __forceinline__ uint4 pack(const float* f, __nv_bfloat16*) {
+  uint4 u;
+  __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&u);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(f[2 * i], f[2 * i + 1]);
+  return u;
+}
+__device__ __forceinline__ uint4 pack(const float* f, float*) {
+  return make_uint4(__float_as_uint(f[0]), __float_as_uint(f[1]), __float_as_uint(f[2]),
+                    __float_as_uint(f[3]));
+}
+
+__device__ __forceinline__ float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
+__device__ __forceinline__ float to_f(float x) { return x; }
+__device__ __forceinline__ void from_f(float x, __nv_bfloat16* p) { *p = __float2bfloat16_rn(x); }
+__device__ __forceinline__ void from_f(float x, float* p) { *p = x; }
+
+// Lane-wise statistics update; returns the lane's scaled partial sums.
+__device__ __forceinline__ void merge_lane(float pm, float ps, float cm, float cs, float* m,
+                                           float* ps2, float* cs2) {
+  const float mx = fmaxf(pm, cm);
+  if (mx == -INFINITY) {  // both partials empty
+    *m = mx;
+    *ps2 = 0.f;
+    *cs2 = 0.f;
+    return;
+  }
+  *m = mx;
+  *ps2 = ps * expf(pm - mx);
+  *cs2 = cs * expf(cm - mx);
+}
+
+// VEC: true when D is a multiple of the 16-byte vector width and the row bases stay aligned.
+template <typename T, bool VEC>
+__global__ void __launch_bounds__(kThreads) merge_sbh_kernel(
+    const T* prev_out, const float* prev_max, const float* prev_sum,  // may alias the outputs
+    const T* __restrict__ cur_out,
+    const float* __restrict__ cur_max, const float* __restrict__ cur_sum, int S, int B, int N,
+    int D, T* out, float* out_max, float* out_sum) {
+  __shared__ float s_po[kRows], s_co[kRows];
+  const int bn = blockIdx.x;  // b * N + n
+  const int b = bn / N, n = bn - b * N;
+  const int s0 = blockIdx.y * kRows;
+  const int rows = min(kRows, S - s0);
+
+  // ---- statistics: ROWS * 8 contiguous floats per array, one per thread ----------------
+  {
+    const int t = threadIdx.x;  // t = row * 8 + lane
+    const int64_t base = ((int64_t)bn * S + s0) * 8;
+    if (t < rows * 8) {
+      const float pm = prev_max[base + t], ps = prev_sum[base + t];
+      const float cm = cur_max[base + t], cs = cur_sum[base + t];
+      float m, ps2, cs2;
+      merge_lane(pm, ps, cm, cs, &m, &ps2, &cs2);
+      const float l = ps2 + cs2;
+      out_max[base + t] = m;
+      out_sum[base + t] = l;
+      if ((t & 7) == 0) {
+        const float inv = l != 0.f ? 1.f / l : 0.f;
+        s_po[t >> 3] = ps2 * inv;
+        s_co[t >> 3] = cs2 * inv;
+      }
+    }
+  }
+  __syncthreads();
+
+  // ---- outputs: row s is D contiguous elements at ((s*B + b)*N + n)*D -------------------
+  const int64_t row_stride = (int64_t)B * N * D;
+  const int64_t row0 = ((int64_t)s0 * B + b) * N * D + (int64_t)n * D;
+  if constexpr (VEC) {
+    constexpr int V = Vec16<T>::n;
+    const int vpr = D / V;                  // vectors per row
+    const int total = rows * vpr;
+    constexpr int kPer = 4;                 // vectors per thread in flight
+    for (int base = 0; base < total; base += kThreads * kPer) {
+      uint4 pv[kPer], cv[kPer];
+      int idx[kPer];
+#pragma unroll
+      for (int u = 0; u < kPer; ++u) {
+        idx[u] = base + u * kThreads + threadIdx.x;
+        if (idx[u] < total) {
+          const int r = idx[u] / vpr, c = idx[u] - r * vpr;
+          const int64_t off = row0 + r * row_stride + (int64_t)c * V;
+          pv[u] = __ldcs(reinterpret_cast<const uint4*>(prev_out + off));
+          cv[u] = __ldcs(reinterpret_cast<const uint4*>(cur_out + off));
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kPer; ++u) {
+        if (idx[u] < total) {
+          const int r = idx[u] / vpr, c = idx[u] - r * vpr;
+          const int64_t off = row0 + r * row_stride + (int64_t)c * V;
+          float a[V], bb[V], o[V];
+          unpack(pv[u], a, (T*)nullptr);
+          unpack(cv[u], bb, (T*)nullptr);
+          const float po = s_po[r], co = s_co[r];
+#pragma unroll
+          for (int i = 0; i < V; ++i) o[i] = fmaf(a[i], po, bb[i] * co);
+          __stcs(reinterpret_cast<uint4*>(out + off), pack(o, (T*)nullptr));
+        }
+      }
+    }
+  } else {
+    const int total = rows * D;
+    for (int i = threadIdx.x; i < total; i += kThreads) {
+      const int r = i / D, d = i - r * D;
+      const int64_t off = row0 + r * row_stride + d;
+      const float o = fmaf(to_f(prev_out[off]), s_po[r], to_f(cur_out[off]) * s_co[r]);
+      from_f(o, out + off);
+    }
+  }
+}
+
+template <typename T>
+cudaError_t launch_typed(const MergeArgs& a, cudaStream_t st) {
+  constexpr int V = Vec16<T>::n;
+  const bool vec = (a.D % V) == 0 && ((uintptr_t)a.prev_out % 16) == 0 &&
+                   ((uintptr_t)a.cur_out % 16) == 0 && ((uintptr_t)a.out % 16) == 0;
+  dim3 grid(a.B * a.N, (a.S + kRows - 1) / kRows);
+  if (vec)
+    merge_sbh_kernel<T, true><<<grid, kThreads, 0, st>>>(
+        (const T*)a.prev_out, a.prev_max, a.prev_sum, (const T*)a.cur_out, a.cur_max, a.cur_sum,
+        a.S, a.B, a.N, a.D, (T*)a.out, a.out_max, a.out_sum);
+  else
+    merge_sbh_kernel<T, false><<<grid, kThreads, 0, st>>>(
+        (const T*)a.prev_out, a.prev_max, a.prev_sum, (const T*)a.cur_out, a.cur_max, a.cur_sum,
+        a.S, a.B, a.N, a.D, (T*)a.out, a.out_max, a.out_sum);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_merge(const MergeArgs& a, cudaStream_t st) {
+  if (a.dtype == ATTN_BF16) return launch_typed<__nv_bfloat16>(a, st);
+  return launch_typed<float>(a, st);
+}
+
+}  // namespace sdpa

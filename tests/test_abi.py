@@ -1,0 +1,125 @@
+"""The C-ABI library builds, loads and exports every function include/attn.h declares; host-side
+argument checks answer without a GPU (no compute call is made here)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import scaled_dot_product_16_b200 as sdpa
+from scaled_dot_product_16_b200 import build as sdpa_build
+from scaled_dot_product_16_b200 import workloads as W
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "attn.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    sdpa_build.build()
+    return sdpa.load_library()
+
+
+def _declared():
+    text = open(HEADER).read()
+    return re.findall(r"ATTN_API\s+[\w\s\*]+?\b(attn_\w+)\s*\(", text)
+
+
+def _enums():
+    text = open(HEADER).read()
+    return {k: int(v) for k, v in re.findall(r"\b(ATTN_[A-Z0-9_]+)\s*=\s*(\d+)", text)}
+
+
+def test_header_declares_the_three_operations():
+    names = set(_declared())
+    assert {"attn_fwd", "attn_sparse_csr", "attn_merge", "attn_get_last_error"} <= names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", sdpa.lib_path()], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (attn_\w+)", out))
+    for name in _declared():
+        assert name in exported, name
+        assert hasattr(lib, name)
+
+
+def test_enum_values_match_binding():
+    e = _enums()
+    for k, v in e.items():
+        if hasattr(sdpa, k):
+            assert getattr(sdpa, k) == v, k
+    assert (W.BF16, W.F32) == (e["ATTN_BF16"], e["ATTN_F32"])
+    assert (W.BHSD, W.TND) == (e["ATTN_BHSD"], e["ATTN_TND"])
+    assert (W.MASK_NONE, W.MASK_CAUSAL_TOPLEFT, W.MASK_CAUSAL_BOTTOMRIGHT) == (
+        e["ATTN_MASK_NONE"], e["ATTN_MASK_CAUSAL_TOPLEFT"], e["ATTN_MASK_CAUSAL_BOTTOMRIGHT"])
+
+
+def test_version_and_strings(lib):
+    assert lib.attn_abi_version() >> 16 == 1
+    for s in range(6):
+        assert lib.attn_status_string(s)
+
+
+def _fwd(lib, **kw):
+    a = dict(q=16, k=16, v=16, cq=None, ck=None, B=1, Sq=8, Skv=8, Nq=2, Nkv=1, D=64, scale=0.125,
+             mask=0, dtype=0, layout=0, out=16, m=None, l=None, stream=None)
+    a.update(kw)
+    return lib.attn_fwd(a["q"], a["k"], a["v"], a["cq"], a["ck"], a["B"], a["Sq"], a["Skv"],
+                        a["Nq"], a["Nkv"], a["D"], a["scale"], a["mask"], a["dtype"], a["layout"],
+                        a["out"], a["m"], a["l"], a["stream"])
+
+
+def test_host_validation_without_gpu(lib):
+    INVALID, UNSUP, OK = sdpa.ATTN_ERR_INVALID, sdpa.ATTN_ERR_UNSUPPORTED, sdpa.ATTN_OK
+    assert _fwd(lib, layout=7) == INVALID
+    assert _fwd(lib, dtype=5) == INVALID
+    assert _fwd(lib, mask=3) == INVALID
+    assert _fwd(lib, Nq=3, Nkv=2) == INVALID         # Nq/Nkv must be an integer
+    assert _fwd(lib, Nq=257, Nkv=1) == INVALID       # Nq in 1..256
+    assert _fwd(lib, D=769) == INVALID               # D in 1..768
+    assert _fwd(lib, scale=0.0) == INVALID
+    assert _fwd(lib, scale=float("nan")) == INVALID
+    assert _fwd(lib, m=16) == INVALID                # max without sum
+    assert _fwd(lib, q=None) == INVALID
+    assert _fwd(lib, D=96) == UNSUP                  # bf16 runs D = 64 or 128
+    assert _fwd(lib, q=18) == INVALID                # bf16 pointers must be 16-byte aligned
+    assert _fwd(lib, layout=1, B=3) == INVALID       # TND needs cumulative lengths
+    assert _fwd(lib, layout=1, B=2049, cq=16, ck=16) == INVALID
+    assert _fwd(lib, layout=1, B=1, Sq=(1 << 20) + 1, cq=16, ck=16) == INVALID
+    assert _fwd(lib, layout=0, cq=16) == INVALID     # BHSD takes no lengths
+    # empty problems succeed without a launch
+    assert _fwd(lib, B=0) == OK
+    assert _fwd(lib, Sq=0) == OK
+    assert _fwd(lib, layout=1, B=0) == OK
+
+
+def test_merge_and_csr_validation_without_gpu(lib):
+    P = 16
+    args = [P] * 6
+    assert lib.attn_merge(*args, 8, 1, 2, 64, 0, 1, None, P, P, P, None) == sdpa.ATTN_ERR_UNSUPPORTED
+    assert lib.attn_merge(*args, 8, 1, 2, 64, 0, 0, P, P, P, P, None) == sdpa.ATTN_ERR_INVALID
+    assert lib.attn_merge(*args, 8, 1, 0, 64, 0, 0, None, P, P, P, None) == sdpa.ATTN_ERR_INVALID
+    assert lib.attn_merge(*args, 0, 1, 2, 64, 0, 0, None, P, P, P, None) == sdpa.ATTN_OK
+    assert lib.attn_sparse_csr(P, P, P, P, P, 1, 1, 4, 0, 4, P, None) == sdpa.ATTN_ERR_INVALID
+    assert lib.attn_sparse_csr(P, P, P, P, P, 1, 1, 4, 300, 4, P, None) == sdpa.ATTN_ERR_UNSUPPORTED
+    assert lib.attn_sparse_csr(P, P, P, P, P, 0, 1, 4, 64, 4, P, None) == sdpa.ATTN_OK
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    monkeypatch.setattr(sdpa, "_lib", None)
+    monkeypatch.setattr(sdpa, "lib_path", lambda: str(tmp_path / "libattn.so"))
+    with pytest.raises(RuntimeError):
+        sdpa.attn_merge(None, None, None, None, None, None, S=1, B=1, N=1, D=1, dtype=0,
+                        out=None, out_max=None, out_sum=None, stream=0)
+
+
+def test_product_never_touches_the_oracle():
+    pkg = os.path.join(ROOT, "scaled_dot_product_16_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                text = open(os.path.join(dirpath, f), encoding="utf-8").read()
+                assert not re.search(r"^\s*(import|from)\s+oracle\b", text, re.M), f
+                assert "attn_oracle" not in text, f

@@ -1,0 +1,98 @@
+"""attn_sparse_csr on the GPU against the float64 oracle (and the Paddle worked example)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import scaled_dot_product_16_b200 as sdpa
+from scaled_dot_product_16_b200 import workloads as W
+from tests import gpu_util as G
+from tests.golden.loader import load as load_golden
+
+pytestmark = pytest.mark.gpu
+
+
+def _run(q, k, v, off, cols, B, H, S, D):
+    dq, dk, dv = (torch.as_tensor(x).float().cuda().contiguous() for x in (q, k, v))
+    doff = torch.from_numpy(np.ascontiguousarray(off, np.int32)).cuda()
+    dcol = torch.from_numpy(np.ascontiguousarray(cols, np.int32)).cuda()
+    out = torch.full_like(dq, float("nan"))
+    sdpa.attn_sparse_csr(dq, dk, dv, doff, dcol, B=B, H=H, S=S, D=D, nnz_cap=cols.shape[-1], out=out)
+    return out.cpu(), sdpa.attn_get_last_error()
+
+
+def test_paddle_worked_example():
+    g = load_golden("paddle_sparse_attention_example.txt")
+    shape = tuple(int(x) for x in g["shape"])
+    q = g["query"].astype(np.float32).reshape(shape)
+    off = g["offset"].astype(np.int32).reshape(1, 1, -1)
+    col = g["columns"].astype(np.int32).reshape(1, 1, -1)
+    out, st = _run(q, q, q, off, col, 1, 1, shape[2], shape[3])
+    assert st == 0
+    # the page prints float32 values to 8 decimals
+    assert np.max(np.abs(out.numpy() - g["output"].reshape(shape))) <= 1e-6
+
+
+def _random_pattern(rng, B, H, S, max_per_row):
+    offs = np.zeros((B, H, S + 1), np.int32)
+    rows = []
+    for bh in range(B * H):
+        cnt = rng.integers(0, max_per_row + 1, size=S)
+        offs.reshape(B * H, S + 1)[bh, 1:] = np.cumsum(cnt)
+        rows.append(rng.integers(0, S, size=int(cnt.sum())))  # unsorted, with repeats
+    cap = max(1, max(len(r) for r in rows))
+    cols = np.zeros((B, H, cap), np.int32)
+    for bh, r in enumerate(rows):
+        cols.reshape(B * H, cap)[bh, :len(r)] = r
+    return offs, cols
+
+
+@pytest.mark.parametrize("D", [64, 1, 13, 40, 128, 256])
+def test_random_patterns(D):
+    rng = np.random.default_rng(D)
+    B, H, S = 2, 3, 97
+    q, k, v = (W.randn((B, H, S, D), 100 + i) for i in range(3))
+    off, cols = _random_pattern(rng, B, H, S, 40)
+    out, st = _run(q, k, v, off, cols, B, H, S, D)
+    assert st == 0
+    ref = oracle.sparse_csr(q, k, v, off, cols, B=B, H=H, S=S, D=D)
+    G.check_out(out.numpy(), ref, W.F32, "csr out")
+
+
+def test_cfg4_full_size():
+    """Configuration 4 at full size: B=2, H=8, S=4096, D=64, window 256 + every 64th column."""
+    inp = W.cfg4_csr(seed=0)
+    out, st = _run(inp.q, inp.k, inp.v, inp.offset, inp.columns, inp.B, inp.H, inp.S, inp.D)
+    assert st == 0
+    ref = oracle.sparse_csr(inp.q, inp.k, inp.v, inp.offset, inp.columns, B=inp.B, H=inp.H,
+                            S=inp.S, D=inp.D)
+    G.check_out(out.numpy(), ref, W.F32, "cfg4 out")
+
+
+def test_full_pattern_equals_dense_attention():
+    B, H, S, D = 1, 2, 150, 64
+    q, k, v = (W.randn((B, H, S, D), 200 + i) for i in range(3))
+    cols = np.broadcast_to(np.tile(np.arange(S, dtype=np.int32), S), (B, H, S * S)).copy()
+    off = np.broadcast_to(np.arange(0, S * S + 1, S, dtype=np.int32), (B, H, S + 1)).copy()
+    out, st = _run(q, k, v, off, cols, B, H, S, D)
+    assert st == 0
+    inp = W.AttnInputs(q, k, v, W.BHSD, W.MASK_NONE, W.F32, B, S, S, H, H, D, 1.0 / np.sqrt(D))
+    dense, _, _ = G.run_fwd(inp)
+    assert np.max(np.abs(out.numpy() - dense.numpy())) <= 2e-6
+
+
+def test_bad_columns_report_data_error():
+    B, H, S, D = 1, 1, 8, 64
+    q = W.randn((B, H, S, D), 1)
+    off = np.arange(S + 1, dtype=np.int32).reshape(1, 1, -1)
+    cols = np.arange(S, dtype=np.int32).reshape(1, 1, -1)
+    cols[0, 0, 3] = S  # out of range
+    out, st = _run(q, q, q, off, cols, B, H, S, D)
+    assert st == sdpa.ATTN_ERR_DATA
+    assert torch.all(out[0, 0, 3] == 0)  # the offending row is written as zeros
+    assert torch.allclose(out[0, 0, 2], q[0, 0, 2])  # single-entry rows are v_j
+    off2 = off.copy()
+    off2[0, 0, 5] = 2  # decreasing row pointer
+    cols[0, 0, 3] = 3
+    out, st = _run(q, q, q, off2, cols, B, H, S, D)
+    assert st == sdpa.ATTN_ERR_DATA

@@ -1,0 +1,162 @@
+"""attn_fwd on the GPU against the float64 oracle (element by element), through the C ABI."""
+import numpy as np
+import pytest
+import torch
+
+import scaled_dot_product_16_b200 as sdpa
+from scaled_dot_product_16_b200 import workloads as W
+from tests import gpu_util as G
+
+pytestmark = pytest.mark.gpu
+
+BF, F32 = torch.bfloat16, torch.float32
+
+
+def _full_check(inp, stats=True):
+    out, m, l = G.run_fwd(inp, stats=stats)
+    ref, rm, rl = G.oracle_fwd(inp)
+    info = G.check_out(G.f64(out), ref, inp.dtype)
+    if stats:
+        G.check_stats(m.numpy(), l.numpy(), rm, rl)
+    return info
+
+
+# ---- configuration 1: dense 2x4x256x64, non-causal, fp32 and bf16 ---------------------------
+@pytest.mark.parametrize("dtype", [F32, BF], ids=["f32", "bf16"])
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_cfg1_dense_small(dtype, seed):
+    _full_check(W.cfg1_dense_small(dtype, seed))
+
+
+# ---- dense BHSD shapes spanning several tiles with ragged tails ------------------------------
+@pytest.mark.parametrize("dtype", [BF, F32], ids=["bf16", "f32"])
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("causal", [False, True], ids=["full", "causal"])
+@pytest.mark.parametrize("S", [1, 100, 256, 300, 640])
+def test_dense_shapes(dtype, D, causal, S):
+    inp = W.dense_bhsd(2, 3, S, D, causal=causal, dtype=dtype, seed=S + D, cfg=11)
+    _full_check(inp)
+
+
+@pytest.mark.parametrize("dtype", [BF, F32], ids=["bf16", "f32"])
+@pytest.mark.parametrize("Sq,Skv", [(200, 700), (700, 200), (129, 1), (1, 513)])
+@pytest.mark.parametrize("mode", [W.MASK_NONE, W.MASK_CAUSAL_TOPLEFT, W.MASK_CAUSAL_BOTTOMRIGHT])
+def test_rectangular_and_masks(dtype, Sq, Skv, mode):
+    inp = W.dense_bhsd(1, 2, Sq, 128, causal=False, dtype=dtype, seed=Sq * 7 + Skv, cfg=12, Skv=Skv)
+    inp.mask_mode = mode
+    _full_check(inp)
+
+
+@pytest.mark.parametrize("dtype", [BF, F32], ids=["bf16", "f32"])
+@pytest.mark.parametrize("Nq,Nkv", [(8, 2), (6, 1), (4, 4)])
+def test_gqa_mqa(dtype, Nq, Nkv):
+    inp = W.dense_bhsd(2, Nq, 333, 128, causal=True, dtype=dtype, seed=Nq + Nkv, cfg=13, Hkv=Nkv)
+    _full_check(inp)
+
+
+# ---- packed varlen (TND) ---------------------------------------------------------------------
+@pytest.mark.parametrize("dtype", [BF, F32], ids=["bf16", "f32"])
+@pytest.mark.parametrize("lens", [[2, 2, 0, 2, 2], [0, 700, 1, 0, 257, 513, 0], [1000], [0, 0, 5]])
+@pytest.mark.parametrize("mode", [W.MASK_NONE, W.MASK_CAUSAL_TOPLEFT])
+def test_varlen(dtype, lens, mode):
+    inp = W.varlen_tnd(lens, 8, 2, 128, causal=False, dtype=dtype, seed=sum(lens), cfg=14,
+                       mask_mode=mode)
+    _full_check(inp)
+
+
+@pytest.mark.parametrize("dtype", [BF, F32], ids=["bf16", "f32"])
+def test_varlen_different_kv_lengths(dtype):
+    lq, lk = [100, 0, 300, 129], [250, 7, 300, 0]
+    for mode in (W.MASK_NONE, W.MASK_CAUSAL_TOPLEFT, W.MASK_CAUSAL_BOTTOMRIGHT):
+        inp = W.varlen_tnd(lq, 4, 1, 64, causal=False, dtype=dtype, seed=5, cfg=15, lengths_kv=lk,
+                           mask_mode=mode)
+        _full_check(inp)
+
+
+def test_cfg3_small_varlen_gqa():
+    """Configuration 3 in miniature: 16 sequences up to 1024 tokens (index 7 empty), GQA 32/8."""
+    inp = W.cfg3_varlen_gqa(seed=0, max_len=1024)
+    _full_check(inp)
+
+
+def test_no_stats_pointer():
+    inp = W.dense_bhsd(1, 2, 300, 128, causal=True, dtype=BF, seed=3, cfg=16)
+    out, _, _ = G.run_fwd(inp, stats=False)
+    ref, _, _ = G.oracle_fwd(inp)
+    G.check_out(G.f64(out), ref, inp.dtype)
+
+
+# ---- full-size configurations: sampled rows ----------------------------------------------------
+def _sampled_check(inp, seed):
+    out, m, l = G.run_fwd(inp)
+    rows_h, rows_t = G.sample_rows(inp, seed)
+    og, mg, lg = G.gather_rows(out, m, l, inp, rows_h, rows_t)
+    ref, rm, rl = G.oracle_rows(inp, rows_h, rows_t)
+    G.check_out(og, ref, inp.dtype)
+    G.check_stats(mg, lg, rm, rl)
+    # every output is finite (no NaN from masked or padded rows)
+    assert torch.isfinite(out.float()).all()
+
+
+def test_cfg2_full_size_sampled():
+    _sampled_check(W.cfg2_dense_causal(seed=0), seed=2)
+
+
+def test_cfg3_full_size_sampled():
+    _sampled_check(W.cfg3_varlen_gqa(seed=0), seed=3)
+
+
+# ---- properties -----------------------------------------------------------------------------------
+def test_deterministic_bitwise():
+    inp = W.cfg3_varlen_gqa(seed=1, max_len=2048)
+    a = G.run_fwd(inp)
+    b = G.run_fwd(inp)
+    for x, y in zip(a, b):
+        assert torch.equal(x, y)
+
+
+def test_varlen_equals_dense_per_sequence():
+    lens = [300, 0, 513]
+    inp = W.varlen_tnd(lens, 4, 2, 128, causal=True, dtype=BF, seed=9, cfg=17)
+    out, m, l = G.run_fwd(inp)
+    start = 0
+    for L in lens:
+        if L == 0:
+            continue
+        q = inp.q[start:start + L].permute(1, 0, 2).unsqueeze(0).contiguous()
+        k = inp.k[start:start + L].permute(1, 0, 2).unsqueeze(0).contiguous()
+        v = inp.v[start:start + L].permute(1, 0, 2).unsqueeze(0).contiguous()
+        d = W.AttnInputs(q, k, v, W.BHSD, W.MASK_CAUSAL_TOPLEFT, W.BF16, 1, L, L, 4, 2, 128, inp.scale)
+        od, md, ld = G.run_fwd(d)
+        assert torch.equal(od[0].permute(1, 0, 2), out[start:start + L])
+        assert torch.equal(md[0].T, m[start:start + L]) and torch.equal(ld[0].T, l[start:start + L])
+        start += L
+
+
+# ---- boundary errors ------------------------------------------------------------------------------
+def test_bad_cu_seqlens_reports_data_error():
+    inp = W.varlen_tnd([100, 200], 2, 2, 128, causal=True, dtype=BF, seed=1, cfg=18)
+    q, k, v, cq, ck = G.to_dev(inp)
+    out = torch.zeros_like(q)
+    bad = torch.tensor([200, 100], dtype=torch.int32, device="cuda")  # decreasing
+    sdpa.attn_fwd(q, k, v, cu_seqlens_q=bad, cu_seqlens_kv=ck, B=2, Sq=300, Skv=300, Nq=2, Nkv=2,
+                  D=128, scale=inp.scale, mask_mode=1, dtype=W.BF16, layout=W.TND, out=out)
+    assert sdpa.attn_get_last_error() == sdpa.ATTN_ERR_DATA
+    assert sdpa.attn_get_last_error() == 0  # read clears the word
+
+
+def test_host_validation():
+    inp = W.dense_bhsd(1, 2, 64, 128, causal=False, dtype=BF, seed=1, cfg=19)
+    q, k, v, _, _ = G.to_dev(inp)
+    out = torch.empty_like(q)
+    kw = dict(B=1, Sq=64, Skv=64, Nq=2, Nkv=2, D=128, scale=0.1, mask_mode=0, dtype=W.BF16,
+              layout=W.BHSD, out=out)
+    with pytest.raises(sdpa.AttnError) as e:
+        sdpa.attn_fwd(q, k, v, **{**kw, "Nkv": 3})
+    assert e.value.status == sdpa.ATTN_ERR_INVALID
+    with pytest.raises(sdpa.AttnError) as e:
+        sdpa.attn_fwd(q, k, v, **{**kw, "D": 96})
+    assert e.value.status == sdpa.ATTN_ERR_UNSUPPORTED
+    with pytest.raises(sdpa.AttnError) as e:
+        sdpa.attn_fwd(q[..., 1:], k, v, **kw)  # misaligned base pointer
+    assert e.value.status == sdpa.ATTN_ERR_INVALID
