@@ -1,0 +1,439 @@
+#!/usr/bin/env python
+"""Benchmark of the attention hot path on B200.
+
+One step runs every operation of the path once, on inputs already resident in HBM:
+  1. attn_fwd on the packed varlen batch: 16 sequences of U{0..8192} tokens (index 7 empty),
+     Nq=32, Nkv=8, D=128, bf16, causal per sequence (the tcgen05 kernel);
+  2. attn_sparse_csr on B=2, H=8, S=4096, D=64 fp32 with a 256-wide window plus every 64th column;
+  3. three attn_merge calls folding 4 partial results of S=8192, B=4, N=32, D=128 (bf16, SBH,
+     statistics [B,N,S,8]) into one, as a 4-chunk ring-attention step would.
+Each operation is timed with CUDA events on the stream it is launched on. The headline `value`
+is attn_fwd TFLOP/s over all ranks (4*Nq*D FLOPs per visible pair, divided by the max over
+ranks of the time); the merge's HBM GB/s is reported beside it (the second half of the metric).
+
+  python bench.py [--gpus N --steps K --warmup W]          # this library
+  python bench.py --impl reference ...                       # the float64 CPU oracle, sampled
+Multi-GPU: launched by torchrun, one process per GPU; every rank runs its own batch (seeded by
+rank, weak scaling) and no data-path collective exists (the path partitions by sequence and
+head); NCCL carries only the barrier and the max-over-ranks of the times.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import scaled_dot_product_16_b200 as sdpa  # noqa: E402
+from scaled_dot_product_16_b200 import metrics as M  # noqa: E402
+from scaled_dot_product_16_b200 import workloads as W  # noqa: E402
+
+METRIC = "attn fwd TFLOP/s & % of BF16 tensor peak; attn_merge HBM GB/s & % of peak"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+# DRAM traffic of one attn_fwd launch on the varlen workload, from an ncu capture (see
+# profiles/); valid only for the kernel source it was measured on.
+TRAFFIC = {"kernel_sha": None, "bytes_per_launch": None}
+
+
+def kernel_sha() -> str:
+    p = os.path.join(ROOT, "scaled_dot_product_16_b200", "csrc", "fwd_bf16_sm100.cu")
+    return hashlib.sha256(open(p, "rb").read()).hexdigest()[:16]
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+# ---------------------------------------------------------------------------------------------
+# distributed plumbing
+# ---------------------------------------------------------------------------------------------
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def reduce(x: float, world: int, op: str) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX if op == "max" else dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+            return
+        t0 = time.time()  # the first sample marks the sampler as running
+        while time.time() - t0 < 15 and self.proc.poll() is None:
+            if os.path.getsize(self.path) > 0:
+                break
+            time.sleep(0.05)
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        self.proc.wait(timeout=10)
+        rows = [l.split(", ") for l in open(self.path).read().strip().splitlines() if l.strip()]
+        os.unlink(self.path)
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            try:
+                sm.append(float(r[1]))
+                smax = float(r[2])
+                for n, v in zip(names, r[5:9]):
+                    if v.strip().lower() == "active":
+                        reasons.add(n)
+            except (ValueError, IndexError):
+                continue
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------------------------
+# workloads on the device
+# ---------------------------------------------------------------------------------------------
+class FwdCase:
+    def __init__(self, inp: W.AttnInputs):
+        self.inp = inp
+        self.q, self.k, self.v = (t.cuda() for t in (inp.q, inp.k, inp.v))
+        self.cq = torch.from_numpy(inp.cu_q).cuda() if inp.cu_q is not None else None
+        self.ck = torch.from_numpy(inp.cu_kv).cuda() if inp.cu_kv is not None else None
+        self.out = torch.empty_like(self.q)
+        shape = (inp.Sq, inp.Nq) if inp.layout == W.TND else (inp.B, inp.Nq, inp.Sq)
+        self.m = torch.empty(shape, device="cuda")
+        self.l = torch.empty(shape, device="cuda")
+        self.flops = M.attn_fwd_flops(inp)
+
+    def run(self, q=None, k=None, v=None, cq=None, ck=None, out=None, m=None, l=None):
+        i = self.inp
+        sdpa.attn_fwd(q if q is not None else self.q, k if k is not None else self.k,
+                      v if v is not None else self.v, cu_seqlens_q=cq if cq is not None else self.cq,
+                      cu_seqlens_kv=ck if ck is not None else self.ck, B=i.B, Sq=i.Sq, Skv=i.Skv,
+                      Nq=i.Nq, Nkv=i.Nkv, D=i.D, scale=i.scale, mask_mode=i.mask_mode, dtype=i.dtype,
+                      layout=i.layout, out=out if out is not None else self.out,
+                      softmax_max=m if m is not None else self.m,
+                      softmax_sum=l if l is not None else self.l)
+
+
+class CsrCase:
+    def __init__(self, inp: W.CsrInputs):
+        self.inp = inp
+        self.q, self.k, self.v = (t.cuda() for t in (inp.q, inp.k, inp.v))
+        self.off = torch.from_numpy(inp.offset).cuda()
+        self.col = torch.from_numpy(inp.columns).cuda()
+        self.out = torch.empty_like(self.q)
+        self.flops = M.csr_flops(inp)
+
+    def run(self):
+        i = self.inp
+        sdpa.attn_sparse_csr(self.q, self.k, self.v, self.off, self.col, B=i.B, H=i.H, S=i.S, D=i.D,
+                             nnz_cap=i.nnz_cap, out=self.out)
+
+
+class MergeCase:
+    """Four partial results (outputs + statistics) folded by three merges into the first."""
+
+    def __init__(self, seed: int, S=8192, B=4, N=32, D=128):
+        self.S, self.B, self.N, self.D = S, B, N, D
+        self.parts = []
+        for c in range(4):
+            o = W.randn((S, B, N * D), W.mix_seed(5, seed, 10 + c), torch.bfloat16).cuda()
+            m, l = W.merge_stats_random(B, N, S, W.mix_seed(5, seed, 20 + c))
+            self.parts.append((o, m.cuda(), l.cuda()))
+        self.acc = [t.clone() for t in self.parts[0]]
+        self.bytes = M.merge_bytes(S, B, N, D, 2)
+
+    def run_one(self, c: int):
+        a, p = self.acc, self.parts[c]
+        sdpa.attn_merge(a[0], a[1], a[2], p[0], p[1], p[2], S=self.S, B=self.B, N=self.N, D=self.D,
+                        dtype=W.BF16, out=a[0], out_max=a[1], out_sum=a[2])
+
+
+# ---------------------------------------------------------------------------------------------
+# CPU oracle (the reported baseline and the reference arm)
+# ---------------------------------------------------------------------------------------------
+def oracle_sample(inp: W.AttnInputs, n_rows: int, seed: int):
+    """Random (head, token) rows of the workload and their algorithmic FLOPs."""
+    rng = np.random.default_rng(seed)
+    rows_t = rng.integers(0, inp.Sq, size=n_rows).astype(np.int64)
+    rows_h = rng.integers(0, inp.Nq, size=n_rows).astype(np.int32)
+    lens = W.lengths_from_cu_seqlens(inp.cu_q)
+    starts = np.concatenate([[0], np.cumsum(lens)[:-1]])
+    seq = np.searchsorted(np.cumsum(lens), rows_t, side="right")
+    i = rows_t - starts[seq]
+    klens = W.lengths_from_cu_seqlens(inp.cu_kv)[seq]
+    vis = np.minimum(i + 1, klens) if inp.mask_mode != W.MASK_NONE else klens
+    return rows_h, rows_t, int(4 * inp.D * vis.sum())
+
+
+def time_oracle(inp: W.AttnInputs, n_rows: int, seed: int):
+    import oracle  # the CPU baseline leg is one of the two places bench.py runs the oracle
+    rows_h, rows_t, flops = oracle_sample(inp, n_rows, seed)
+    t0 = time.perf_counter()
+    oracle.attn_fwd_rows(inp.q, inp.k, inp.v, rows_h, rows_t, cu_q=inp.cu_q, cu_kv=inp.cu_kv, B=inp.B,
+                         Sq=inp.Sq, Skv=inp.Skv, Nq=inp.Nq, Nkv=inp.Nkv, D=inp.D, scale=inp.scale,
+                         mask_mode=inp.mask_mode, layout=inp.layout)
+    return flops, time.perf_counter() - t0
+
+
+def oracle_threads() -> int:
+    return int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+
+
+def cpu_baseline(inp: W.AttnInputs, budget_s: float = 20.0) -> dict:
+    """The oracle as it stands on this host's cores, on a bounded row sample of the workload."""
+    n = 64
+    flops, dt = time_oracle(inp, n, 1234)
+    while dt < 1.0 and n < 1 << 20:  # calibrate on growing samples
+        n *= 4
+        flops, dt = time_oracle(inp, n, 1234)
+    n = max(n, int(n * budget_s / dt))  # then one sample sized to about the budget
+    flops, dt = time_oracle(inp, n, 4321)
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": oracle_threads(), "kind": "oracle",
+            "sample": f"{n} random (head, query-token) rows of the varlen batch, all their visible keys; "
+                      f"{flops / 1e9:.1f} GFLOP in {dt:.1f} s"}
+
+
+# ---------------------------------------------------------------------------------------------
+def config_dict(fwd: FwdCase, world: int) -> dict:
+    i = fwd.inp
+    return {"workload": "varlen TND causal GQA bf16: 16 seqs U{0..8192} (idx 7 empty), Nq=32 Nkv=8 D=128; "
+                        "plus CSR fp32 2x8x4096x64 (window 256 + every 64th) and 3 SBH merges 8192x4x32x128 bf16",
+            "tokens_per_rank": int(i.Sq), "n_seq": int(i.B), "Nq": i.Nq, "Nkv": i.Nkv, "D": i.D,
+            "causal": True, "parallelism": f"replicas x{world} (sequence partition, no collective)",
+            "l2": "inputs larger than L2 (attn_fwd 0.9 GB, merge 1.0 GB per step), no flush"}
+
+
+def run_reference(args, rank: int, world: int):
+    if rank != 0:
+        return
+    inp = W.cfg3_varlen_gqa(seed=0, max_len=args.max_len)
+    rows = args.ref_rows
+    for s in range(args.warmup):
+        time_oracle(inp, max(8, rows // 8), 100 + s)
+    fl, dt = 0, 0.0
+    for s in range(args.steps):
+        f, d = time_oracle(inp, rows, 1000 + s)
+        fl += f
+        dt += d
+    val = fl / dt / 1e12
+    line = {"impl": "reference", "metric": METRIC, "value": val, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": "varlen TND causal GQA (oracle rows)", "max_len": args.max_len},
+            "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": oracle_threads(), "kind": "oracle",
+                             "sample": f"{rows} random (head, token) rows per step"},
+            "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args, rank: int, world: int, local: int):
+    sdpa.load_library()
+    peaks, peak_src = load_peaks()
+    fwd = FwdCase(W.cfg3_varlen_gqa(seed=rank, max_len=args.max_len))
+    parts = args.parts.split(",")
+    csr = CsrCase(W.cfg4_csr(seed=rank)) if "csr" in parts else None
+    mrg = MergeCase(seed=rank) if "merge" in parts else None
+    stream = torch.cuda.current_stream()
+    launches_per_step = 1 + (1 if csr else 0) + (3 if mrg else 0)
+
+    def step(ev):
+        ev[0].record(stream)
+        fwd.run()
+        ev[1].record(stream)
+        if csr:
+            csr.run()
+        ev[2].record(stream)
+        if mrg:
+            for c in (1, 2, 3):
+                mrg.run_one(c)
+        ev[3].record(stream)
+
+    for _ in range(args.warmup):
+        step([torch.cuda.Event(enable_timing=True) for _ in range(4)])
+    torch.cuda.synchronize()
+    assert sdpa.attn_get_last_error() == 0
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks.start()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for s in range(args.steps):
+        step(evs[s])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop()
+    status = sdpa.attn_get_last_error()
+    if status != 0:
+        raise RuntimeError(f"device status {status} during the timed region")
+
+    fwd_ms = sum(e[0].elapsed_time(e[1]) for e in evs)
+    csr_ms = sum(e[1].elapsed_time(e[2]) for e in evs)
+    mrg_ms = sum(e[2].elapsed_time(e[3]) for e in evs)
+    total_ms = t_start.elapsed_time(t_end)
+    fwd_ms_max = reduce(fwd_ms, world, "max")
+    total_ms_max = reduce(total_ms, world, "max")
+    flops_all = reduce(float(fwd.flops) * args.steps, world, "sum")
+    value = flops_all / (fwd_ms_max / 1e3) / 1e12
+
+    # dominant kernel roofline (attn_fwd, timed inside a long step: sustained peak)
+    achieved = fwd.flops / (fwd_ms / args.steps / 1e3) / 1e12
+    peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    traffic = TRAFFIC["bytes_per_launch"] if TRAFFIC["kernel_sha"] == kernel_sha() else None
+    line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": total_ms_max / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": config_dict(fwd, world),
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                         "frac": achieved / peak, "traffic": traffic,
+                         "kernel": "attn_fwd bf16 (tcgen05)",
+                         "peak_source": f"{peak_src} bf16_tflops_sustained"},
+            "parts": {"attn_fwd": {"ms": fwd_ms / args.steps, "tflops": achieved,
+                                   "flops_per_call": fwd.flops,
+                                   "frac_of_burst_peak": achieved / float(peaks.get("bf16_tflops", 1590.0))}},
+            "gpu_launches": launches_per_step * args.steps, "clocks": clk}
+    if csr:
+        line["parts"]["attn_sparse_csr"] = {"ms": csr_ms / args.steps,
+                                            "gflops": csr.flops / (csr_ms / args.steps / 1e3) / 1e9}
+    if mrg:
+        gbs = mrg.bytes * 3 / (mrg_ms / args.steps / 1e3) / 1e9
+        hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+        line["parts"]["attn_merge"] = {"ms_per_call": mrg_ms / args.steps / 3, "gbs": gbs,
+                                       "frac_of_hbm": gbs / hbm, "bytes_per_call": mrg.bytes,
+                                       "peak_source": f"{peak_src} hbm_gbs"}
+
+    # end to end through the public API: pinned host inputs -> device -> attn_fwd -> host
+    if args.e2e_steps > 0:
+        i = fwd.inp
+        hq, hk, hv = (t.pin_memory() for t in (i.q, i.k, i.v))
+        hcq = torch.from_numpy(i.cu_q).pin_memory()
+        ho = torch.empty(fwd.out.shape, dtype=fwd.out.dtype).pin_memory()
+        hm = torch.empty(fwd.m.shape).pin_memory()
+        hl = torch.empty(fwd.l.shape).pin_memory()
+        dq, dk, dv = torch.empty_like(fwd.q), torch.empty_like(fwd.k), torch.empty_like(fwd.v)
+        dcq = torch.empty_like(fwd.cq)
+
+        def e2e_step():
+            dq.copy_(hq, non_blocking=True)
+            dk.copy_(hk, non_blocking=True)
+            dv.copy_(hv, non_blocking=True)
+            dcq.copy_(hcq, non_blocking=True)
+            fwd.run(dq, dk, dv, dcq, dcq, fwd.out, fwd.m, fwd.l)
+            ho.copy_(fwd.out, non_blocking=True)
+            hm.copy_(fwd.m, non_blocking=True)
+            hl.copy_(fwd.l, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        barrier(world)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        e_ms = reduce(a.elapsed_time(b), world, "max")
+        e_flops = reduce(float(fwd.flops) * args.e2e_steps, world, "sum")
+        h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hcq))
+        d2h = sum(t.numel() * t.element_size() for t in (ho, hm, hl))
+        line["e2e"] = {"value": e_flops / (e_ms / 1e3) / 1e12, "unit": "TFLOP/s",
+                       "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                       "steps": args.e2e_steps, "what": "attn_fwd with pinned-host inputs copied in "
+                       "and outputs + statistics copied back, per step"}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(fwd.inp, args.cpu_budget)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--max-len", type=int, default=8192, help="max sequence length of the varlen batch")
+    ap.add_argument("--parts", default="fwd,csr,merge", help="operations in a step (fwd always runs)")
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=20.0, help="seconds of oracle work for cpu_baseline")
+    ap.add_argument("--ref-rows", type=int, default=2048, help="oracle rows per reference step")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    rank, world, local = dist_setup()
+    try:
+        if args.impl == "reference":
+            run_reference(args, rank, world)
+        else:
+            run_ours(args, rank, world, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()
