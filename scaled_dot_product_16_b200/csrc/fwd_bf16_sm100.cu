@@ -49,6 +49,38 @@ constexpr int kTmaWarp = 9;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale when the max grows by > 2^8
 constexpr uint64_t kWaitLimitNs = 200ull * 1000ull * 1000ull;  // 200 ms per barrier wait
+#ifndef SDPA_SUSPEND_NS
+#define SDPA_SUSPEND_NS 20000
+#endif
+constexpr uint32_t kSuspendNs = SDPA_SUSPEND_NS;  // longest hardware suspension per try_wait
+
+#ifndef SDPA_EMU_EVERY
+#define SDPA_EMU_EVERY 4
+#endif
+// One exp2 pair in kEmuEvery goes to the FMA-pipe polynomial (0: none).
+constexpr int kEmuEvery = SDPA_EMU_EVERY;
+
+// 2^x for a pair on the FMA/ALU pipes. Range reduction after Cody and Waite: x = j + f with
+// j = round(x) (adding 1.5 * 2^23 rounds to nearest and leaves j in the low mantissa bits) and
+// f in [-1/2, 1/2]; 2^f by a degree-3 polynomial fitted here by the Remez exchange for minimum
+// relative error (csrc/fit_exp2_poly.py, max relative error 7.5e-5); 2^j is added into the
+// exponent field. Inputs below -125 (including -inf from masking) give exactly 0.
+__device__ __forceinline__ void exp2_poly2(float x0, float x1, float& p0, float& p1) {
+  constexpr float kShift = 12582912.0f;  // 1.5 * 2^23
+  constexpr float c0 = 9.999280572e-01f, c1 = 6.932609677e-01f, c2 = 2.426111251e-01f,
+                  c3 = 5.517166853e-02f;
+  float t0, t1, j0, j1, f0, f1, q0, q1;
+  fadd2(x0, x1, kShift, kShift, t0, t1);
+  fadd2(t0, t1, -kShift, -kShift, j0, j1);
+  ffma2(j0, j1, -1.f, -1.f, x0, x1, f0, f1);  // f = x - j
+  ffma2(c3, c3, f0, f1, c2, c2, q0, q1);
+  ffma2(q0, q1, f0, f1, c1, c1, q0, q1);
+  ffma2(q0, q1, f0, f1, c0, c0, q0, q1);
+  const uint32_t b0 = __float_as_uint(q0) + (__float_as_uint(t0) << 23);
+  const uint32_t b1 = __float_as_uint(q1) + (__float_as_uint(t1) << 23);
+  p0 = x0 < -125.f ? 0.f : __uint_as_float(b0);
+  p1 = x1 < -125.f ? 0.f : __uint_as_float(b1);
+}
 
 template <int HD>
 struct Cfg {
@@ -80,17 +112,15 @@ struct Barriers {
 // With heed_abort = false (used when draining work already issued) only the time bound applies.
 __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort,
                                          int* status, bool heed_abort = true) {
-  if (mbar_try_wait(bar, parity)) return true;
+  if (mbar_try_wait_sleep(bar, parity, kSuspendNs)) return true;
   const uint64_t t0 = globaltimer_ns();
-  for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 255u) == 0) {
-      if (heed_abort && *abort) return false;
-      if (globaltimer_ns() - t0 > kWaitLimitNs) {
-        *abort = 1;
-        report(status, ATTN_ERR_TIMEOUT);
-        return false;
-      }
+  for (;;) {
+    if (mbar_try_wait_sleep(bar, parity, kSuspendNs)) return true;
+    if (heed_abort && *abort) return false;
+    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      *abort = 1;
+      report(status, ATTN_ERR_TIMEOUT);
+      return false;
     }
   }
 }
@@ -190,7 +220,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar_addr(&bars->drain), 1);
     for (int q = 0; q < 2; ++q) {
       mbar_init(bar_addr(&bars->s_full[q]), 1);
-      mbar_init(bar_addr(&bars->p_ready[q]), kBM);
+      mbar_init(bar_addr(&bars->p_ready[q]), 4);  // one arrival per softmax warp
       mbar_init(bar_addr(&bars->o_done[q]), 1);
     }
     bars->abort = 0;
@@ -251,26 +281,28 @@ __global__ void __launch_bounds__(kThreads, 1)
     // =============================== MMA issue ==========================================
     if (lane == 0) {
       const uint32_t S0 = tmem, S1 = tmem + 128, O0 = tmem + 256, O1 = tmem + 256 + HD;
+      // Descriptors are built once. K-step kk of an operand adds a constant to the start
+      // address field (shared-memory addresses stay below 256 KB, so the 14-bit field never
+      // carries), which keeps the issue loop at a few instructions per MMA.
+      const uint64_t dq0 = smem_desc_sw128(sQ, 16, 1024);
+      const uint64_t dq1 = dq0 + (uint64_t)(C::kTileBytes >> 4);
+      const uint64_t dk0 = smem_desc_sw128(sKV, 16, 1024);
+      const uint64_t dv0 = smem_desc_sw128(sKV, kBN * 128, 1024);
+      const uint32_t kvfull0 = bar_addr(&bars->kv_full[0]), kvempty0 = bar_addr(&bars->kv_empty[0]);
       auto full = [&](int i) {
-        return wait_bar(bar_addr(&bars->kv_full[i % C::kStages]), (i / C::kStages) & 1, abort,
-                        a.status);
+        return wait_bar(kvfull0 + 8 * (i % C::kStages), (i / C::kStages) & 1, abort, a.status);
       };
-      auto release = [&](int i) { mma_commit(bar_addr(&bars->kv_empty[i % C::kStages])); };
-      auto kv_smem = [&](int i) { return sKV + (i % C::kStages) * C::kTileBytes; };
-      auto issue_qk = [&](uint32_t d, uint32_t q_smem, uint32_t k_smem) {
-#pragma unroll
-        for (int kk = 0; kk < HD / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * (kBM * 128) + (kk & 3) * 32;
-          mma_ss(d, smem_desc_sw128(q_smem + off, 16, 1024), smem_desc_sw128(k_smem + off, 16, 1024),
-                 C::kIdescQK, kk > 0);
-        }
+      auto release = [&](int i) { mma_commit(kvempty0 + 8 * (i % C::kStages)); };
+      auto issue_qk = [&](uint32_t d, uint64_t dq, int i) {
+        const uint64_t dk = dk0 + (uint64_t)(((i % C::kStages) * C::kTileBytes) >> 4);
+        if constexpr (HD == 128)
+          mma_ss_chain8(d, dq, dk, C::kIdescQK, 0u);
+        else
+          mma_ss_chain4(d, dq, dk, C::kIdescQK, 0u);
       };
-      auto issue_pv = [&](uint32_t d, uint32_t p_tmem, uint32_t v_smem, bool acc) {
-#pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk) {
-          mma_ts(d, p_tmem + kk * 8, smem_desc_sw128(v_smem + kk * 2048, kBN * 128, 1024),
-                 C::kIdescPV, (acc || kk > 0) ? 1u : 0u);
-        }
+      auto issue_pv = [&](uint32_t d, uint32_t p_tmem, int i, bool acc) {
+        const uint64_t dv = dv0 + (uint64_t)(((i % C::kStages) * C::kTileBytes) >> 4);
+        mma_ts_chain8(d, p_tmem, dv, C::kIdescPV, acc ? 1u : 0u);
       };
       bool ok = true;
       if (n1 > 0) {
@@ -280,11 +312,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (ok && n1 > 0) {
         tc_fence_after();
         if (n0 > 0) {
-          issue_qk(S0, sQ, kv_smem(0));
+          issue_qk(S0, dq0, 0);
           mma_commit(bar_addr(&bars->s_full[0]));
         }
         if (has1) {
-          issue_qk(S1, sQ + C::kTileBytes, kv_smem(0));
+          issue_qk(S1, dq1, 0);
           mma_commit(bar_addr(&bars->s_full[1]));
         }
         release(0);
@@ -296,7 +328,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (j < n0) {
           if (!(ok = wait_bar(bar_addr(&bars->p_ready[0]), j & 1, abort, a.status))) break;
           tc_fence_after();
-          issue_pv(O0, S0, kv_smem(iv), j > 0);
+          issue_pv(O0, S0, iv, j > 0);
           if (j == n0 - 1) mma_commit(bar_addr(&bars->o_done[0]));
         }
         const bool next = j + 1 < n1;
@@ -304,20 +336,20 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!(ok = full(ik))) break;
           tc_fence_after();
           if (j + 1 < n0) {
-            issue_qk(S0, sQ, kv_smem(ik));
+            issue_qk(S0, dq0, ik);
             mma_commit(bar_addr(&bars->s_full[0]));
           }
         }
         if (has1) {
           if (!(ok = wait_bar(bar_addr(&bars->p_ready[1]), j & 1, abort, a.status))) break;
           tc_fence_after();
-          issue_pv(O1, S1, kv_smem(iv), j > 0);
+          issue_pv(O1, S1, iv, j > 0);
           if (j == n1 - 1) mma_commit(bar_addr(&bars->o_done[1]));
         }
         release(iv);
         if (next) {
           if (has1) {
-            issue_qk(S1, sQ + C::kTileBytes, kv_smem(ik));
+            issue_qk(S1, dq1, ik);
             mma_commit(bar_addr(&bars->s_full[1]));
           }
           release(ik);
@@ -360,14 +392,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int c = 0; c < kBN; ++c)
             if (kbase + c >= lim) s[c >> 5][c & 31] = -INFINITY;
         }
+        // row max: a tree of 3-input maxima over the 128 scores
         float mx[8];
 #pragma unroll
-        for (int x = 0; x < 8; ++x) mx[x] = s[x >> 1][(x & 1) * 16];
-#pragma unroll
-        for (int c = 0; c < kBN; ++c)
-          if ((c & 15) != 0) mx[c >> 4] = fmaxf(mx[c >> 4], s[c >> 5][c & 31]);
-        const float tmax = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                                 fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+        for (int x = 0; x < 8; ++x) {
+          const float* v = &s[x >> 1][(x & 1) * 16];
+          const float a0 = fmax3(v[0], v[1], v[2]), a1 = fmax3(v[3], v[4], v[5]);
+          const float a2 = fmax3(v[6], v[7], v[8]), a3 = fmax3(v[9], v[10], v[11]);
+          const float a4 = fmax3(v[12], v[13], v[14]);
+          mx[x] = fmax3(fmax3(a0, a1, a2), fmax3(a3, a4, v[15]), a0);
+        }
+        const float tmax = fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]),
+                                 fmaxf(mx[6], mx[7]));
         mraw = fmaxf(mraw, tmax);
         const float tmax2 = tmax * scale_log2;
         bool bump = tmax2 > m + kRescaleThreshold;  // also true for the first finite max
@@ -378,16 +414,25 @@ __global__ void __launch_bounds__(kThreads, 1)
           l *= corr;
         }
         const float muse = m == -INFINITY ? 0.f : m;
-        float rs[4] = {0.f, 0.f, 0.f, 0.f};
+        // P = 2^(s * scale_log2 - m) with packed (two-lane) FMA and add; exp2 on the MUFU unit
+        // (and, for one pair in kEmuEvery, on the FMA pipe).
+        float2 rs[4] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
+        const float2 sc2 = make_float2(scale_log2, scale_log2), nm2 = make_float2(-muse, -muse);
         uint32_t pk[2][32];
 #pragma unroll
         for (int c = 0; c < kBN; c += 2) {
-          const float p0 = ex2(fmaf(s[c >> 5][c & 31], scale_log2, -muse));
-          const float p1 = ex2(fmaf(s[c >> 5][(c + 1) & 31], scale_log2, -muse));
-          rs[(c >> 1) & 3] += p0 + p1;
+          const float2 x = __ffma2_rn(make_float2(s[c >> 5][c & 31], s[c >> 5][(c + 1) & 31]), sc2, nm2);
+          float p0, p1;
+          if (kEmuEvery > 0 && ((c >> 1) % (kEmuEvery > 0 ? kEmuEvery : 1)) == kEmuEvery - 1) {
+            exp2_poly2(x.x, x.y, p0, p1);
+          } else {
+            p0 = ex2(x.x);
+            p1 = ex2(x.y);
+          }
+          rs[(c >> 1) & 3] = __fadd2_rn(rs[(c >> 1) & 3], make_float2(p0, p1));
           pk[c >> 6][(c >> 1) & 31] = pack_bf16x2(p0, p1);
         }
-        l += (rs[0] + rs[1]) + (rs[2] + rs[3]);
+        l += ((rs[0].x + rs[0].y) + (rs[1].x + rs[1].y)) + ((rs[2].x + rs[2].y) + (rs[3].x + rs[3].y));
         // rescale O (complete up to tile j-1: the S_j commit covers every earlier MMA)
         if (__any_sync(0xffffffffu, bump && j > 0)) {
           const float f = (bump && j > 0) ? corr : 1.f;
@@ -405,7 +450,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_st32(S + 32, pk[1]);
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(bar_addr(&bars->p_ready[q]));
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_addr(&bars->p_ready[q]));
       }
     }
     // ---- epilogue: O / l -> bf16, statistics ------------------------------------------------

@@ -52,6 +52,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Same, but the waiting thread may be suspended by the hardware for up to `suspend_ns` (it wakes
+// as soon as the phase completes) instead of spinning; waiting warps then leave the issue slots
+// and the shared-memory pipe to the warps doing work.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity, uint32_t suspend_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(suspend_ns)
+      : "memory");
+  return ok != 0;
+}
+
 // ---------------------------------------------------------------------------------------------
 // TMA (no multicast)
 // ---------------------------------------------------------------------------------------------
@@ -156,6 +171,61 @@ __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_
       "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
+// One whole K loop of MMAs issued from a single asm block (no per-MMA setup beyond a 32-bit add
+// on the descriptor's start-address word), so that the issuing thread keeps ahead of the tensor
+// core even when it shares its scheduler with busy softmax warps.
+//   mma_ss_chain: D (+)= A B^T, both K-major with 128-byte swizzle; K = 16 * steps. The start
+//   address advances 32 B per step inside a 128-byte atom and by `box_off` (16-byte units) every
+//   4 steps (the next 64-element TMA box).
+//   mma_ts_chain: D (+)= A B, A (P) in TMEM advancing 8 columns per step, B (V) MN-major,
+//   advancing `b_step` (16-byte units) per step.
+#define SDPA_MMA_SS_STEP(OFF)                                       \
+  "add.u32 x, alo, " #OFF ";\n\tadd.u32 y, blo, " #OFF ";\n\t"      \
+  "mov.b64 a, {x, ahi};\n\tmov.b64 b, {y, bhi};\n\t"                \
+  "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, t;\n\t"
+__device__ __forceinline__ void mma_ss_chain8(uint32_t d, uint64_t da, uint64_t db, uint32_t idesc,
+                                              uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p, t;\n\t.reg .b64 a, b;\n\t.reg .b32 alo, ahi, blo, bhi, x, y;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\tsetp.ne.b32 t, %5, 0;\n\t"
+      "mov.b64 {alo, ahi}, %1;\n\tmov.b64 {blo, bhi}, %2;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t"
+      SDPA_MMA_SS_STEP(2) SDPA_MMA_SS_STEP(4) SDPA_MMA_SS_STEP(6)
+      SDPA_MMA_SS_STEP(1024) SDPA_MMA_SS_STEP(1026) SDPA_MMA_SS_STEP(1028) SDPA_MMA_SS_STEP(1030)
+      "}" ::"r"(d), "l"(da), "l"(db), "r"(idesc), "r"(acc), "r"(1u)
+      : "memory");
+}
+__device__ __forceinline__ void mma_ss_chain4(uint32_t d, uint64_t da, uint64_t db, uint32_t idesc,
+                                              uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p, t;\n\t.reg .b64 a, b;\n\t.reg .b32 alo, ahi, blo, bhi, x, y;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\tsetp.ne.b32 t, %5, 0;\n\t"
+      "mov.b64 {alo, ahi}, %1;\n\tmov.b64 {blo, bhi}, %2;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t"
+      SDPA_MMA_SS_STEP(2) SDPA_MMA_SS_STEP(4) SDPA_MMA_SS_STEP(6)
+      "}" ::"r"(d), "l"(da), "l"(db), "r"(idesc), "r"(acc), "r"(1u)
+      : "memory");
+}
+#undef SDPA_MMA_SS_STEP
+#define SDPA_MMA_TS_STEP(K)                                                 \
+  "add.u32 x, %1, " #K "*8;\n\tadd.u32 y, blo, " #K "*128;\n\t"             \
+  "mov.b64 b, {y, bhi};\n\t"                                                  \
+  "tcgen05.mma.cta_group::1.kind::f16 [%0], [x], b, %3, t;\n\t"
+// 8 steps of 16 keys: A columns +8 per step, B start address +2048 B (128 units) per step.
+__device__ __forceinline__ void mma_ts_chain8(uint32_t d, uint32_t a_tmem, uint64_t db, uint32_t idesc,
+                                              uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p, t;\n\t.reg .b64 b;\n\t.reg .b32 blo, bhi, x, y;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\tsetp.ne.b32 t, %5, 0;\n\t"
+      "mov.b64 {blo, bhi}, %2;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t"
+      SDPA_MMA_TS_STEP(1) SDPA_MMA_TS_STEP(2) SDPA_MMA_TS_STEP(3) SDPA_MMA_TS_STEP(4)
+      SDPA_MMA_TS_STEP(5) SDPA_MMA_TS_STEP(6) SDPA_MMA_TS_STEP(7)
+      "}" ::"r"(d), "r"(a_tmem), "l"(db), "r"(idesc), "r"(acc), "r"(1u)
+      : "memory");
+}
+#undef SDPA_MMA_TS_STEP
+
 // Arrive once on `bar` when every tcgen05 operation issued so far by this thread has finished.
 __device__ __forceinline__ void mma_commit(uint32_t bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
@@ -189,6 +259,25 @@ __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// Packed fp32 pairs (sm_100 f32x2 instructions, through the CUDA builtins so that the compiler
+// allocates the register pairs): one issue slot for two lanes of work.
+__device__ __forceinline__ void ffma2(float a0, float a1, float b0, float b1, float c0, float c1,
+                                      float& d0, float& d1) {
+  const float2 r = __ffma2_rn(make_float2(a0, a1), make_float2(b0, b1), make_float2(c0, c1));
+  d0 = r.x;
+  d1 = r.y;
+}
+__device__ __forceinline__ void fadd2(float a0, float a1, float b0, float b1, float& d0, float& d1) {
+  const float2 r = __fadd2_rn(make_float2(a0, a1), make_float2(b0, b1));
+  d0 = r.x;
+  d1 = r.y;
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
