@@ -42,9 +42,10 @@ from scaled_dot_product_16_b200 import workloads as W  # noqa: E402
 METRIC = "attn fwd TFLOP/s & % of BF16 tensor peak; attn_merge HBM GB/s & % of peak"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
-# DRAM traffic of one attn_fwd launch on the varlen workload, from an ncu capture (see
-# profiles/); valid only for the kernel source it was measured on.
-TRAFFIC = {"kernel_sha": None, "bytes_per_launch": None}
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one attn_fwd launch on the
+# full varlen workload, from a one-pass ncu capture (profiles/attn_fwd_bf16_varlen.md); it is
+# reported only while the kernel source still has the hash it was measured on.
+TRAFFIC = {"kernel_sha": "22e5c2d45f4a957d", "bytes_per_launch": 938_170_000 + 601_440_000}
 
 
 def kernel_sha() -> str:
