@@ -51,7 +51,7 @@ def _bind(path: str):
     lib.oracle_attn_fwd_rows.restype = I
     lib.oracle_sparse_csr.argtypes = [P, P, P, I, P, P, I, I, I, I, I64, P]
     lib.oracle_sparse_csr.restype = I
-    lib.oracle_merge.argtypes = [P, P, P, P, P, P, I, I, I, I, I, P, P, P]
+    lib.oracle_merge.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, P, P, P]
     lib.oracle_merge.restype = I
     lib.oracle_round_bf16_array.argtypes = [P, I64, P]
     lib.oracle_round_bf16_array.restype = None
@@ -98,6 +98,8 @@ def _elem(x) -> Tuple[np.ndarray, int]:
             x = x.detach().cpu().contiguous()
             if x.dtype == torch.bfloat16:
                 return x.view(torch.int16).numpy().view(np.uint16), BF16
+            if x.dtype == torch.float16:
+                return x.numpy().astype(np.float64), F64  # exact widening
             x = x.numpy()
     except ImportError:  # pragma: no cover
         pass
@@ -189,17 +191,24 @@ def sparse_csr(q, k, v, offset, columns, *, B: int, H: int, S: int, D: int):
     return out
 
 
-def merge(prev_out, prev_max, prev_sum, cur_out, cur_max, cur_sum, *, S: int, B: int, N: int, D: int):
-    """Ring-attention update, SBH layout. Returns (out float64 [S,B,N*D], max, sum [B,N,S,8])."""
+def merge(prev_out, prev_max, prev_sum, cur_out, cur_max, cur_sum, *, S: int, B: int, N: int, D: int,
+          layout: int = BHSD):
+    """Ring-attention update. layout BHSD (the page's SBH): out [S,B,N*D], stats [B,N,S,8];
+    layout TND: out [T,N*D] with T = S, stats [T,N,8]. Returns (out float64, max, sum)."""
     lib = _load()
     (po, co), et = _same_type(prev_out, cur_out)
     stats = [np.ascontiguousarray(_widen(*_elem(x)), dtype=np.float64)
              for x in (prev_max, prev_sum, cur_max, cur_sum)]
-    out = np.zeros((S, B, N * D))
-    om = np.zeros((B, N, S, 8))
-    osum = np.zeros((B, N, S, 8))
+    if layout == BHSD:
+        out = np.zeros((S, B, N * D))
+        om = np.zeros((B, N, S, 8))
+    else:
+        out = np.zeros((S, N * D))
+        om = np.zeros((S, N, 8))
+    osum = np.zeros_like(om)
     rc = lib.oracle_merge(_ptr(po), _ptr(stats[0]), _ptr(stats[1]), _ptr(co), _ptr(stats[2]),
-                          _ptr(stats[3]), et, S, B, N, D, _ptr(out), _ptr(om), _ptr(osum))
+                          _ptr(stats[3]), et, S, B, N, D, int(layout), _ptr(out), _ptr(om),
+                          _ptr(osum))
     if rc != 0:
         raise ValueError(f"oracle_merge rejected its arguments (code {rc})")
     return out, om, osum

@@ -284,26 +284,39 @@ int oracle_sparse_csr(const void *q, const void *k, const void *v, int et, const
 }
 
 /*
- * Ring-attention partial merge ("npu_ring_attention_update", 小算子等价计算逻辑), SBH layout:
- * prev_out / cur_out [S, B, N*D]; statistics [B, N, S, 8] (float32 values in double here).
- * Lane-wise over the 8 statistic lanes:
+ * Ring-attention partial merge ("npu_ring_attention_update", 小算子等价计算逻辑 and 前向接口).
+ * Lane-wise over the 8 statistic lanes of each row:
  *     m = max(pm, cm), ps' = ps * exp(pm - m), cs' = cs * exp(cm - m), l = ps' + cs'.
- * Output: out = prev * (ps'[0] / l[0]) + cur * (cs'[0] / l[0]) with lane 0 of each row,
- * in double (the caller rounds to the output type).
+ * Output: out = prev * (ps'[0] / l[0]) + cur * (cs'[0] / l[0]) with lane 0 of each row, in
+ * double (the caller rounds to the output type).
+ * Layouts (layout argument):
+ *   ORC_BHSD ("SBH" on the page): outputs [S, B, N*D], statistics [B, N, S, 8];
+ *   ORC_TND: outputs [T, N*D] with T = S (B unused), statistics [T, N, 8] (token-major, as
+ *            the TND tensors themselves).
  * Where both maxima are -inf (both sides empty) the lane gives m = -inf, ps' = cs' = 0, l = 0,
  * and where the lane-0 sum l is 0 the output scales are 0 (the plain formula would divide
  * 0 by 0).
  */
 int oracle_merge(const void *prev_out, const double *prev_max, const double *prev_sum,
                  const void *cur_out, const double *cur_max, const double *cur_sum, int et,
-                 int S, int B, int N, int D, double *out, double *out_max, double *out_sum) {
-  int64_t row, nrows = (int64_t)B * N * S;
-  if (S < 0 || B < 0 || N <= 0 || D <= 0) return -1;
+                 int S, int B, int N, int D, int layout, double *out, double *out_max,
+                 double *out_sum) {
+  int64_t row, nrows;
+  if (S < 0 || N <= 0 || D <= 0) return -1;
+  if (layout == ORC_BHSD && B < 0) return -1;
+  nrows = layout == ORC_BHSD ? (int64_t)B * N * S : (int64_t)S * N;
 #pragma omp parallel for schedule(static)
   for (row = 0; row < nrows; ++row) {
-    /* row = (b * N + n) * S + s, the statistics' own order */
-    int64_t s = row % S, bn = row / S, n = bn % N, b = bn / N, lane, d;
+    int64_t lane, d, obase;
     double ps_scaled[8], cs_scaled[8], l[8], po, co;
+    if (layout == ORC_BHSD) {
+      /* row = (b * N + n) * S + s, the statistics' own order; output (s, b, n*D + d) */
+      int64_t s = row % S, bn = row / S, n = bn % N, b = bn / N;
+      obase = ((s * B + b) * N + n) * (int64_t)D;
+    } else {
+      /* row = t * N + n for both the statistics and the output */
+      obase = row * (int64_t)D;
+    }
     for (lane = 0; lane < 8; ++lane) {
       int64_t x = row * 8 + lane;
       double pm = prev_max[x], cm = cur_max[x];
@@ -322,8 +335,7 @@ int oracle_merge(const void *prev_out, const double *prev_max, const double *pre
     po = l[0] != 0.0 ? ps_scaled[0] / l[0] : 0.0;
     co = l[0] != 0.0 ? cs_scaled[0] / l[0] : 0.0;
     for (d = 0; d < D; ++d) {
-      /* [S, B, N*D]: element (s, b, n*D + d) */
-      int64_t x = ((s * B + b) * N + n) * (int64_t)D + d;
+      int64_t x = obase + d;
       out[x] = ld(prev_out, x, et) * po + ld(cur_out, x, et) * co;
     }
   }

@@ -408,6 +408,54 @@ def pin_merge_order_independent():
         assert np.max(np.abs(x - y)) <= 1e-12
 
 
+def pin_merge_tnd_matches_sbh_relayout():
+    """The TND merge ([T, N*D] outputs, [T, N, 8] statistics) equals the SBH merge of the same
+    rows laid out as B = 1 ([T, 1, N*D] outputs, [1, N, T, 8] statistics)."""
+    r = _rng(34)
+    T, N, D = 7, 3, 4
+    po, co = r.standard_normal((T, N * D)), r.standard_normal((T, N * D))
+    pm, cm = r.standard_normal((T, N, 8)), r.standard_normal((T, N, 8))
+    ps, cs = 1 + np.abs(r.standard_normal((T, N, 8))), 1 + np.abs(r.standard_normal((T, N, 8)))
+    tnd = oracle.merge(po, pm, ps, co, cm, cs, S=T, B=1, N=N, D=D, layout=TND)
+    to_sbh = lambda x: np.ascontiguousarray(np.transpose(x, (1, 0, 2))[None])  # [T,N,8] -> [1,N,T,8]
+    sbh = oracle.merge(po[:, None], to_sbh(pm), to_sbh(ps), co[:, None], to_sbh(cm), to_sbh(cs),
+                       S=T, B=1, N=N, D=D, layout=BHSD)
+    assert np.array_equal(tnd[0], sbh[0][:, 0])
+    assert np.array_equal(tnd[1], np.transpose(sbh[1][0], (1, 0, 2)))
+    assert np.array_equal(tnd[2], np.transpose(sbh[2][0], (1, 0, 2)))
+
+
+def pin_merge_tnd_chunks_equal_full_varlen():
+    """Varlen attention over two key chunks of every sequence, merged in TND layout, equals
+    attention over all keys."""
+    r = _rng(35)
+    lens = np.array([5, 0, 9, 3])
+    cu = W.cu_seqlens_from_lengths(lens)
+    T, Nq, Nkv, D = int(cu[-1]), 4, 2, 3
+    q = r.standard_normal((T, Nq, D))
+    k = r.standard_normal((T, Nkv, D)) * 2
+    v = r.standard_normal((T, Nkv, D))
+    kw = dict(Nq=Nq, Nkv=Nkv, D=D, scale=0.4, mask_mode=NONE, layout=TND)
+    full, fm, fl = oracle.attn_fwd(q, k, v, cu_q=cu, cu_kv=cu, B=len(lens), Sq=T, Skv=T, **kw)
+    starts = np.concatenate([[0], cu[:-1]])
+    parts = []
+    for half in range(2):
+        idx, lk = [], []
+        for s0, L in zip(starts, lens):
+            a, b = (0, L // 2) if half == 0 else (L // 2, L)
+            idx.extend(range(s0 + a, s0 + b))
+            lk.append(b - a)
+        idx = np.array(idx, dtype=np.int64)
+        ck = W.cu_seqlens_from_lengths(lk)
+        o, m, l = oracle.attn_fwd(q, k[idx], v[idx], cu_q=cu, cu_kv=ck, B=len(lens), Sq=T,
+                                  Skv=int(ck[-1]), **kw)
+        parts.append((o.reshape(T, Nq * D), np.repeat(m[..., None], 8, -1), np.repeat(l[..., None], 8, -1)))
+    out, om, ol = oracle.merge(*parts[0], *parts[1], S=T, B=0, N=Nq, D=D, layout=TND)
+    assert np.max(np.abs(out - full.reshape(T, Nq * D))) <= 1e-12
+    assert np.max(np.abs(om[..., 0] - fm)) <= 1e-13
+    assert np.max(np.abs(ol[..., 0] / fl - 1)) <= 1e-12
+
+
 # ---------------------------------------------------------------------------------------------
 # bf16 rounding
 # ---------------------------------------------------------------------------------------------

@@ -38,7 +38,8 @@ MUTANTS = [
     ("merge_exp_sign", "prev_sum[x] * exp(pm - m)", "prev_sum[x] * exp(m - pm)", 0),
     ("merge_uses_lane_1", "po = l[0] != 0.0 ? ps_scaled[0] / l[0] : 0.0;",
      "po = l[1] != 0.0 ? ps_scaled[1] / l[1] : 0.0;", 0),
-    ("merge_bsh_indexing", "((s * B + b) * N + n) * (int64_t)D + d", "((b * S + s) * N + n) * (int64_t)D + d", 0),
+    ("merge_bsh_indexing", "obase = ((s * B + b) * N + n) * (int64_t)D;", "obase = ((b * S + s) * N + n) * (int64_t)D;", 0),
+    ("merge_tnd_head_major", "obase = row * (int64_t)D;", "obase = ((row % N) * S + row / N) * (int64_t)D;", 0),
     ("merge_swapped_sides", "ld(prev_out, x, et) * po + ld(cur_out, x, et) * co",
      "ld(prev_out, x, et) * co + ld(cur_out, x, et) * po", 0),
     ("merge_sum_not_rescaled", "cs_scaled[lane] = cur_sum[x] * exp(cm - m);", "cs_scaled[lane] = cur_sum[x];", 0),
