@@ -53,7 +53,7 @@ typedef enum {
   ATTN_ERR_TIMEOUT = 5      /* device-side: a pipeline wait exceeded its bound          */
 } attn_status;
 
-typedef enum { ATTN_BF16 = 0, ATTN_F32 = 1 } attn_dtype;
+typedef enum { ATTN_BF16 = 0, ATTN_F32 = 1, ATTN_F16 = 2 } attn_dtype;
 
 typedef enum { ATTN_BHSD = 0, ATTN_TND = 1 } attn_layout;
 
@@ -82,13 +82,15 @@ typedef enum {
  *   occupies tokens [cu[b-1], cu[b]) with cu[-1] = 0, and cu[B-1] must equal the total.
  *   Lengths [2,2,0,2,2] are passed as [2,4,4,6,8]; zero-length sequences are allowed.
  * GQA/MQA: query head h reads key/value head h / (Nq / Nkv); Nq must be a multiple of Nkv.
- * dtype: ATTN_BF16 (q, k, v, out bfloat16; fp32 accumulation; D = 64 or 128) or
- *        ATTN_F32 (float32 throughout, CUDA-core FMA; 1 <= D <= 256).
+ * dtype: ATTN_BF16 or ATTN_F16 (q, k, v, out bfloat16 or float16; tensor cores with fp32
+ *        accumulation; D = 64 or 128), or ATTN_F32 (float32 throughout, CUDA-core FMA;
+ *        1 <= D <= 256).
  * softmax_max / softmax_sum may both be NULL to skip the statistics.
  * Limits (from the constraints): 1 <= Nq <= 256, D <= 768 (larger D is ATTN_ERR_INVALID;
  * sizes this build does not run are ATTN_ERR_UNSUPPORTED), Tq, Tkv <= 1M tokens and
- * B <= 2048 for TND. Empty problems (B = 0, Sq = 0 or a total of 0 tokens) return ATTN_OK
- * without a launch. For ATTN_BF16, q, k, v and out must be 16-byte aligned.
+ * B <= 2048 for TND; scale must be finite and > 0. Empty problems (B = 0, Sq = 0 or a total
+ * of 0 tokens) return ATTN_OK without a launch. For ATTN_BF16 and ATTN_F16, q, k, v and out
+ * must be 16-byte aligned.
  * Data errors: cumulative lengths that decrease or do not end at the totals set ATTN_ERR_DATA
  * in the status word; the affected outputs are not written.
  */
@@ -130,10 +132,17 @@ ATTN_API int attn_sparse_csr(const float* q, const float* k, const float* v,
  * computed in float32 and rounded once (to nearest even) to the output type.
  *
  * layout = ATTN_BHSD means the page's "SBH" layout:
- *   prev_out, cur_out, out     [S, B, N*D] of `dtype` (ATTN_BF16 or ATTN_F32)
+ *   prev_out, cur_out, out     [S, B, N*D] of `dtype` (ATTN_BF16, ATTN_F16 or ATTN_F32)
  *   prev_/cur_/out_ max, sum   float32 [B, N, S, 8]
- * layout = ATTN_TND is not run by this build (ATTN_ERR_UNSUPPORTED); actual_seq_qlen is
- * reserved for it and must be NULL.
+ *   actual_seq_qlen must be NULL.
+ * layout = ATTN_TND (packed tokens; S is the total token count T):
+ *   prev_out, cur_out, out     [T, N*D] of `dtype`
+ *   prev_/cur_/out_ max, sum   float32 [T, N, 8] (token-major, like the TND tensors)
+ *   actual_seq_qlen            NULL, or a device int64 array of B cumulative query lengths
+ *                              (no leading zero, as attn_fwd's cu_seqlens). The merge is per
+ *                              token, so the lengths only fix T: if they decrease or do not
+ *                              end at T the status word records ATTN_ERR_DATA (the merge still
+ *                              runs over all T tokens).
  * A lane whose two maxima are both -inf (two empty partials) gives m = -inf, l = 0 and, on
  * lane 0, an output row of zeros; where the lane-0 l is 0 the output scales are 0.
  * Outputs may alias the prev_* inputs (in-place accumulation); no other overlap is allowed.

@@ -17,12 +17,12 @@ from typing import Optional
 
 __all__ = [
     "attn_fwd", "attn_sparse_csr", "attn_merge", "attn_get_last_error", "AttnError",
-    "ATTN_BF16", "ATTN_F32", "ATTN_BHSD", "ATTN_TND", "ATTN_MASK_NONE",
+    "ATTN_BF16", "ATTN_F32", "ATTN_F16", "ATTN_BHSD", "ATTN_TND", "ATTN_MASK_NONE",
     "ATTN_MASK_CAUSAL_TOPLEFT", "ATTN_MASK_CAUSAL_BOTTOMRIGHT", "lib_path", "load_library",
 ]
 
 ATTN_OK, ATTN_ERR_INVALID, ATTN_ERR_UNSUPPORTED, ATTN_ERR_CUDA, ATTN_ERR_DATA, ATTN_ERR_TIMEOUT = range(6)
-ATTN_BF16, ATTN_F32 = 0, 1
+ATTN_BF16, ATTN_F32, ATTN_F16 = 0, 1, 2
 ATTN_BHSD, ATTN_TND = 0, 1
 ATTN_MASK_NONE, ATTN_MASK_CAUSAL_TOPLEFT, ATTN_MASK_CAUSAL_BOTTOMRIGHT = 0, 1, 2
 

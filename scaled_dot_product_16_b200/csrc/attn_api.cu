@@ -71,7 +71,7 @@ int attn_fwd(const void* q, const void* k, const void* v, const int32_t* cu_seql
              float scale, int mask_mode, int dtype, int layout, void* out, float* softmax_max,
              float* softmax_sum, void* stream) {
   if (layout != ATTN_BHSD && layout != ATTN_TND) return ATTN_ERR_INVALID;
-  if (dtype != ATTN_BF16 && dtype != ATTN_F32) return ATTN_ERR_INVALID;
+  if (dtype != ATTN_BF16 && dtype != ATTN_F32 && dtype != ATTN_F16) return ATTN_ERR_INVALID;
   if (mask_mode < ATTN_MASK_NONE || mask_mode > ATTN_MASK_CAUSAL_BOTTOMRIGHT) return ATTN_ERR_INVALID;
   if (B < 0 || Sq < 0 || Skv < 0) return ATTN_ERR_INVALID;
   if (Nq < 1 || Nq > 256 || Nkv < 1 || Nq % Nkv != 0) return ATTN_ERR_INVALID;
@@ -89,7 +89,7 @@ int attn_fwd(const void* q, const void* k, const void* v, const int32_t* cu_seql
   if (q == nullptr || out == nullptr) return ATTN_ERR_INVALID;
   if (Skv > 0 && (k == nullptr || v == nullptr)) return ATTN_ERR_INVALID;
   if (dtype == ATTN_F32 && D > 256) return ATTN_ERR_UNSUPPORTED;
-  if (dtype == ATTN_BF16) {
+  if (dtype == ATTN_BF16 || dtype == ATTN_F16) {
     if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return ATTN_ERR_INVALID;
   }
@@ -109,6 +109,7 @@ int attn_fwd(const void* q, const void* k, const void* v, const int32_t* cu_seql
   a.scale = scale;
   a.mask_mode = mask_mode;
   a.layout = layout;
+  a.dtype = dtype;
   a.out = out;
   a.smax = softmax_max;
   a.ssum = softmax_sum;
@@ -152,13 +153,15 @@ int attn_merge(const void* prev_out, const float* prev_max, const float* prev_su
                const void* cur_out, const float* cur_max, const float* cur_sum, int S, int B,
                int N, int D, int dtype, int layout, const int64_t* actual_seq_qlen, void* out,
                float* out_max, float* out_sum, void* stream) {
-  if (dtype != ATTN_BF16 && dtype != ATTN_F32) return ATTN_ERR_INVALID;
+  if (dtype != ATTN_BF16 && dtype != ATTN_F32 && dtype != ATTN_F16) return ATTN_ERR_INVALID;
   if (layout != ATTN_BHSD && layout != ATTN_TND) return ATTN_ERR_INVALID;
   if (S < 0 || B < 0 || N < 1 || D < 1) return ATTN_ERR_INVALID;
-  if (layout == ATTN_TND) return ATTN_ERR_UNSUPPORTED;
-  if (actual_seq_qlen != nullptr) return ATTN_ERR_INVALID;
-  if ((int64_t)S * B == 0) return ATTN_OK;
-  if ((int64_t)B * N > 0x7fffffffLL || S > 65535LL * 32) return ATTN_ERR_UNSUPPORTED;
+  if (layout == ATTN_BHSD && actual_seq_qlen != nullptr) return ATTN_ERR_INVALID;
+  if (layout == ATTN_TND && actual_seq_qlen != nullptr && (B < 1 || B > kMaxCu)) return ATTN_ERR_INVALID;
+  const int64_t rows = layout == ATTN_TND ? (int64_t)S * N : (int64_t)S * B;
+  if (rows == 0) return ATTN_OK;
+  if (layout == ATTN_BHSD && ((int64_t)B * N > 0x7fffffffLL || S > 65535LL * 8)) return ATTN_ERR_UNSUPPORTED;
+  if (layout == ATTN_TND && rows > 0x7fffffffLL * 8) return ATTN_ERR_UNSUPPORTED;
   if (!prev_out || !prev_max || !prev_sum || !cur_out || !cur_max || !cur_sum || !out ||
       !out_max || !out_sum)
     return ATTN_ERR_INVALID;
@@ -174,9 +177,14 @@ int attn_merge(const void* prev_out, const float* prev_max, const float* prev_su
   a.N = N;
   a.D = D;
   a.dtype = dtype;
+  a.layout = layout;
+  a.seq_qlen = actual_seq_qlen;
   a.out = out;
   a.out_max = out_max;
   a.out_sum = out_sum;
+  int sms = 0;
+  int rc = device_state(&a.status, &sms);
+  if (rc != ATTN_OK) return rc;
   const cudaError_t e = sdpa::launch_merge(a, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }

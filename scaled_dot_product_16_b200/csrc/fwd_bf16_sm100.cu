@@ -1,4 +1,4 @@
-// fwd_bf16_sm100.cu -- fused attention forward for bf16 on B200 (sm_100a).
+// fwd_bf16_sm100.cu -- fused attention forward for bf16 (and fp16) on B200 (sm_100a).
 //
 // O = softmax(scale * Q K^T + mask) V with per-row softmax max / sum, for dense BHSD or packed
 // TND batches with GQA/MQA head ratios and causal masks ("aclnnFlashAttentionVarLenScore",
@@ -82,7 +82,7 @@ __device__ __forceinline__ void exp2_poly2(float x0, float x1, float& p0, float&
   p1 = x1 < -125.f ? 0.f : __uint_as_float(b1);
 }
 
-template <int HD>
+template <int HD, bool F16>
 struct Cfg {
   static constexpr int kBoxes = HD / 64;                 // 64-element (128-byte) TMA boxes
   static constexpr int kTileBytes = kBM * HD * 2;        // one Q, K or V tile
@@ -91,8 +91,9 @@ struct Cfg {
   static constexpr int kKVOff = 2 * kTileBytes;
   static constexpr int kBarOff = kKVOff + kStages * kTileBytes;
   static constexpr int kSmemBytes = kBarOff + 256 + 1024;  // barriers + 1 KB for alignment
-  static constexpr uint32_t kIdescQK = idesc_bf16_f32(kBM, kBN, 0, 0);
-  static constexpr uint32_t kIdescPV = idesc_bf16_f32(kBM, HD, 0, 1);
+  static constexpr uint32_t kFmt = F16 ? 0u : 1u;  // instruction-descriptor operand format
+  static constexpr uint32_t kIdescQK = idesc_f16_f32(kBM, kBN, 0, 0, kFmt);
+  static constexpr uint32_t kIdescPV = idesc_f16_f32(kBM, HD, 0, 1, kFmt);
 };
 
 struct Barriers {
@@ -132,12 +133,12 @@ struct Work {
   int row0;         // first row (within the sequence) of this block's 256 rows
 };
 
-template <int HD>
+template <int HD, bool F16>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, FwdArgs a, int units_per_seq,
                     float scale_log2) {
-  using C = Cfg<HD>;
+  using C = Cfg<HD, F16>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   Barriers* bars = reinterpret_cast<Barriers*>(smem + C::kBarOff);
@@ -430,7 +431,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             p1 = ex2(x.y);
           }
           rs[(c >> 1) & 3] = __fadd2_rn(rs[(c >> 1) & 3], make_float2(p0, p1));
-          pk[c >> 6][(c >> 1) & 31] = pack_bf16x2(p0, p1);
+          pk[c >> 6][(c >> 1) & 31] = pack16x2<F16>(p0, p1);
         }
         l += ((rs[0].x + rs[0].y) + (rs[1].x + rs[1].y)) + ((rs[2].x + rs[2].y) + (rs[3].x + rs[3].y));
         // rescale O (complete up to tile j-1: the S_j commit covers every earlier MMA)
@@ -461,7 +462,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (q == 0 || has1) {
       const bool store = r < rows;
       const bool bhsd = a.layout == ATTN_BHSD;
-      __nv_bfloat16* out = static_cast<__nv_bfloat16*>(a.out);
+      uint16_t* out = static_cast<uint16_t*>(a.out);  // bf16 or f16 bit patterns
       const int64_t orow = bhsd ? (((int64_t)w.b * a.Nq + w.h) * a.Sq + i) * HD
                                 : ((int64_t)(w.q0 + i) * a.Nq + w.h) * HD;
       const float inv = (l > 0.f && ok) ? 1.f / l : 0.f;
@@ -479,8 +480,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint32_t pkd[16];
 #pragma unroll
           for (int x = 0; x < 16; ++x)
-            pkd[x] = pack_bf16x2(inv == 0.f ? 0.f : __uint_as_float(o[2 * x]) * inv,
-                                 inv == 0.f ? 0.f : __uint_as_float(o[2 * x + 1]) * inv);
+            pkd[x] = pack16x2<F16>(inv == 0.f ? 0.f : __uint_as_float(o[2 * x]) * inv,
+                                   inv == 0.f ? 0.f : __uint_as_float(o[2 * x + 1]) * inv);
           uint4* dst = reinterpret_cast<uint4*>(out + orow + c * 32);
 #pragma unroll
           for (int x = 0; x < 4; ++x)
@@ -528,40 +529,42 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// 3-D map over a bf16 tensor viewed as (D, dim1, dim2), box (64, box1, box2), 128-byte swizzle.
+// 3-D map over a 16-bit tensor viewed as (D, dim1, dim2), box (64, box1, box2), 128-byte swizzle.
 bool make_map(CUtensorMap* m, const void* base, uint64_t D, uint64_t dim1, uint64_t dim2,
-              uint64_t stride1_bytes, uint64_t stride2_bytes, uint32_t box1, uint32_t box2) {
+              uint64_t stride1_bytes, uint64_t stride2_bytes, uint32_t box1, uint32_t box2,
+              bool f16) {
   EncodeTiledFn fn = encode_fn();
   if (fn == nullptr) return false;
   const cuuint64_t dims[3] = {D, dim1, dim2};
   const cuuint64_t strides[2] = {stride1_bytes, stride2_bytes};
   const cuuint32_t box[3] = {64, box1, box2};
   const cuuint32_t estr[3] = {1, 1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+  return fn(m, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+            const_cast<void*>(base), dims, strides, box,
             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int HD>
+template <int HD, bool F16>
 cudaError_t launch_hd(const FwdArgs& a, cudaStream_t st) {
-  using C = Cfg<HD>;
+  using C = Cfg<HD, F16>;
   CUtensorMap tq, tk, tv;
   const uint64_t D = HD;
   bool ok;
   if (a.layout == ATTN_BHSD) {
     // (d, s, b*h): rows of a head are contiguous
-    ok = make_map(&tq, a.q, D, a.Sq, (uint64_t)a.B * a.Nq, D * 2, (uint64_t)a.Sq * D * 2, kBM, 1) &&
-         make_map(&tk, a.k, D, a.Skv, (uint64_t)a.B * a.Nkv, D * 2, (uint64_t)a.Skv * D * 2, kBN, 1) &&
-         make_map(&tv, a.v, D, a.Skv, (uint64_t)a.B * a.Nkv, D * 2, (uint64_t)a.Skv * D * 2, kBN, 1);
+    ok = make_map(&tq, a.q, D, a.Sq, (uint64_t)a.B * a.Nq, D * 2, (uint64_t)a.Sq * D * 2, kBM, 1, F16) &&
+         make_map(&tk, a.k, D, a.Skv, (uint64_t)a.B * a.Nkv, D * 2, (uint64_t)a.Skv * D * 2, kBN, 1, F16) &&
+         make_map(&tv, a.v, D, a.Skv, (uint64_t)a.B * a.Nkv, D * 2, (uint64_t)a.Skv * D * 2, kBN, 1, F16);
   } else {
     // (d, head, token): a tile is 128 tokens of one head
     const uint64_t tq_rows = a.Sq > 0 ? a.Sq : 1, tk_rows = a.Skv > 0 ? a.Skv : 1;
-    ok = make_map(&tq, a.q, D, a.Nq, tq_rows, D * 2, (uint64_t)a.Nq * D * 2, 1, kBM) &&
-         make_map(&tk, a.k, D, a.Nkv, tk_rows, D * 2, (uint64_t)a.Nkv * D * 2, 1, kBN) &&
-         make_map(&tv, a.v, D, a.Nkv, tk_rows, D * 2, (uint64_t)a.Nkv * D * 2, 1, kBN);
+    ok = make_map(&tq, a.q, D, a.Nq, tq_rows, D * 2, (uint64_t)a.Nq * D * 2, 1, kBM, F16) &&
+         make_map(&tk, a.k, D, a.Nkv, tk_rows, D * 2, (uint64_t)a.Nkv * D * 2, 1, kBN, F16) &&
+         make_map(&tv, a.v, D, a.Nkv, tk_rows, D * 2, (uint64_t)a.Nkv * D * 2, 1, kBN, F16);
   }
   if (!ok) return cudaErrorInvalidValue;
-  cudaError_t e = cudaFuncSetAttribute(fwd_bf16_kernel<HD>,
+  cudaError_t e = cudaFuncSetAttribute(fwd_bf16_kernel<HD, F16>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return e;
   int units_per_seq = 0;
@@ -576,7 +579,7 @@ cudaError_t launch_hd(const FwdArgs& a, cudaStream_t st) {
   if (blocks <= 0) return cudaSuccess;
   if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
   const float scale_log2 = a.scale * 1.4426950408889634f;
-  fwd_bf16_kernel<HD><<<(unsigned)blocks, kThreads, C::kSmemBytes, st>>>(tq, tk, tv, a,
+  fwd_bf16_kernel<HD, F16><<<(unsigned)blocks, kThreads, C::kSmemBytes, st>>>(tq, tk, tv, a,
                                                                            units_per_seq, scale_log2);
   return cudaGetLastError();
 }
@@ -584,8 +587,9 @@ cudaError_t launch_hd(const FwdArgs& a, cudaStream_t st) {
 }  // namespace
 
 cudaError_t launch_fwd_bf16(const FwdArgs& a, cudaStream_t st) {
-  if (a.D == 128) return launch_hd<128>(a, st);
-  return launch_hd<64>(a, st);
+  const bool f16 = a.dtype == ATTN_F16;
+  if (a.D == 128) return f16 ? launch_hd<128, true>(a, st) : launch_hd<128, false>(a, st);
+  return f16 ? launch_hd<64, true>(a, st) : launch_hd<64, false>(a, st);
 }
 
 }  // namespace sdpa

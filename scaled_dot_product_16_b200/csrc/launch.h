@@ -14,7 +14,7 @@ struct FwdArgs {
   const int32_t* cu_kv;  // TND only
   int B, Sq, Skv, Nq, Nkv, D;
   float scale;
-  int mask_mode, layout;
+  int mask_mode, layout, dtype;
   void* out;
   float* smax;  // may be null (with ssum)
   float* ssum;
@@ -41,10 +41,12 @@ struct MergeArgs {
   const void* cur_out;
   const float* cur_max;
   const float* cur_sum;
-  int S, B, N, D, dtype;
+  int S, B, N, D, dtype, layout;
+  const int64_t* seq_qlen;  // TND only, may be null
   void* out;
   float* out_max;
   float* out_sum;
+  int* status;
 };
 
 cudaError_t launch_merge(const MergeArgs& a, cudaStream_t st);

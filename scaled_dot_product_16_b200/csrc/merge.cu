@@ -4,7 +4,8 @@
 //   m = max(pm, cm), ps' = ps * exp(pm - m), cs' = cs * exp(cm - m), l = ps' + cs',
 // and out = prev * (ps'_0 / l_0) + cur * (cs'_0 / l_0) with lane 0 of each (b, n, s) row.
 //
-// SBH layout: outputs [S, B, N*D]; statistics [B, N, S, 8] fp32.
+// SBH layout: outputs [S, B, N*D]; statistics [B, N, S, 8] fp32. TND layout: outputs
+// [T, N*D]; statistics [T, N, 8] fp32 (rows t*N + n, contiguous in both).
 //
 // The kernel is HBM-bound (about 1 GB moved per call at S=8192, B=4, N=32, D=128), so the
 // design is about access shape and bytes in flight only:
@@ -16,6 +17,8 @@
 //   * blocks are small (8 rows, 64 threads, 2 vectors per thread and input): in a sweep of
 //     block shapes on B200 this reached 79 % of the measured copy bandwidth, against 67 % for
 //     64-row blocks, because many small independent blocks keep more requests in flight.
+#include <cuda_fp16.h>
+
 #include "common.cuh"
 #include "launch.h"
 
@@ -45,12 +48,25 @@ template <>
 struct Vec16<float> {
   static constexpr int n = 4;
 };
+template <>
+struct Vec16<__half> {
+  static constexpr int n = 8;
+};
 
 __device__ __forceinline__ void unpack(const uint4& u, float* f, __nv_bfloat16*) {
   const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const float2 t = __bfloat1622float2(h[i]);
+    f[2 * i] = t.x;
+    f[2 * i + 1] = t.y;
+  }
+}
+__device__ __forceinline__ void unpack(const uint4& u, float* f, __half*) {
+  const __half2* h = reinterpret_cast<const __half2*>(&u);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 t = __half22float2(h[i]);
     f[2 * i] = t.x;
     f[2 * i + 1] = t.y;
   }
@@ -68,6 +84,13 @@ __device__ __forceinline__ uint4 pack(const float* f, __nv_bfloat16*) {
   for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(f[2 * i], f[2 * i + 1]);
   return u;
 }
+__device__ __forceinline__ uint4 pack(const float* f, __half*) {
+  uint4 u;
+  __half2* h = reinterpret_cast<__half2*>(&u);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) h[i] = __floats2half2_rn(f[2 * i], f[2 * i + 1]);
+  return u;
+}
 __device__ __forceinline__ uint4 pack(const float* f, float*) {
   return make_uint4(__float_as_uint(f[0]), __float_as_uint(f[1]), __float_as_uint(f[2]),
                     __float_as_uint(f[3]));
@@ -75,6 +98,8 @@ __device__ __forceinline__ uint4 pack(const float* f, float*) {
 
 __device__ __forceinline__ float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
 __device__ __forceinline__ float to_f(float x) { return x; }
+__device__ __forceinline__ float to_f(__half x) { return __half2float(x); }
+__device__ __forceinline__ void from_f(float x, __half* p) { *p = __float2half_rn(x); }
 __device__ __forceinline__ void from_f(float x, __nv_bfloat16* p) { *p = __float2bfloat16_rn(x); }
 __device__ __forceinline__ void from_f(float x, float* p) { *p = x; }
 
@@ -95,22 +120,24 @@ __device__ __forceinline__ void merge_lane(float pm, float ps, float cm, float c
 
 // Generic path: a block of ROWS = 32 rows loads the statistics, then the outputs.
 // VEC: true when D is a multiple of the 16-byte vector width and the row bases stay aligned.
-template <typename T, bool VEC>
+template <typename T, bool VEC, bool FLAT>
 __global__ void __launch_bounds__(kThreads) merge_sbh_kernel(
     const T* prev_out, const float* prev_max, const float* prev_sum,  // may alias the outputs
     const T* __restrict__ cur_out,
     const float* __restrict__ cur_max, const float* __restrict__ cur_sum, int S, int B, int N,
     int D, T* out, float* out_max, float* out_sum) {
   __shared__ float s_po[kRows], s_co[kRows];
-  const int bn = blockIdx.x;  // b * N + n
-  const int b = bn / N, n = bn - b * N;
-  const int s0 = blockIdx.y * kRows;
-  const int rows = min(kRows, S - s0);
+  // SBH: block (b*N + n, s-block); FLAT (TND): block = kRows consecutive rows t*N + n
+  const int bn = FLAT ? 0 : blockIdx.x;
+  const int b = FLAT ? 0 : bn / N, n = FLAT ? 0 : bn - b * N;
+  const int64_t s0 = FLAT ? (int64_t)blockIdx.x * kRows : (int64_t)blockIdx.y * kRows;
+  const int64_t nrow_all = FLAT ? (int64_t)S * N : (int64_t)S;
+  const int rows = (int)min((int64_t)kRows, nrow_all - s0);
 
   // ---- statistics: ROWS * 8 contiguous floats per array, one per thread ----------------
   {
     const int t = threadIdx.x;  // t = row * 8 + lane
-    const int64_t base = ((int64_t)bn * S + s0) * 8;
+    const int64_t base = FLAT ? s0 * 8 : ((int64_t)bn * S + s0) * 8;
     if (t < rows * 8) {
       const float pm = prev_max[base + t], ps = prev_sum[base + t];
       const float cm = cur_max[base + t], cs = cur_sum[base + t];
@@ -128,9 +155,9 @@ __global__ void __launch_bounds__(kThreads) merge_sbh_kernel(
   }
   __syncthreads();
 
-  // ---- outputs: row s is D contiguous elements at ((s*B + b)*N + n)*D -------------------
-  const int64_t row_stride = (int64_t)B * N * D;
-  const int64_t row0 = ((int64_t)s0 * B + b) * N * D + (int64_t)n * D;
+  // ---- outputs: SBH row s is D contiguous elements at ((s*B + b)*N + n)*D; FLAT row r at r*D
+  const int64_t row_stride = FLAT ? (int64_t)D : (int64_t)B * N * D;
+  const int64_t row0 = FLAT ? s0 * D : ((int64_t)s0 * B + b) * N * D + (int64_t)n * D;
   if constexpr (VEC) {
     constexpr int V = Vec16<T>::n;
     const int vpr = D / V;                  // vectors per row
@@ -182,7 +209,7 @@ __global__ void __launch_bounds__(kThreads) merge_sbh_kernel(
 // element read and written by the same thread, so the outputs may alias prev_*) and hands
 // the lane-0 output scales through shared memory. The barrier therefore overlaps the bulk
 // loads instead of preceding them.
-template <typename T, int ROWS, int THREADS, int PER>
+template <typename T, int ROWS, int THREADS, int PER, bool FLAT>
 __global__ void __launch_bounds__(THREADS) merge_sbh_vec_kernel(
     const T* prev_out, const float* prev_max, const float* prev_sum,  // may alias the outputs
     const T* __restrict__ cur_out, const float* __restrict__ cur_max,
@@ -190,14 +217,16 @@ __global__ void __launch_bounds__(THREADS) merge_sbh_vec_kernel(
     float* out_sum) {
   constexpr int V = Vec16<T>::n;
   __shared__ float s_po[ROWS], s_co[ROWS];
-  const int bn = blockIdx.x;  // b * N + n
-  const int b = bn / N, n = bn - b * N;
-  const int s0 = blockIdx.y * ROWS;
-  const int rows = min(ROWS, S - s0);
+  // SBH: block (b*N + n, s-block); FLAT (TND): block = ROWS consecutive rows t*N + n
+  const int bn = FLAT ? 0 : blockIdx.x;
+  const int b = FLAT ? 0 : bn / N, n = FLAT ? 0 : bn - b * N;
+  const int64_t s0 = FLAT ? (int64_t)blockIdx.x * ROWS : (int64_t)blockIdx.y * ROWS;
+  const int64_t nrow_all = FLAT ? (int64_t)S * N : (int64_t)S;
+  const int rows = (int)min((int64_t)ROWS, nrow_all - s0);
   const int vpr = D / V;  // vectors per row
   const int total = rows * vpr;
-  const int64_t row_stride = (int64_t)B * N * D;
-  const int64_t row0 = ((int64_t)s0 * B + b) * N * D + (int64_t)n * D;
+  const int64_t row_stride = FLAT ? (int64_t)D : (int64_t)B * N * D;
+  const int64_t row0 = FLAT ? s0 * D : ((int64_t)s0 * B + b) * N * D + (int64_t)n * D;
 
   // 1. bulk loads of the partial outputs, all in flight at once
   uint4 pv[PER], cv[PER];
@@ -212,7 +241,7 @@ __global__ void __launch_bounds__(THREADS) merge_sbh_vec_kernel(
     }
   }
   // 2. lane-wise statistics, one (row, lane) element per thread
-  const int64_t st0 = ((int64_t)bn * S + s0) * 8;
+  const int64_t st0 = FLAT ? s0 * 8 : ((int64_t)bn * S + s0) * 8;
   for (int t = threadIdx.x; t < rows * 8; t += THREADS) {
     const float pm = prev_max[st0 + t], ps = prev_sum[st0 + t];
     const float cm = cur_max[st0 + t], cs = cur_sum[st0 + t];
@@ -246,36 +275,68 @@ __global__ void __launch_bounds__(THREADS) merge_sbh_vec_kernel(
   }
 }
 
-template <typename T, int ROWS, int THREADS, int PER>
+template <typename T, int ROWS, int THREADS, int PER, bool FLAT>
 void launch_vec(const MergeArgs& a, cudaStream_t st) {
-  dim3 grid(a.B * a.N, (a.S + ROWS - 1) / ROWS);
-  merge_sbh_vec_kernel<T, ROWS, THREADS, PER><<<grid, THREADS, 0, st>>>(
+  const dim3 grid = FLAT ? dim3((unsigned)(((int64_t)a.S * a.N + ROWS - 1) / ROWS), 1)
+                         : dim3(a.B * a.N, (a.S + ROWS - 1) / ROWS);
+  merge_sbh_vec_kernel<T, ROWS, THREADS, PER, FLAT><<<grid, THREADS, 0, st>>>(
       (const T*)a.prev_out, a.prev_max, a.prev_sum, (const T*)a.cur_out, a.cur_max, a.cur_sum,
       a.S, a.B, a.N, a.D, (T*)a.out, a.out_max, a.out_sum);
 }
 
-template <typename T>
-cudaError_t launch_typed(const MergeArgs& a, cudaStream_t st) {
+template <typename T, bool FLAT>
+void launch_generic(const MergeArgs& a, bool vec, cudaStream_t st) {
+  const dim3 grid = FLAT ? dim3((unsigned)(((int64_t)a.S * a.N + kRows - 1) / kRows), 1)
+                         : dim3(a.B * a.N, (a.S + kRows - 1) / kRows);
+  if (vec)
+    merge_sbh_kernel<T, true, FLAT><<<grid, kThreads, 0, st>>>(
+        (const T*)a.prev_out, a.prev_max, a.prev_sum, (const T*)a.cur_out, a.cur_max, a.cur_sum,
+        a.S, a.B, a.N, a.D, (T*)a.out, a.out_max, a.out_sum);
+  else
+    merge_sbh_kernel<T, false, FLAT><<<grid, kThreads, 0, st>>>(
+        (const T*)a.prev_out, a.prev_max, a.prev_sum, (const T*)a.cur_out, a.cur_max, a.cur_sum,
+        a.S, a.B, a.N, a.D, (T*)a.out, a.out_max, a.out_sum);
+}
+
+template <typename T, bool FLAT>
+void launch_layout(const MergeArgs& a, cudaStream_t st) {
   constexpr int V = Vec16<T>::n;
   const bool vec = (a.D % V) == 0 && ((uintptr_t)a.prev_out % 16) == 0 &&
                    ((uintptr_t)a.cur_out % 16) == 0 && ((uintptr_t)a.out % 16) == 0;
   // tiny blocks (8 rows x 64 threads x 2 vectors) measured fastest: many independent blocks
   const int vpr = a.D / V;
   constexpr int R = SDPA_MERGE_ROWS, TH = SDPA_MERGE_THREADS, PR = SDPA_MERGE_PER;
-  if (vec && R * vpr <= PR * TH) {
-    launch_vec<T, R, TH, PR>(a, st);
-  } else if (vec && 16 * vpr <= 4 * 256) {
-    launch_vec<T, 16, 256, 4>(a, st);
+  if (vec && R * vpr <= PR * TH)
+    launch_vec<T, R, TH, PR, FLAT>(a, st);
+  else if (vec && 16 * vpr <= 4 * 256)
+    launch_vec<T, 16, 256, 4, FLAT>(a, st);
+  else
+    launch_generic<T, FLAT>(a, vec, st);
+}
+
+// Cumulative query lengths of a TND merge (int64, B entries, no leading zero): they only fix
+// the token count, so the check is that they never decrease and end at T.
+__global__ void check_seq_qlen_kernel(const int64_t* cu, int B, int64_t T, int* status) {
+  int64_t prev_end = 0;
+  bool bad = false;
+  for (int c0 = 0; c0 < B; c0 += 32) {
+    const int i = c0 + threadIdx.x;
+    const int64_t end = i < B ? cu[i] : 0;
+    int64_t start = __shfl_up_sync(0xffffffffu, end, 1);
+    if (threadIdx.x == 0) start = prev_end;
+    bad |= i < B && (end < start || (i == B - 1 && end != T));
+    prev_end = __shfl_sync(0xffffffffu, end, 31);
+  }
+  if (__any_sync(0xffffffffu, bad) && threadIdx.x == 0) report(status, ATTN_ERR_DATA);
+}
+
+template <typename T>
+cudaError_t launch_typed(const MergeArgs& a, cudaStream_t st) {
+  if (a.layout == ATTN_TND) {
+    if (a.seq_qlen != nullptr) check_seq_qlen_kernel<<<1, 32, 0, st>>>(a.seq_qlen, a.B, a.S, a.status);
+    launch_layout<T, true>(a, st);
   } else {
-    dim3 grid(a.B * a.N, (a.S + kRows - 1) / kRows);
-    if (vec)
-      merge_sbh_kernel<T, true><<<grid, kThreads, 0, st>>>(
-          (const T*)a.prev_out, a.prev_max, a.prev_sum, (const T*)a.cur_out, a.cur_max, a.cur_sum,
-          a.S, a.B, a.N, a.D, (T*)a.out, a.out_max, a.out_sum);
-    else
-      merge_sbh_kernel<T, false><<<grid, kThreads, 0, st>>>(
-          (const T*)a.prev_out, a.prev_max, a.prev_sum, (const T*)a.cur_out, a.cur_max, a.cur_sum,
-          a.S, a.B, a.N, a.D, (T*)a.out, a.out_max, a.out_sum);
+    launch_layout<T, false>(a, st);
   }
   return cudaGetLastError();
 }
@@ -284,6 +345,7 @@ cudaError_t launch_typed(const MergeArgs& a, cudaStream_t st) {
 
 cudaError_t launch_merge(const MergeArgs& a, cudaStream_t st) {
   if (a.dtype == ATTN_BF16) return launch_typed<__nv_bfloat16>(a, st);
+  if (a.dtype == ATTN_F16) return launch_typed<__half>(a, st);
   return launch_typed<float>(a, st);
 }
 

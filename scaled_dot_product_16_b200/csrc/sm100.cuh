@@ -244,8 +244,16 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr, uint32_t lbo,
   return d;
 }
 
-// Instruction descriptor for kind::f16 with bf16 A/B, fp32 D, dense.
+// Instruction descriptor for kind::f16 with 16-bit A/B (fmt 1 = bf16, 0 = f16), fp32 D, dense.
 // a_mn / b_mn: 1 when the operand is MN-major (contiguous along M or N) instead of K-major.
+__host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N, int a_mn, int b_mn, uint32_t fmt) {
+  return (1u << 4)                      // D format: f32
+         | (fmt << 7)                   // A format
+         | (fmt << 10)                  // B format
+         | ((uint32_t)a_mn << 15) | ((uint32_t)b_mn << 16)
+         | ((uint32_t)(N >> 3) << 17)   // N / 8
+         | ((uint32_t)(M >> 4) << 24);  // M / 16
+}
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int a_mn, int b_mn) {
   return (1u << 4)                      // D format: f32
          | (1u << 7)                    // A format: bf16
@@ -280,10 +288,29 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return d;
 }
 
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// Two fp32 values to a packed pair of 16-bit floats (round to nearest even).
+template <bool F16>
+__device__ __forceinline__ uint32_t pack16x2(float lo, float hi);
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
+}
+
+template <>
+__device__ __forceinline__ uint32_t pack16x2<false>(float lo, float hi) {
+  return pack_bf16x2(lo, hi);
+}
+template <>
+__device__ __forceinline__ uint32_t pack16x2<true>(float lo, float hi) {
+  return pack_f16x2(lo, hi);
 }
 
 }  // namespace sm100

@@ -28,7 +28,11 @@ import torch
 # Layout / mask / dtype codes, matching the values of the C header enums.
 BHSD, TND = 0, 1
 MASK_NONE, MASK_CAUSAL_TOPLEFT, MASK_CAUSAL_BOTTOMRIGHT = 0, 1, 2
-BF16, F32 = 0, 1
+BF16, F32, F16 = 0, 1, 2
+
+
+def dtype_code(dtype: torch.dtype) -> int:
+    return {torch.bfloat16: BF16, torch.float32: F32, torch.float16: F16}[dtype]
 
 
 def _gen(seed: int) -> torch.Generator:
@@ -120,7 +124,7 @@ def dense_bhsd(B, H, S, D, *, causal: bool, dtype: torch.dtype, seed: int, cfg: 
     k = randn((B, Hkv, Skv, D), mix_seed(cfg, seed, 1), dtype)
     v = randn((B, Hkv, Skv, D), mix_seed(cfg, seed, 2), dtype)
     return AttnInputs(q, k, v, BHSD, MASK_CAUSAL_TOPLEFT if causal else MASK_NONE,
-                      BF16 if dtype == torch.bfloat16 else F32, B, S, Skv, H, Hkv, D,
+                      dtype_code(dtype), B, S, Skv, H, Hkv, D,
                       1.0 / float(np.sqrt(D)))
 
 
@@ -135,7 +139,7 @@ def varlen_tnd(lengths_q, Nq, Nkv, D, *, causal: bool, dtype: torch.dtype, seed:
     v = randn((Tk, Nkv, D), mix_seed(cfg, seed, 2), dtype)
     if mask_mode is None:
         mask_mode = MASK_CAUSAL_TOPLEFT if causal else MASK_NONE
-    return AttnInputs(q, k, v, TND, mask_mode, BF16 if dtype == torch.bfloat16 else F32,
+    return AttnInputs(q, k, v, TND, mask_mode, dtype_code(dtype),
                       len(cu_q), Tq, Tk, Nq, Nkv, D, 1.0 / float(np.sqrt(D)), cu_q, cu_kv)
 
 

@@ -2,7 +2,7 @@
 float64 oracle under the stated tolerances.
 
 Tolerances (written here, used by every parity test):
-  * bf16 outputs: |gpu - exact| <= max(1e-2, one bf16 ulp of the exact value). The exact
+  * bf16 (and fp16) outputs: |gpu - exact| <= max(1e-2, one ulp of the exact value). The exact
     (float64) value is compared directly; a correctly rounded bf16 result is within half an
     ulp of it, and for |o| >= 4 half an ulp is already 1.6e-2, above 1e-2.
   * fp32 outputs: |gpu - exact| <= 1e-5.
@@ -31,11 +31,19 @@ def bf16_ulp(x: np.ndarray) -> np.ndarray:
     return np.exp2(e - 7)
 
 
+def f16_ulp(x: np.ndarray) -> np.ndarray:
+    ax = np.abs(x)
+    e = np.floor(np.log2(np.maximum(ax, 2.0 ** -14)))
+    return np.exp2(e - 10)
+
+
 def check_out(gpu: np.ndarray, ref: np.ndarray, dtype: int, what: str = "out") -> dict:
     gpu = gpu.astype(np.float64)
     err = np.abs(gpu - ref)
     if dtype == W.BF16:
         tol = np.maximum(BF16_ABS, bf16_ulp(ref))
+    elif dtype == W.F16:
+        tol = np.maximum(BF16_ABS, f16_ulp(ref))
     else:
         tol = np.full_like(ref, F32_ABS)
     bad = ~(err <= tol)

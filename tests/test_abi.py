@@ -84,6 +84,8 @@ def test_host_validation_without_gpu(lib):
     assert _fwd(lib, m=16) == INVALID                # max without sum
     assert _fwd(lib, q=None) == INVALID
     assert _fwd(lib, D=96) == UNSUP                  # bf16 runs D = 64 or 128
+    assert _fwd(lib, D=96, dtype=2) == UNSUP         # fp16 too
+    assert _fwd(lib, dtype=3) == INVALID
     assert _fwd(lib, q=18) == INVALID                # bf16 pointers must be 16-byte aligned
     assert _fwd(lib, layout=1, B=3) == INVALID       # TND needs cumulative lengths
     assert _fwd(lib, layout=1, B=2049, cq=16, ck=16) == INVALID
@@ -98,8 +100,10 @@ def test_host_validation_without_gpu(lib):
 def test_merge_and_csr_validation_without_gpu(lib):
     P = 16
     args = [P] * 6
-    assert lib.attn_merge(*args, 8, 1, 2, 64, 0, 1, None, P, P, P, None) == sdpa.ATTN_ERR_UNSUPPORTED
-    assert lib.attn_merge(*args, 8, 1, 2, 64, 0, 0, P, P, P, P, None) == sdpa.ATTN_ERR_INVALID
+    assert lib.attn_merge(*args, 8, 1, 2, 64, 3, 0, None, P, P, P, None) == sdpa.ATTN_ERR_INVALID  # dtype
+    assert lib.attn_merge(*args, 8, 1, 2, 64, 0, 0, P, P, P, P, None) == sdpa.ATTN_ERR_INVALID  # SBH + lengths
+    assert lib.attn_merge(*args, 8, 0, 2, 64, 0, 1, P, P, P, P, None) == sdpa.ATTN_ERR_INVALID  # TND, B = 0
+    assert lib.attn_merge(*args, 0, 0, 2, 64, 0, 1, None, P, P, P, None) == sdpa.ATTN_OK        # T = 0
     assert lib.attn_merge(*args, 8, 1, 0, 64, 0, 0, None, P, P, P, None) == sdpa.ATTN_ERR_INVALID
     assert lib.attn_merge(*args, 0, 1, 2, 64, 0, 0, None, P, P, P, None) == sdpa.ATTN_OK
     assert lib.attn_sparse_csr(P, P, P, P, P, 1, 1, 4, 0, 4, P, None) == sdpa.ATTN_ERR_INVALID

@@ -160,3 +160,26 @@ def test_host_validation():
     with pytest.raises(sdpa.AttnError) as e:
         sdpa.attn_fwd(q[..., 1:], k, v, **kw)  # misaligned base pointer
     assert e.value.status == sdpa.ATTN_ERR_INVALID
+
+
+# ---- fp16 on the tensor-core path ---------------------------------------------------------------
+F16 = torch.float16
+
+
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("causal", [False, True], ids=["full", "causal"])
+def test_f16_dense(D, causal):
+    _full_check(W.dense_bhsd(2, 3, 300, D, causal=causal, dtype=F16, seed=D, cfg=21))
+
+
+def test_f16_varlen_gqa():
+    _full_check(W.varlen_tnd([0, 700, 1, 257, 0, 513], 8, 2, 128, causal=True, dtype=F16, seed=4, cfg=22))
+
+
+def test_f16_matches_bf16_path_structure():
+    """Same inputs rounded to fp16 and to bf16: both paths agree with the exact result."""
+    base = W.dense_bhsd(1, 2, 200, 128, causal=True, dtype=torch.float32, seed=5, cfg=23)
+    for dt in (F16, BF):
+        inp = W.AttnInputs(base.q.to(dt), base.k.to(dt), base.v.to(dt), W.BHSD, W.MASK_CAUSAL_TOPLEFT,
+                           W.dtype_code(dt), 1, 200, 200, 2, 2, 128, base.scale)
+        _full_check(inp)

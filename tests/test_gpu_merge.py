@@ -132,3 +132,51 @@ def test_merge_chain_equals_full_attention_small():
 def test_merge_chain_cfg5_full_size():
     """Configuration 5: S=8192, B=4, N=32, D=128; Skv=8192 split into 4 chunks of 2048."""
     _merge_chain_check(4, 32, 8192, 8192, 128, seed=0, sampled=True)
+
+
+# ---- TND layout and fp16 ---------------------------------------------------------------------
+def _merge_tnd_gpu(po, pm, ps, co, cm, cs, T, N, D, dtype, seq_qlen=None, B=0):
+    dev = [t.cuda().contiguous() for t in (po, pm, ps, co, cm, cs)]
+    out, om, osum = torch.empty_like(dev[0]), torch.empty_like(dev[1]), torch.empty_like(dev[2])
+    sq = None if seq_qlen is None else torch.as_tensor(seq_qlen, dtype=torch.int64).cuda()
+    sdpa.attn_merge(*dev, S=T, B=B, N=N, D=D, dtype=dtype, out=out, out_max=om, out_sum=osum,
+                    layout=sdpa.ATTN_TND, actual_seq_qlen=sq)
+    return out.cpu(), om.cpu(), osum.cpu(), sdpa.attn_get_last_error()
+
+
+@pytest.mark.parametrize("dtype,tdt", [(W.BF16, torch.bfloat16), (W.F16, torch.float16), (W.F32, torch.float32)],
+                         ids=["bf16", "f16", "f32"])
+@pytest.mark.parametrize("T,N,D", [(1000, 4, 128), (37, 3, 40), (513, 12, 1)])
+def test_merge_tnd(dtype, tdt, T, N, D):
+    po = W.randn((T, N * D), 41, tdt)
+    co = W.randn((T, N * D), 42, tdt)
+    pm, ps = W.merge_stats_random(1, T, N, 43, lanes_equal=False)
+    cm, cs = W.merge_stats_random(1, T, N, 45, lanes_equal=False)
+    pm, ps, cm, cs = (x[0] for x in (pm, ps, cm, cs))  # [T, N, 8]
+    out, om, osum, st = _merge_tnd_gpu(po, pm, ps, co, cm, cs, T, N, D, dtype)
+    assert st == 0
+    ro, rm, rs = oracle.merge(po, pm, ps, co, cm, cs, S=T, B=0, N=N, D=D, layout=W.TND)
+    G.check_out(G.f64(out), ro, dtype, "tnd merge out")
+    G.check_stats(om.numpy(), osum.numpy(), rm, rs, "tnd merge stats")
+
+
+def test_merge_tnd_seq_qlen_checked():
+    T, N, D = 64, 2, 128
+    po = W.randn((T, N * D), 51, torch.bfloat16)
+    pm, ps = W.merge_stats_random(1, T, N, 52)
+    pm, ps = pm[0], ps[0]
+    _, _, _, st = _merge_tnd_gpu(po, pm, ps, po, pm, ps, T, N, D, W.BF16, seq_qlen=[10, 10, 64], B=3)
+    assert st == 0
+    _, _, _, st = _merge_tnd_gpu(po, pm, ps, po, pm, ps, T, N, D, W.BF16, seq_qlen=[10, 5, 64], B=3)
+    assert st == sdpa.ATTN_ERR_DATA
+    _, _, _, st = _merge_tnd_gpu(po, pm, ps, po, pm, ps, T, N, D, W.BF16, seq_qlen=[10, 20, 63], B=3)
+    assert st == sdpa.ATTN_ERR_DATA
+
+
+@pytest.mark.parametrize("S,B,N,D", [(100, 2, 3, 128), (37, 3, 5, 40)])
+def test_merge_f16_sbh(S, B, N, D):
+    po = W.randn((S, B, N * D), 61, torch.float16)
+    co = W.randn((S, B, N * D), 62, torch.float16)
+    pm, ps = W.merge_stats_random(B, N, S, 63)
+    cm, cs = W.merge_stats_random(B, N, S, 65)
+    _check_merge(po, pm, ps, co, cm, cs, S, B, N, D, W.F16)
