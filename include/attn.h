@@ -6,6 +6,7 @@
  *   attn_fwd         O = softmax(scale * Q K^T + mask) V, with per-row softmax max and sum.
  *   attn_sparse_csr  the same softmax restricted to the entries of a CSR pattern (fp32).
  *   attn_merge       merge of two partial attention results from their max/sum statistics.
+ *   attn_fwd_accumulate  attn_fwd over one chunk of keys folded into a running merge result.
  *
  * Conventions shared by every call
  *   - All tensor pointers are DEVICE pointers owned by the caller. The library allocates no
@@ -99,6 +100,32 @@ ATTN_API int attn_fwd(const void* q, const void* k, const void* v,
              int B, int Sq, int Skv, int Nq, int Nkv, int D,
              float scale, int mask_mode, int dtype, int layout,
              void* out, float* softmax_max, float* softmax_sum, void* stream);
+
+/*
+ * attn_fwd_accumulate -- attention forward over one chunk of keys, folded into a running
+ * accumulator (the fused form of attn_fwd followed by attn_merge).
+ *
+ * Defined by: the attn_fwd definition above for this chunk's keys, and the lane-wise update of
+ * "npu_ring_attention_update" (MindSpeed op doc, 小算子等价计算逻辑) for the fold: for each of
+ * the 8 statistic lanes m = max(pm, m_c), ps' = ps e^(pm - m), cs' = l_c e^(m_c - m),
+ * l = ps' + cs'; out = acc_out * ps'_0 / l_0 + o_c * cs'_0 / l_0, where (o_c, m_c, l_c) are this
+ * chunk's output row and statistics, computed in fp32 and never rounded before the fold.
+ * Calling it for every chunk of a split key range (first = 1 for the first chunk) gives the
+ * attention over the whole key range, as a ring of devices would compute it.
+ *
+ * Arguments are those of attn_fwd (k, v, cu_seqlens_kv and Skv describe this chunk of keys),
+ * except the outputs, which are the accumulator in the layouts of attn_merge:
+ *   layout = ATTN_BHSD: acc_out [Sq, B, Nq*D] ("SBH"), acc_max / acc_sum float32 [B, Nq, Sq, 8]
+ *   layout = ATTN_TND:  acc_out [Tq, Nq*D],             acc_max / acc_sum float32 [Tq, Nq, 8]
+ * acc_out has the element type `dtype`. first = 1 overwrites the accumulator (all 8 lanes get
+ * this chunk's statistics); first = 0 folds into it (it must hold an earlier call's result).
+ * Calls that fold into the same accumulator must not overlap on the device.
+ */
+ATTN_API int attn_fwd_accumulate(const void* q, const void* k, const void* v,
+                                 const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_kv,
+                                 int B, int Sq, int Skv, int Nq, int Nkv, int D,
+                                 float scale, int mask_mode, int dtype, int layout, int first,
+                                 void* acc_out, float* acc_max, float* acc_sum, void* stream);
 
 /*
  * attn_sparse_csr -- CSR-sparse attention forward, float32.

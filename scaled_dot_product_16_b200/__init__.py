@@ -16,7 +16,7 @@ import threading
 from typing import Optional
 
 __all__ = [
-    "attn_fwd", "attn_sparse_csr", "attn_merge", "attn_get_last_error", "AttnError",
+    "attn_fwd", "attn_fwd_accumulate", "attn_sparse_csr", "attn_merge", "attn_get_last_error", "AttnError",
     "ATTN_BF16", "ATTN_F32", "ATTN_F16", "ATTN_BHSD", "ATTN_TND", "ATTN_MASK_NONE",
     "ATTN_MASK_CAUSAL_TOPLEFT", "ATTN_MASK_CAUSAL_BOTTOMRIGHT", "lib_path", "load_library",
 ]
@@ -55,6 +55,8 @@ def load_library():
         P, I, I64, F = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float
         lib.attn_fwd.argtypes = [P, P, P, P, P, I, I, I, I, I, I, F, I, I, I, P, P, P, P]
         lib.attn_fwd.restype = I
+        lib.attn_fwd_accumulate.argtypes = [P, P, P, P, P, I, I, I, I, I, I, F, I, I, I, I, P, P, P, P]
+        lib.attn_fwd_accumulate.restype = I
         lib.attn_sparse_csr.argtypes = [P, P, P, P, P, I, I, I, I, I64, P, P]
         lib.attn_sparse_csr.restype = I
         lib.attn_merge.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, P, P, P, P, P]
@@ -108,6 +110,19 @@ def attn_fwd(q, k, v, *, cu_seqlens_q=None, cu_seqlens_kv=None, B: int, Sq: int,
                         int(B), int(Sq), int(Skv), int(Nq), int(Nkv), int(D), float(scale),
                         int(mask_mode), int(dtype), int(layout), _ptr(out), _ptr(softmax_max),
                         _ptr(softmax_sum), _stream(stream)), "attn_fwd")
+
+
+def attn_fwd_accumulate(q, k, v, *, cu_seqlens_q=None, cu_seqlens_kv=None, B: int, Sq: int, Skv: int,
+                        Nq: int, Nkv: int, D: int, scale: float, mask_mode: int, dtype: int,
+                        layout: int, first: bool, acc_out, acc_max, acc_sum, stream=None) -> None:
+    """attn_fwd over one chunk of keys, folded into a running accumulator in attn_merge's
+    layouts (see ``attn_fwd_accumulate`` in include/attn.h)."""
+    lib = load_library()
+    _check(lib.attn_fwd_accumulate(_ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens_q),
+                                   _ptr(cu_seqlens_kv), int(B), int(Sq), int(Skv), int(Nq), int(Nkv),
+                                   int(D), float(scale), int(mask_mode), int(dtype), int(layout),
+                                   1 if first else 0, _ptr(acc_out), _ptr(acc_max), _ptr(acc_sum),
+                                   _stream(stream)), "attn_fwd_accumulate")
 
 
 def attn_sparse_csr(q, k, v, csr_offset, csr_columns, *, B: int, H: int, S: int, D: int,

@@ -66,10 +66,14 @@ const char* attn_status_string(int s) {
   }
 }
 
-int attn_fwd(const void* q, const void* k, const void* v, const int32_t* cu_seqlens_q,
+}  // extern "C"
+
+namespace {
+
+int fwd_impl(const void* q, const void* k, const void* v, const int32_t* cu_seqlens_q,
              const int32_t* cu_seqlens_kv, int B, int Sq, int Skv, int Nq, int Nkv, int D,
              float scale, int mask_mode, int dtype, int layout, void* out, float* softmax_max,
-             float* softmax_sum, void* stream) {
+             float* softmax_sum, int acc_mode, void* stream) {
   if (layout != ATTN_BHSD && layout != ATTN_TND) return ATTN_ERR_INVALID;
   if (dtype != ATTN_BF16 && dtype != ATTN_F32 && dtype != ATTN_F16) return ATTN_ERR_INVALID;
   if (mask_mode < ATTN_MASK_NONE || mask_mode > ATTN_MASK_CAUSAL_BOTTOMRIGHT) return ATTN_ERR_INVALID;
@@ -78,6 +82,7 @@ int attn_fwd(const void* q, const void* k, const void* v, const int32_t* cu_seql
   if (D < 1 || D > 768) return ATTN_ERR_INVALID;
   if (!(scale > 0.f) || scale == INFINITY) return ATTN_ERR_INVALID;  // finite and positive
   if ((softmax_max == nullptr) != (softmax_sum == nullptr)) return ATTN_ERR_INVALID;
+  if (acc_mode != 0 && softmax_max == nullptr) return ATTN_ERR_INVALID;
   if (layout == ATTN_TND) {
     if (B > kMaxCu || Sq > kMaxTokens || Skv > kMaxTokens) return ATTN_ERR_INVALID;
     if (B > 0 && (cu_seqlens_q == nullptr || cu_seqlens_kv == nullptr)) return ATTN_ERR_INVALID;
@@ -110,6 +115,7 @@ int attn_fwd(const void* q, const void* k, const void* v, const int32_t* cu_seql
   a.mask_mode = mask_mode;
   a.layout = layout;
   a.dtype = dtype;
+  a.acc_mode = acc_mode;
   a.out = out;
   a.smax = softmax_max;
   a.ssum = softmax_sum;
@@ -118,6 +124,28 @@ int attn_fwd(const void* q, const void* k, const void* v, const int32_t* cu_seql
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const cudaError_t e = dtype == ATTN_F32 ? sdpa::launch_fwd_f32(a, st) : sdpa::launch_fwd_bf16(a, st);
   return e == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+int attn_fwd(const void* q, const void* k, const void* v, const int32_t* cu_seqlens_q,
+             const int32_t* cu_seqlens_kv, int B, int Sq, int Skv, int Nq, int Nkv, int D,
+             float scale, int mask_mode, int dtype, int layout, void* out, float* softmax_max,
+             float* softmax_sum, void* stream) {
+  return fwd_impl(q, k, v, cu_seqlens_q, cu_seqlens_kv, B, Sq, Skv, Nq, Nkv, D, scale, mask_mode,
+                  dtype, layout, out, softmax_max, softmax_sum, 0, stream);
+}
+
+int attn_fwd_accumulate(const void* q, const void* k, const void* v, const int32_t* cu_seqlens_q,
+                        const int32_t* cu_seqlens_kv, int B, int Sq, int Skv, int Nq, int Nkv,
+                        int D, float scale, int mask_mode, int dtype, int layout, int first,
+                        void* acc_out, float* acc_max, float* acc_sum, void* stream) {
+  if (acc_out == nullptr || acc_max == nullptr || acc_sum == nullptr) return ATTN_ERR_INVALID;
+  if (first != 0 && first != 1) return ATTN_ERR_INVALID;
+  return fwd_impl(q, k, v, cu_seqlens_q, cu_seqlens_kv, B, Sq, Skv, Nq, Nkv, D, scale, mask_mode,
+                  dtype, layout, acc_out, acc_max, acc_sum, first ? 1 : 2, stream);
 }
 
 int attn_sparse_csr(const float* q, const float* k, const float* v, const int32_t* csr_offset,

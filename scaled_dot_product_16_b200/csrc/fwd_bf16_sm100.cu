@@ -126,6 +126,53 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile
   }
 }
 
+constexpr int kAccNone = 0, kAccFirst = 1, kAccMerge = 2;
+
+// Fold one row's result (max m_loc, sum l_loc, output o = O * f_o) into an accumulator row
+// with the lane-wise update of "npu_ring_attention_update" (小算子等价计算逻辑): for each of the
+// 8 statistic lanes m = max(pm, m_loc), ps' = ps e^(pm - m), cs' = l_loc e^(m_loc - m),
+// l = ps' + cs'; the output becomes prev * ps'_0 / l_0 + o * cs'_0 / l_0. On the first chunk the
+// accumulator is simply overwritten. Returns the two output factors.
+__device__ __forceinline__ void merge_into_stats(const FwdArgs& a, int64_t so, float m_loc, float l_loc,
+                                                 float* f_prev, float* f_o) {
+  float4* mx = reinterpret_cast<float4*>(a.smax + so);
+  float4* sm = reinterpret_cast<float4*>(a.ssum + so);
+  if (a.acc_mode == kAccFirst) {
+    const float4 mv = make_float4(m_loc, m_loc, m_loc, m_loc), lv = make_float4(l_loc, l_loc, l_loc, l_loc);
+    mx[0] = mv; mx[1] = mv; sm[0] = lv; sm[1] = lv;
+    *f_prev = 0.f;
+    return;
+  }
+  float pm[8], ps[8];
+  *reinterpret_cast<float4*>(pm) = mx[0];
+  *reinterpret_cast<float4*>(pm + 4) = mx[1];
+  *reinterpret_cast<float4*>(ps) = sm[0];
+  *reinterpret_cast<float4*>(ps + 4) = sm[1];
+  float nm[8], nl[8], ps0 = 0.f, cs0 = 0.f;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const float mk = fmaxf(pm[k], m_loc);
+    float a1 = 0.f, a2 = 0.f;
+    if (mk != -INFINITY) {
+      a1 = ps[k] * expf(pm[k] - mk);
+      a2 = l_loc * expf(m_loc - mk);
+    }
+    nm[k] = mk;
+    nl[k] = a1 + a2;
+    if (k == 0) {
+      ps0 = a1;
+      cs0 = a2;
+    }
+  }
+  mx[0] = *reinterpret_cast<float4*>(nm);
+  mx[1] = *reinterpret_cast<float4*>(nm + 4);
+  sm[0] = *reinterpret_cast<float4*>(nl);
+  sm[1] = *reinterpret_cast<float4*>(nl + 4);
+  const float inv = nl[0] != 0.f ? 1.f / nl[0] : 0.f;
+  *f_prev = ps0 * inv;
+  *f_o *= cs0 * inv;
+}
+
 struct Work {
   int b, h, g;      // sequence, query head, key/value head
   int q0, sq;       // first query token and query length of the sequence
@@ -463,9 +510,27 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool store = r < rows;
       const bool bhsd = a.layout == ATTN_BHSD;
       uint16_t* out = static_cast<uint16_t*>(a.out);  // bf16 or f16 bit patterns
-      const int64_t orow = bhsd ? (((int64_t)w.b * a.Nq + w.h) * a.Sq + i) * HD
-                                : ((int64_t)(w.q0 + i) * a.Nq + w.h) * HD;
-      const float inv = (l > 0.f && ok) ? 1.f / l : 0.f;
+      // this row's own result: o = O / l, max and sum in natural-log units
+      const bool any = l > 0.f && ok;
+      const float m_loc = any ? mraw * a.scale : -INFINITY;
+      const float l_loc = any ? l * ex2(m - mraw * scale_log2) : 0.f;
+      float f_o = any ? 1.f / l : 0.f;  // factor on the unnormalised O in TMEM
+      float f_prev = 0.f;               // factor on the accumulator's previous output row
+      int64_t orow, so;
+      if (a.acc_mode == kAccNone) {
+        orow = bhsd ? (((int64_t)w.b * a.Nq + w.h) * a.Sq + i) * HD : ((int64_t)(w.q0 + i) * a.Nq + w.h) * HD;
+        so = bhsd ? ((int64_t)w.b * a.Nq + w.h) * a.Sq + i : (int64_t)(w.q0 + i) * a.Nq + w.h;
+        if (store && a.smax != nullptr) {
+          a.smax[so] = m_loc;
+          a.ssum[so] = l_loc;
+        }
+      } else {
+        // accumulator in the merge layouts: BHSD -> output [Sq, B, Nq*D] (SBH), statistics
+        // [B, Nq, Sq, 8]; TND -> output [T, Nq*D], statistics [T, Nq, 8]
+        orow = bhsd ? (((int64_t)i * a.B + w.b) * a.Nq + w.h) * HD : ((int64_t)(w.q0 + i) * a.Nq + w.h) * HD;
+        so = (bhsd ? ((int64_t)w.b * a.Nq + w.h) * a.Sq + i : (int64_t)(w.q0 + i) * a.Nq + w.h) * 8;
+        if (store) merge_into_stats(a, so, m_loc, l_loc, &f_prev, &f_o);
+      }
 #pragma unroll
       for (int c = 0; c < HD / 32; ++c) {
         uint32_t o[32];
@@ -477,23 +542,34 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int x = 0; x < 32; ++x) o[x] = 0u;
         }
         if (store) {
+          uint4* dst = reinterpret_cast<uint4*>(out + orow + c * 32);
+          uint32_t prev[16];
+          if (a.acc_mode == kAccMerge) {
+#pragma unroll
+            for (int x = 0; x < 4; ++x) {
+              const uint4 t = dst[x];
+              prev[4 * x] = t.x;
+              prev[4 * x + 1] = t.y;
+              prev[4 * x + 2] = t.z;
+              prev[4 * x + 3] = t.w;
+            }
+          }
           uint32_t pkd[16];
 #pragma unroll
-          for (int x = 0; x < 16; ++x)
-            pkd[x] = pack16x2<F16>(inv == 0.f ? 0.f : __uint_as_float(o[2 * x]) * inv,
-                                   inv == 0.f ? 0.f : __uint_as_float(o[2 * x + 1]) * inv);
-          uint4* dst = reinterpret_cast<uint4*>(out + orow + c * 32);
+          for (int x = 0; x < 16; ++x) {
+            float v0 = f_o == 0.f ? 0.f : __uint_as_float(o[2 * x]) * f_o;
+            float v1 = f_o == 0.f ? 0.f : __uint_as_float(o[2 * x + 1]) * f_o;
+            if (a.acc_mode == kAccMerge) {
+              const float2 pv = unpack16x2<F16>(prev[x]);
+              v0 = fmaf(pv.x, f_prev, v0);
+              v1 = fmaf(pv.y, f_prev, v1);
+            }
+            pkd[x] = pack16x2<F16>(v0, v1);
+          }
 #pragma unroll
           for (int x = 0; x < 4; ++x)
             dst[x] = make_uint4(pkd[4 * x], pkd[4 * x + 1], pkd[4 * x + 2], pkd[4 * x + 3]);
         }
-      }
-      if (store && a.smax != nullptr) {
-        const int64_t so = bhsd ? ((int64_t)w.b * a.Nq + w.h) * a.Sq + i
-                                : (int64_t)(w.q0 + i) * a.Nq + w.h;
-        const bool any = l > 0.f && ok;
-        a.smax[so] = any ? mraw * a.scale : -INFINITY;
-        a.ssum[so] = any ? l * ex2(m - mraw * scale_log2) : 0.f;
       }
     }
   }

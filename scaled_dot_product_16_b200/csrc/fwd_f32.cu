@@ -184,19 +184,63 @@ __global__ void __launch_bounds__(kWarps * 32) fwd_f32_kernel(FwdArgs a, int til
 #pragma unroll
   for (int r = 0; r < kRowsPerWarp; ++r) {
     const int i = row0 + warp * kRowsPerWarp + r;
-    if (i >= sq) continue;
-    const float inv = l[r] > 0.f ? 1.f / l[r] : 0.f;
-    const int64_t o = qoff(i);
+    if (i >= sq) continue;  // warp-uniform
+    const bool any = l[r] > 0.f;
+    const float m_loc = any ? m[r] : -INFINITY;
+    const float l_loc = l[r];
+    float f_o = any ? 1.f / l[r] : 0.f;
+    float f_prev = 0.f;
+    int64_t o;
+    if (a.acc_mode == 0) {
+      o = qoff(i);
+      if (lane == 0 && a.smax != nullptr) {
+        const int64_t so = a.layout == ATTN_BHSD ? ((int64_t)b * a.Nq + h) * a.Sq + i
+                                                 : (int64_t)(q0 + i) * a.Nq + h;
+        a.smax[so] = m_loc;
+        a.ssum[so] = l_loc;
+      }
+    } else {
+      // accumulator in the merge layouts: BHSD -> output [Sq, B, Nq*D] (SBH), statistics
+      // [B, Nq, Sq, 8]; TND -> output [T, Nq*D], statistics [T, Nq, 8]. Lanes 0-7 update the
+      // 8 statistic lanes ("npu_ring_attention_update", 小算子等价计算逻辑); lane 0's factors
+      // rescale the output row.
+      o = a.layout == ATTN_BHSD ? (((int64_t)i * a.B + b) * a.Nq + h) * D : qoff(i);
+      const int64_t so = (a.layout == ATTN_BHSD ? ((int64_t)b * a.Nq + h) * a.Sq + i
+                                                : (int64_t)(q0 + i) * a.Nq + h) * 8;
+      float ps2 = 0.f, cs2 = 0.f, nl = 0.f;
+      if (lane < 8) {
+        if (a.acc_mode == 1) {
+          a.smax[so + lane] = m_loc;
+          a.ssum[so + lane] = l_loc;
+          cs2 = l_loc;
+          nl = l_loc;
+        } else {
+          const float pm = a.smax[so + lane], ps = a.ssum[so + lane];
+          const float mk = fmaxf(pm, m_loc);
+          if (mk != -INFINITY) {
+            ps2 = ps * expf(pm - mk);
+            cs2 = l_loc * expf(m_loc - mk);
+          }
+          nl = ps2 + cs2;
+          a.smax[so + lane] = mk;
+          a.ssum[so + lane] = nl;
+        }
+      }
+      ps2 = __shfl_sync(0xffffffffu, ps2, 0);
+      cs2 = __shfl_sync(0xffffffffu, cs2, 0);
+      nl = __shfl_sync(0xffffffffu, nl, 0);
+      const float inv = nl != 0.f ? 1.f / nl : 0.f;
+      f_prev = a.acc_mode == 1 ? 0.f : ps2 * inv;
+      f_o = a.acc_mode == 1 ? f_o : f_o * cs2 * inv;
+    }
 #pragma unroll
     for (int t = 0; t < DT; ++t) {
       const int d = lane + 32 * t;
-      if (d < D) O[o + d] = acc[r][t] * inv;
-    }
-    if (lane == 0 && a.smax != nullptr) {
-      const int64_t so = a.layout == ATTN_BHSD ? ((int64_t)b * a.Nq + h) * a.Sq + i
-                                               : (int64_t)(q0 + i) * a.Nq + h;
-      a.smax[so] = l[r] > 0.f ? m[r] : -INFINITY;
-      a.ssum[so] = l[r];
+      if (d < D) {
+        float v = acc[r][t] * f_o;
+        if (a.acc_mode == 2) v = fmaf(O[o + d], f_prev, v);
+        O[o + d] = v;
+      }
     }
   }
 }

@@ -15,9 +15,10 @@ struct FwdArgs {
   int B, Sq, Skv, Nq, Nkv, D;
   float scale;
   int mask_mode, layout, dtype;
-  void* out;
-  float* smax;  // may be null (with ssum)
-  float* ssum;
+  int acc_mode;  // 0: plain output; 1: overwrite an accumulator; 2: merge into it
+  void* out;     // output, or the accumulator's output (merge layouts) when acc_mode != 0
+  float* smax;   // statistics (may be null with ssum when acc_mode == 0), or the accumulator's
+  float* ssum;   // [.., 8]-lane statistics when acc_mode != 0
   int* status;  // device status word
   int num_sms;
 };
