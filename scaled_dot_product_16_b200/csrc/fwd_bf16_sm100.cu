@@ -55,20 +55,27 @@ constexpr uint64_t kWaitLimitNs = 200ull * 1000ull * 1000ull;  // 200 ms per bar
 constexpr uint32_t kSuspendNs = SDPA_SUSPEND_NS;  // longest hardware suspension per try_wait
 
 #ifndef SDPA_EMU_EVERY
-#define SDPA_EMU_EVERY 4
+#define SDPA_EMU_EVERY 5
 #endif
 // One exp2 pair in kEmuEvery goes to the FMA-pipe polynomial (0: none).
 constexpr int kEmuEvery = SDPA_EMU_EVERY;
+#ifndef SDPA_STAGES_D128
+#define SDPA_STAGES_D128 4
+#endif
 
 // 2^x for a pair on the FMA/ALU pipes. Range reduction after Cody and Waite: x = j + f with
 // j = round(x) (adding 1.5 * 2^23 rounds to nearest and leaves j in the low mantissa bits) and
 // f in [-1/2, 1/2]; 2^f by a degree-3 polynomial fitted here by the Remez exchange for minimum
 // relative error (csrc/fit_exp2_poly.py, max relative error 7.5e-5); 2^j is added into the
-// exponent field. Inputs below -125 (including -inf from masking) give exactly 0.
+// exponent field. Inputs are clamped at -126 first (one max per lane instead of a compare and a
+// select): from there down, -inf from masking included, the result is a positive value below
+// 2^-125, which the callers treat as zero (rows that see no key at all are caught by their max).
 __device__ __forceinline__ void exp2_poly2(float x0, float x1, float& p0, float& p1) {
   constexpr float kShift = 12582912.0f;  // 1.5 * 2^23
   constexpr float c0 = 9.999280572e-01f, c1 = 6.932609677e-01f, c2 = 2.426111251e-01f,
                   c3 = 5.517166853e-02f;
+  x0 = fmaxf(x0, -126.f);
+  x1 = fmaxf(x1, -126.f);
   float t0, t1, j0, j1, f0, f1, q0, q1;
   fadd2(x0, x1, kShift, kShift, t0, t1);
   fadd2(t0, t1, -kShift, -kShift, j0, j1);
@@ -76,21 +83,21 @@ __device__ __forceinline__ void exp2_poly2(float x0, float x1, float& p0, float&
   ffma2(c3, c3, f0, f1, c2, c2, q0, q1);
   ffma2(q0, q1, f0, f1, c1, c1, q0, q1);
   ffma2(q0, q1, f0, f1, c0, c0, q0, q1);
-  const uint32_t b0 = __float_as_uint(q0) + (__float_as_uint(t0) << 23);
-  const uint32_t b1 = __float_as_uint(q1) + (__float_as_uint(t1) << 23);
-  p0 = x0 < -125.f ? 0.f : __uint_as_float(b0);
-  p1 = x1 < -125.f ? 0.f : __uint_as_float(b1);
+  p0 = __uint_as_float(__float_as_uint(q0) + (__float_as_uint(t0) << 23));
+  p1 = __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23));
 }
 
 template <int HD, bool F16>
 struct Cfg {
   static constexpr int kBoxes = HD / 64;                 // 64-element (128-byte) TMA boxes
   static constexpr int kTileBytes = kBM * HD * 2;        // one Q, K or V tile
-  static constexpr int kStages = HD == 128 ? 4 : 6;      // K/V ring depth
+  static constexpr int kStages = HD == 128 ? SDPA_STAGES_D128 : 6;  // K/V ring depth
   static constexpr int kQOff = 0;
   static constexpr int kKVOff = 2 * kTileBytes;
   static constexpr int kBarOff = kKVOff + kStages * kTileBytes;
   static constexpr int kSmemBytes = kBarOff + 256 + 1024;  // barriers + 1 KB for alignment
+  static_assert(kStages >= 2 && kStages <= 8, "barrier arrays hold 8 stages");
+  static_assert(kSmemBytes <= 232448, "227 KB of shared memory per block");
   static constexpr uint32_t kFmt = F16 ? 0u : 1u;  // instruction-descriptor operand format
   static constexpr uint32_t kIdescQK = idesc_f16_f32(kBM, kBN, 0, 0, kFmt);
   static constexpr uint32_t kIdescPV = idesc_f16_f32(kBM, HD, 0, 1, kFmt);
@@ -511,7 +518,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool bhsd = a.layout == ATTN_BHSD;
       uint16_t* out = static_cast<uint16_t*>(a.out);  // bf16 or f16 bit patterns
       // this row's own result: o = O / l, max and sum in natural-log units
-      const bool any = l > 0.f && ok;
+      // a row that saw no key keeps mraw = -inf (its sum holds only the polynomial's tiny
+      // values for masked scores) and gives a zero output, max -inf and sum 0
+      const bool any = mraw > -INFINITY && l > 0.f && ok;
       const float m_loc = any ? mraw * a.scale : -INFINITY;
       const float l_loc = any ? l * ex2(m - mraw * scale_log2) : 0.f;
       float f_o = any ? 1.f / l : 0.f;  // factor on the unnormalised O in TMEM

@@ -17,7 +17,7 @@ def _coeffs():
 
 def _emulate(x):
     c0, c1, c2, c3 = _coeffs()
-    x = x.astype(np.float32)
+    x = np.maximum(x.astype(np.float32), np.float32(-126.0))
     shift = np.float32(12582912.0)
     with np.errstate(invalid="ignore", over="ignore"):
         t = (x + shift).astype(np.float32)
@@ -27,8 +27,7 @@ def _emulate(x):
         q = (q * f + c1).astype(np.float32)
         q = (q * f + c0).astype(np.float32)
         bits = (q.view(np.uint32) + (t.view(np.uint32) << np.uint32(23))).astype(np.uint32)
-    out = bits.view(np.float32)
-    return np.where(x < -125.0, np.float32(0.0), out)
+    return bits.view(np.float32)
 
 
 def test_relative_error_over_the_used_range():
@@ -40,6 +39,14 @@ def test_relative_error_over_the_used_range():
     assert rel.max() <= 8e-5, rel.max()
 
 
-def test_masked_and_underflow_give_zero():
-    x = np.array([-np.inf, -1e30, -200.0, -125.5], dtype=np.float32)
-    assert np.all(_emulate(x) == 0.0)
+def test_masked_and_underflow_stay_below_2_to_minus_125():
+    """Scores set to -inf by a mask and anything under -125.5 land on a non-negative value below
+    2^-125 (never NaN, never an overflowed exponent); from -125.5 up the error bound holds."""
+    x = np.concatenate([np.array([-np.inf, -1e30, -200.0, -127.0, -126.0], dtype=np.float32),
+                        np.linspace(-130.0, -125.5, 10_001, dtype=np.float32)])
+    y = _emulate(x)
+    assert np.all(np.isfinite(y)) and np.all(y >= 0.0)
+    assert np.all(y.astype(np.float64) < 2.0 ** -125)
+    x = np.linspace(-125.5, -120.0, 100_001, dtype=np.float32)
+    rel = np.abs(_emulate(x).astype(np.float64) / np.exp2(x.astype(np.float64)) - 1.0)
+    assert rel.max() <= 8e-5, rel.max()
