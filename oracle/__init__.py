@@ -49,6 +49,12 @@ def _bind(path: str):
     lib.oracle_attn_fwd_rows.argtypes = [P, P, P, I, P, P, I, I, I, I, I, I, D, I, I,
                                          P, P, I64, P, P, P]
     lib.oracle_attn_fwd_rows.restype = I
+    lib.oracle_attn_fwd_ext.argtypes = [P, P, P, I, P, P, I, I, I, I, I, I, I, D, I, I64, I64,
+                                        P, I64, I64, I, P, P, P]
+    lib.oracle_attn_fwd_ext.restype = I
+    lib.oracle_attn_fwd_ext_rows.argtypes = [P, P, P, I, P, P, I, I, I, I, I, I, I, D, I, I64, I64,
+                                             P, I64, I64, I, P, P, I64, P, P, P]
+    lib.oracle_attn_fwd_ext_rows.restype = I
     lib.oracle_sparse_csr.argtypes = [P, P, P, I, P, P, I, I, I, I, I64, P]
     lib.oracle_sparse_csr.restype = I
     lib.oracle_merge.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, P, P, P]
@@ -173,6 +179,72 @@ def attn_fwd_rows(q, k, v, rows_h, rows_t, *, cu_q=None, cu_kv=None, B: int, Sq:
                                   _ptr(rh), _ptr(rt), n, _ptr(out), _ptr(m), _ptr(l))
     if rc != 0:
         raise ValueError(f"oracle_attn_fwd_rows rejected its arguments (code {rc})")
+    return out, m, l
+
+
+MASK_BAND = 3
+
+
+def _mask(mask):
+    if mask is None:
+        return None
+    try:
+        import torch
+        if isinstance(mask, torch.Tensor):
+            mask = mask.detach().cpu().numpy()
+    except ImportError:  # pragma: no cover
+        pass
+    return np.ascontiguousarray(mask, dtype=np.uint8)
+
+
+def attn_fwd_ext(q, k, v, *, cu_q=None, cu_kv=None, B: int, Sq: int, Skv: int, Nq: int, Nkv: int,
+                 Dqk: int, Dv: int, scale: float, mask_mode: int, pre_tokens: int = 0,
+                 next_tokens: int = 0, mask=None, mask_bstride: int = 0, mask_rstride: int = 0,
+                 layout: int):
+    """Masked forward (band limits, explicit uint8 mask with 1 = excluded, value head size Dv).
+    Returns (out float64 [.., Nq, Dv] in q's layout, softmax_max, softmax_sum)."""
+    lib = _load()
+    (qa, ka, va), et = _same_type(q, k, v)
+    cq, ck = _cu(cu_q), _cu(cu_kv)
+    mk = _mask(mask)
+    if layout == BHSD:
+        out = np.zeros((B, Nq, Sq, Dv))
+        m = np.zeros((B, Nq, Sq))
+    else:
+        out = np.zeros((Sq, Nq, Dv))
+        m = np.zeros((Sq, Nq))
+    l = np.zeros_like(m)
+    rc = lib.oracle_attn_fwd_ext(_ptr(qa), _ptr(ka), _ptr(va), et, _ptr(cq), _ptr(ck), B, Sq, Skv,
+                                 Nq, Nkv, Dqk, Dv, float(scale), int(mask_mode), int(pre_tokens),
+                                 int(next_tokens), _ptr(mk), int(mask_bstride), int(mask_rstride),
+                                 int(layout), _ptr(out), _ptr(m), _ptr(l))
+    if rc != 0:
+        raise ValueError(f"oracle_attn_fwd_ext rejected its arguments (code {rc})")
+    return out, m, l
+
+
+def attn_fwd_ext_rows(q, k, v, rows_h, rows_t, *, cu_q=None, cu_kv=None, B: int, Sq: int,
+                      Skv: int, Nq: int, Nkv: int, Dqk: int, Dv: int, scale: float,
+                      mask_mode: int, pre_tokens: int = 0, next_tokens: int = 0, mask=None,
+                      mask_bstride: int = 0, mask_rstride: int = 0, layout: int):
+    """Selected rows of attn_fwd_ext. Returns (out [n, Dv], max [n], sum [n])."""
+    lib = _load()
+    (qa, ka, va), et = _same_type(q, k, v)
+    cq, ck = _cu(cu_q), _cu(cu_kv)
+    mk = _mask(mask)
+    rh = np.ascontiguousarray(rows_h, dtype=np.int32)
+    rt = np.ascontiguousarray(rows_t, dtype=np.int64)
+    n = int(rh.shape[0])
+    out = np.zeros((n, Dv))
+    m = np.zeros(n)
+    l = np.zeros(n)
+    rc = lib.oracle_attn_fwd_ext_rows(_ptr(qa), _ptr(ka), _ptr(va), et, _ptr(cq), _ptr(ck), B, Sq,
+                                      Skv, Nq, Nkv, Dqk, Dv, float(scale), int(mask_mode),
+                                      int(pre_tokens), int(next_tokens), _ptr(mk),
+                                      int(mask_bstride), int(mask_rstride), int(layout), _ptr(rh),
+                                      _ptr(rt), n, _ptr(out), _ptr(m), _ptr(l))
+    if rc != 0:
+        raise ValueError(f"oracle_attn_fwd_ext_rows rejected its arguments (code {rc})")
     return out, m, l
 
 

@@ -224,6 +224,157 @@ int oracle_attn_fwd_rows(const void *q, const void *k, const void *v, int et,
 }
 
 /*
+ * Masked forward with band limits, an explicit mask and a value head size of its own
+ * ("aclnnFlashAttentionVarLenScore", 约束说明: preTokens / nextTokens band, attenMaskOptional,
+ * qD == kD >= vD). The page only lists these inputs; the table that defines the sparse modes is
+ * not on it, so the readings are:
+ *   band (mode 3):      key j is visible to query row i iff i - pre <= j <= i + next, with i and j
+ *                       positions within the sequence (top-left aligned); pre + next >= 0 so the
+ *                       band is not empty ("preTokens and nextTokens must intersect").
+ *   explicit mask:      uint8, 1 = masked out (the page forbids a row of all 1s, so 1 excludes);
+ *                       element (b, i, j) at mask[b * mask_bstride + i * mask_rstride + j].
+ *                       Combined with the mode by AND: a key must pass both.
+ *   value head size Dv: v is [.., Nkv, Dv] in the q/k layout, out is [.., Nq, Dv].
+ * Rows with no visible key give out = 0, max = -inf, sum = 0, as elsewhere here.
+ */
+#define ORC_MASK_BAND 3
+
+static int key_visible(int mask_mode, int64_t i, int64_t j, int64_t sq, int64_t sk, int64_t pre,
+                       int64_t next, const uint8_t *mask, int64_t mrow, int64_t mask_rstride) {
+  if (j < 0 || j >= sk) return 0;
+  if (mask_mode == ORC_MASK_TOPLEFT && j > i) return 0;
+  if (mask_mode == ORC_MASK_BOTTOMRIGHT && j > i + sk - sq) return 0;
+  if (mask_mode == ORC_MASK_BAND && (j < i - pre || j > i + next)) return 0;
+  if (mask != NULL && mask[mrow + i * mask_rstride + j] != 0) return 0;
+  return 1;
+}
+
+/* One query row over every key of its sequence, each tested by key_visible. */
+static void attn_row_ext(const void *q, const void *k, const void *v, int et, int layout,
+                         int64_t b, int64_t tq0, int64_t tk0, int64_t i, int64_t h, int64_t g,
+                         int64_t lq, int64_t lk, int64_t Nq, int64_t Nkv, int64_t Sq, int64_t Skv,
+                         int64_t Dqk, int64_t Dv, double scale, int mask_mode, int64_t pre,
+                         int64_t next, const uint8_t *mask, int64_t mask_bstride,
+                         int64_t mask_rstride, double *s, double *o, double *m, double *l) {
+  int64_t j, d, nvis = 0;
+  double mx = -INFINITY, sum = 0.0;
+  for (d = 0; d < Dv; ++d) o[d] = 0.0;
+  for (j = 0; j < lk; ++j) {
+    double acc = 0.0;
+    if (!key_visible(mask_mode, i, j, lq, lk, pre, next, mask, b * mask_bstride, mask_rstride)) {
+      s[j] = -INFINITY;
+      continue;
+    }
+    for (d = 0; d < Dqk; ++d)
+      acc += ld(q, offs(layout, b, tq0, i, h, d, Nq, Sq, Dqk), et) *
+             ld(k, offs(layout, b, tk0, j, g, d, Nkv, Skv, Dqk), et);
+    s[j] = scale * acc;
+    if (s[j] > mx) mx = s[j];
+    ++nvis;
+  }
+  if (nvis == 0) {
+    *m = -INFINITY;
+    *l = 0.0;
+    return;
+  }
+  for (j = 0; j < lk; ++j) {
+    s[j] = s[j] == -INFINITY ? 0.0 : exp(s[j] - mx);
+    sum += s[j];
+  }
+  for (j = 0; j < lk; ++j)
+    if (s[j] != 0.0)
+      for (d = 0; d < Dv; ++d) o[d] += s[j] * ld(v, offs(layout, b, tk0, j, g, d, Nkv, Skv, Dv), et);
+  for (d = 0; d < Dv; ++d) o[d] /= sum;
+  *m = mx;
+  *l = sum;
+}
+
+static int ext_args_bad(int B, int Sq, int Skv, int Nq, int Nkv, int Dqk, int Dv, int mask_mode,
+                        int64_t pre, int64_t next) {
+  if (B < 0 || Sq < 0 || Skv < 0 || Nq <= 0 || Nkv <= 0 || Dqk <= 0 || Nq % Nkv) return 1;
+  if (Dv <= 0 || Dv > Dqk) return 1;
+  if (mask_mode < ORC_MASK_NONE || mask_mode > ORC_MASK_BAND) return 1;
+  if (mask_mode == ORC_MASK_BAND && pre + next < 0) return 1;
+  return 0;
+}
+
+/* Sequence b and position i of query token tok (b*Sq + i for BHSD, packed index for TND). */
+static void locate(int layout, const int32_t *cu_q, int64_t Sq, int64_t tok, int64_t *b, int64_t *i) {
+  if (layout == ORC_BHSD) {
+    *b = tok / Sq;
+    *i = tok % Sq;
+  } else {
+    int64_t bb = 0;
+    while (cu_q[bb] <= tok) ++bb;
+    *b = bb;
+    *i = tok - (bb == 0 ? 0 : cu_q[bb - 1]);
+  }
+}
+
+/*
+ * All rows: out is [B,Nq,Sq,Dv] (BHSD) or [Tq,Nq,Dv] (TND); smax/ssum as for oracle_attn_fwd.
+ * Returns 0, -1 on bad arguments, -2 on bad cumulative lengths.
+ */
+int oracle_attn_fwd_ext(const void *q, const void *k, const void *v, int et, const int32_t *cu_q,
+                        const int32_t *cu_kv, int B, int Sq, int Skv, int Nq, int Nkv, int Dqk,
+                        int Dv, double scale, int mask_mode, int64_t pre, int64_t next,
+                        const uint8_t *mask, int64_t mask_bstride, int64_t mask_rstride,
+                        int layout, double *out, double *smax, double *ssum) {
+  int64_t nrows, r, group;
+  if (ext_args_bad(B, Sq, Skv, Nq, Nkv, Dqk, Dv, mask_mode, pre, next)) return -1;
+  if (layout == ORC_TND && (check_cu(cu_q, B, Sq) || check_cu(cu_kv, B, Skv))) return -2;
+  group = Nq / Nkv;
+  nrows = (layout == ORC_BHSD ? (int64_t)B * Sq : (int64_t)Sq) * Nq;
+#pragma omp parallel
+  {
+    double *s = (double *)malloc(sizeof(double) * (size_t)(Skv > 0 ? Skv : 1));
+#pragma omp for schedule(dynamic, 16)
+    for (r = 0; r < nrows; ++r) {
+      int64_t h = r % Nq, b, i, tq0, tk0, lq, lk, so;
+      locate(layout, cu_q, Sq, r / Nq, &b, &i);
+      seq_range(layout, cu_q, b, Sq, &tq0, &lq);
+      seq_range(layout, cu_kv, b, Skv, &tk0, &lk);
+      so = layout == ORC_BHSD ? ((int64_t)b * Nq + h) * Sq + i : (tq0 + i) * Nq + h;
+      attn_row_ext(q, k, v, et, layout, b, tq0, tk0, i, h, h / group, lq, lk, Nq, Nkv, Sq, Skv,
+                   Dqk, Dv, scale, mask_mode, pre, next, mask, mask_bstride, mask_rstride, s,
+                   out + offs(layout, b, tq0, i, h, 0, Nq, Sq, Dv), smax + so, ssum + so);
+    }
+    free(s);
+  }
+  return 0;
+}
+
+/* Chosen rows only (head rows_h[r], query token rows_t[r]); out_rows is [n, Dv]. */
+int oracle_attn_fwd_ext_rows(const void *q, const void *k, const void *v, int et,
+                             const int32_t *cu_q, const int32_t *cu_kv, int B, int Sq, int Skv,
+                             int Nq, int Nkv, int Dqk, int Dv, double scale, int mask_mode,
+                             int64_t pre, int64_t next, const uint8_t *mask, int64_t mask_bstride,
+                             int64_t mask_rstride, int layout, const int32_t *rows_h,
+                             const int64_t *rows_t, int64_t n, double *out_rows, double *m_rows,
+                             double *l_rows) {
+  int64_t r, group;
+  if (ext_args_bad(B, Sq, Skv, Nq, Nkv, Dqk, Dv, mask_mode, pre, next)) return -1;
+  if (layout == ORC_TND && (check_cu(cu_q, B, Sq) || check_cu(cu_kv, B, Skv))) return -2;
+  group = Nq / Nkv;
+#pragma omp parallel
+  {
+    double *s = (double *)malloc(sizeof(double) * (size_t)(Skv > 0 ? Skv : 1));
+#pragma omp for schedule(dynamic, 1)
+    for (r = 0; r < n; ++r) {
+      int64_t h = rows_h[r], b, i, tq0, tk0, lq, lk;
+      locate(layout, cu_q, Sq, rows_t[r], &b, &i);
+      seq_range(layout, cu_q, b, Sq, &tq0, &lq);
+      seq_range(layout, cu_kv, b, Skv, &tk0, &lk);
+      attn_row_ext(q, k, v, et, layout, b, tq0, tk0, i, h, h / group, lq, lk, Nq, Nkv, Sq, Skv,
+                   Dqk, Dv, scale, mask_mode, pre, next, mask, mask_bstride, mask_rstride, s,
+                   out_rows + r * Dv, m_rows + r, l_rows + r);
+    }
+    free(s);
+  }
+  return 0;
+}
+
+/*
  * CSR-sparse attention ("paddle.nn.functional.sparse_attention"): for every (b, h, i) the
  * softmax runs over the stored entries c in [offset[i], offset[i+1]) of that (b, h) slice,
  * key j = columns[c], scale 1/sqrt(D). q, k, v, out are [B, H, S, D].

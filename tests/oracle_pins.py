@@ -322,6 +322,180 @@ def pin_rows_api_matches_full():
 
 
 # ---------------------------------------------------------------------------------------------
+# Masked forward: band limits, explicit mask, value head size
+# ---------------------------------------------------------------------------------------------
+BAND = oracle.MASK_BAND
+BIG = 1 << 40
+
+
+def _ext_bhsd(q, k, v, mode, pre=0, nxt=0, mask=None, bstride=0, rstride=0, scale=None):
+    B, Nq, Sq, D = q.shape
+    _, Nkv, Skv, Dv = v.shape
+    scale = 1.0 / math.sqrt(D) if scale is None else scale
+    return oracle.attn_fwd_ext(q, k, v, B=B, Sq=Sq, Skv=Skv, Nq=Nq, Nkv=Nkv, Dqk=D, Dv=Dv,
+                               scale=scale, mask_mode=mode, pre_tokens=pre, next_tokens=nxt,
+                               mask=mask, mask_bstride=bstride, mask_rstride=rstride, layout=BHSD)
+
+
+def _check_against_torch(out, m, l, q, k, v, vis, gqa=False):
+    """vis: bool [B, Sq, Skv] (True = attend). Rows with a visible key match torch's float64
+    SDPA with that boolean mask; rows without one give out 0, max -inf, sum 0."""
+    B, Nq, Sq, _ = q.shape
+    for b in range(B):
+        rows = vis[b].any(axis=1)
+        if rows.any():
+            mk = np.broadcast_to(vis[b][rows], (1, Nq, int(rows.sum()), vis.shape[2])).copy()
+            ref = _torch_sdpa(q[b:b + 1, :, rows], k[b:b + 1], v[b:b + 1], mask=mk, gqa=gqa)
+            assert np.max(np.abs(out[b:b + 1, :, rows] - ref)) <= 1e-12
+        assert np.all(out[b, :, ~rows] == 0.0)
+        assert np.all(np.isneginf(m[b, :, ~rows])) and np.all(l[b, :, ~rows] == 0.0)
+
+
+def pin_band_matches_torch_mask():
+    """Band reading: key j visible to row i iff i - pre <= j <= i + next."""
+    r = _rng(30)
+    for (Sq, Skv) in [(9, 9), (6, 11), (11, 6)]:
+        B, Nq, Nkv, D = 2, 4, 2, 3
+        q = r.standard_normal((B, Nq, Sq, D))
+        k = r.standard_normal((B, Nkv, Skv, D))
+        v = r.standard_normal((B, Nkv, Skv, D))
+        i, j = np.arange(Sq)[:, None], np.arange(Skv)[None, :]
+        for pre, nxt in [(2, 1), (0, 0), (3, -1), (-1, 3), (0, 5), (100, 100), (-4, 4)]:
+            out, m, l = _ext_bhsd(q, k, v, BAND, pre, nxt)
+            vis = np.broadcast_to((j >= i - pre) & (j <= i + nxt), (B, Sq, Skv))
+            _check_against_torch(out, m, l, q, k, v, vis, gqa=True)
+
+
+def pin_band_limits_and_diagonal():
+    r = _rng(31)
+    B, H, S, D = 2, 2, 8, 3
+    q, k, v = (r.standard_normal((B, H, S, D)) for _ in range(3))
+    # an unbounded band is the full attention; no look-ahead with unbounded look-back is causal
+    o_full, m_full, l_full = _bhsd(q, k, v, NONE)
+    o_b, m_b, l_b = _ext_bhsd(q, k, v, BAND, BIG, BIG)
+    assert np.max(np.abs(o_b - o_full)) <= 1e-14 and np.max(np.abs(l_b - l_full)) <= 1e-13
+    o_c, _, _ = _bhsd(q, k, v, TL)
+    o_b, _, _ = _ext_bhsd(q, k, v, BAND, BIG, 0)
+    assert np.max(np.abs(o_b - o_c)) <= 1e-14
+    # a band of width one: each row sees only its own key, o = v_i, sum = 1, max = scale q_i.k_i
+    o, m, l = _ext_bhsd(q, k, v, BAND, 0, 0)
+    assert np.array_equal(o, v) and np.all(l == 1.0)
+    assert np.max(np.abs(m - np.einsum("bhsd,bhsd->bhs", q, k) / math.sqrt(D))) <= 1e-15
+
+
+def pin_explicit_mask_matches_torch():
+    """uint8 mask, 1 = excluded, element (b, i, j) at b*bstride + i*rstride + j; combined
+    with the mode by AND."""
+    r = _rng(32)
+    B, Nq, Nkv, Sq, Skv, D = 3, 2, 1, 7, 10, 4
+    q = r.standard_normal((B, Nq, Sq, D))
+    k = r.standard_normal((B, Nkv, Skv, D))
+    v = r.standard_normal((B, Nkv, Skv, D))
+    rs = Skv + 3                                   # padded rows
+    bs = Sq * rs + 5                               # padded batches
+    flat = (r.random(B * bs) < 0.35).astype(np.uint8)
+    flat[1 * bs + 2 * rs: 1 * bs + 2 * rs + Skv] = 1   # batch 1, row 2 fully excluded
+    excl = np.stack([flat[b * bs: b * bs + Sq * rs].reshape(Sq, rs)[:, :Skv] for b in range(B)])
+    i, j = np.arange(Sq)[:, None], np.arange(Skv)[None, :]
+    for mode, base in [(NONE, np.ones((Sq, Skv), bool)), (TL, j <= i), (BR, j <= i + Skv - Sq),
+                       (BAND, (j >= i - 1) & (j <= i + 2))]:
+        out, m, l = _ext_bhsd(q, k, v, mode, 1, 2, mask=flat, bstride=bs, rstride=rs)
+        _check_against_torch(out, m, l, q, k, v, (excl == 0) & base[None], gqa=True)
+    # stride 0 across batches: one mask shared by every batch
+    out, m, l = _ext_bhsd(q, k, v, NONE, mask=flat, bstride=0, rstride=rs)
+    _check_against_torch(out, m, l, q, k, v, np.broadcast_to(excl[0] == 0, (B, Sq, Skv)), gqa=True)
+
+
+def pin_value_head_size():
+    """qD == kD >= vD: the scores use D = Dqk, the output has Dv columns (torch SDPA allows a
+    value head size of its own)."""
+    r = _rng(33)
+    B, H, Sq, Skv, D = 2, 3, 6, 9, 8
+    for Dv in (1, 3, 8):
+        q = r.standard_normal((B, H, Sq, D))
+        k = r.standard_normal((B, H, Skv, D))
+        v = r.standard_normal((B, H, Skv, Dv))
+        out, _, _ = _ext_bhsd(q, k, v, NONE)
+        assert out.shape == (B, H, Sq, Dv)
+        assert np.max(np.abs(out - _torch_sdpa(q, k, v))) <= 1e-12
+        i, j = np.arange(Sq)[:, None], np.arange(Skv)[None, :]
+        out, m, l = _ext_bhsd(q, k, v, BR)
+        _check_against_torch(out, m, l, q, k, v, np.broadcast_to(j <= i + Skv - Sq, (B, Sq, Skv)))
+
+
+def pin_ext_varlen_per_sequence():
+    """TND with a band and a per-sequence mask equals torch on each sequence's slice; the mask
+    is indexed by in-sequence positions with one batch stride per sequence."""
+    r = _rng(34)
+    lens_q = np.array([5, 0, 7, 3])
+    lens_k = np.array([6, 4, 7, 0])
+    cq, ck = W.cu_seqlens_from_lengths(lens_q), W.cu_seqlens_from_lengths(lens_k)
+    Tq, Tk, Nq, Nkv, D, Dv = int(cq[-1]), int(ck[-1]), 4, 2, 3, 2
+    q = r.standard_normal((Tq, Nq, D))
+    k = r.standard_normal((Tk, Nkv, D))
+    v = r.standard_normal((Tk, Nkv, Dv))
+    rs, bs = 8, 8 * 8
+    flat = (r.random(len(lens_q) * bs) < 0.3).astype(np.uint8)
+    pre, nxt = 2, 1
+    out, m, l = oracle.attn_fwd_ext(q, k, v, cu_q=cq, cu_kv=ck, B=len(lens_q), Sq=Tq, Skv=Tk,
+                                    Nq=Nq, Nkv=Nkv, Dqk=D, Dv=Dv, scale=0.4, mask_mode=BAND,
+                                    pre_tokens=pre, next_tokens=nxt, mask=flat, mask_bstride=bs,
+                                    mask_rstride=rs, layout=TND)
+    sq0 = np.concatenate([[0], cq[:-1]])
+    sk0 = np.concatenate([[0], ck[:-1]])
+    for b in range(len(lens_q)):
+        Sq, Skv = int(lens_q[b]), int(lens_k[b])
+        if Sq == 0:
+            continue
+        i, j = np.arange(Sq)[:, None], np.arange(Skv)[None, :]
+        excl = flat[b * bs: b * bs + Sq * rs].reshape(Sq, rs)[:, :Skv]
+        vis = ((j >= i - pre) & (j <= i + nxt) & (excl == 0))[None]
+        qs = _slice_bhsd(q, sq0[b], cq[b])
+        ks, vs = _slice_bhsd(k, sk0[b], ck[b]), _slice_bhsd(v, sk0[b], ck[b])
+        o_b = np.transpose(out[sq0[b]:cq[b]], (1, 0, 2))[None]
+        m_b = m[sq0[b]:cq[b]].T[None]
+        l_b = l[sq0[b]:cq[b]].T[None]
+        if Skv == 0:
+            assert np.all(o_b == 0.0) and np.all(np.isneginf(m_b)) and np.all(l_b == 0.0)
+            continue
+        def sd(qq, kk, vv, mask=None, gqa=False):
+            return F.scaled_dot_product_attention(
+                torch.from_numpy(qq), torch.from_numpy(kk), torch.from_numpy(vv),
+                attn_mask=None if mask is None else torch.from_numpy(mask), scale=0.4,
+                enable_gqa=gqa).numpy()
+        rows = vis[0].any(axis=1)
+        if rows.any():
+            mk = np.broadcast_to(vis[0][rows], (1, Nq, int(rows.sum()), Skv)).copy()
+            ref = sd(qs[:, :, rows], ks, vs, mask=mk, gqa=True)
+            assert np.max(np.abs(o_b[:, :, rows] - ref)) <= 1e-12
+        assert np.all(o_b[:, :, ~rows] == 0.0) and np.all(l_b[:, :, ~rows] == 0.0)
+
+
+def pin_ext_rows_and_rejections():
+    r = _rng(35)
+    B, Nq, Nkv, S, D, Dv = 2, 4, 2, 9, 4, 2
+    q = r.standard_normal((B, Nq, S, D))
+    k = r.standard_normal((B, Nkv, S, D))
+    v = r.standard_normal((B, Nkv, S, Dv))
+    mask = (r.random(S * S) < 0.2).astype(np.uint8)
+    kw = dict(B=B, Sq=S, Skv=S, Nq=Nq, Nkv=Nkv, Dqk=D, Dv=Dv, scale=0.3, mask_mode=BAND,
+              pre_tokens=3, next_tokens=2, mask=mask, mask_bstride=0, mask_rstride=S, layout=BHSD)
+    out, m, l = oracle.attn_fwd_ext(q, k, v, **kw)
+    rows_t = np.array([0, 5, 9, 17, 12])
+    rows_h = np.array([1, 0, 3, 2, 2])
+    o2, m2, l2 = oracle.attn_fwd_ext_rows(q, k, v, rows_h, rows_t, **kw)
+    b, i = rows_t // S, rows_t % S
+    assert np.array_equal(o2, out[b, rows_h, i])
+    assert np.array_equal(m2, m[b, rows_h, i]) and np.array_equal(l2, l[b, rows_h, i])
+    for bad in (dict(pre_tokens=-3, next_tokens=2), dict(Dv=D + 1), dict(mask_mode=4)):
+        try:
+            oracle.attn_fwd_ext(q, k, v, **{**kw, **bad})
+        except ValueError:
+            continue
+        raise AssertionError(f"accepted {bad}")
+
+
+# ---------------------------------------------------------------------------------------------
 # Merge (ring-attention update)
 # ---------------------------------------------------------------------------------------------
 def _to_sbh(o_bnsd):

@@ -44,6 +44,13 @@ MUTANTS = [
      "ld(prev_out, x, et) * co + ld(cur_out, x, et) * po", 0),
     ("merge_sum_not_rescaled", "cs_scaled[lane] = cur_sum[x] * exp(cm - m);", "cs_scaled[lane] = cur_sum[x];", 0),
     ("bf16_truncates", "nearbyint(m * 256.0)", "floor(m * 256.0)", 0),
+    ("band_lower_off_by_one", "(j < i - pre || j > i + next)", "(j <= i - pre || j > i + next)", 0),
+    ("band_upper_sign", "(j < i - pre || j > i + next)", "(j < i - pre || j > i - next)", 0),
+    ("mask_polarity", "mask[mrow + i * mask_rstride + j] != 0", "mask[mrow + i * mask_rstride + j] == 0", 0),
+    ("mask_row_stride_ignored", "mask[mrow + i * mask_rstride + j]", "mask[mrow + i * sk + j]", 0),
+    ("mask_batch_stride_ignored", "b * mask_bstride, mask_rstride))", "0 * mask_bstride, mask_rstride))", 0),
+    ("mask_key_shifted", "mask[mrow + i * mask_rstride + j]", "mask[mrow + i * mask_rstride + (j + 1) % sk]", 0),
+    ("scores_over_value_dims", "for (d = 0; d < Dqk; ++d)\n      acc +=", "for (d = 0; d < Dv; ++d)\n      acc +=", 0),
 ]
 
 
