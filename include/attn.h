@@ -7,6 +7,7 @@
  *   attn_sparse_csr  the same softmax restricted to the entries of a CSR pattern (fp32).
  *   attn_merge       merge of two partial attention results from their max/sum statistics.
  *   attn_fwd_accumulate  attn_fwd over one chunk of keys folded into a running merge result.
+ *   attn_fwd_masked  attn_fwd with band limits, an explicit mask and a value head size Dv.
  *
  * Conventions shared by every call
  *   - All tensor pointers are DEVICE pointers owned by the caller. The library allocates no
@@ -61,7 +62,8 @@ typedef enum { ATTN_BHSD = 0, ATTN_TND = 1 } attn_layout;
 typedef enum {
   ATTN_MASK_NONE = 0,
   ATTN_MASK_CAUSAL_TOPLEFT = 1,    /* key j visible to query i iff j <= i                  */
-  ATTN_MASK_CAUSAL_BOTTOMRIGHT = 2 /* key j visible iff j <= i + Skv_b - Sq_b (per sequence) */
+  ATTN_MASK_CAUSAL_BOTTOMRIGHT = 2, /* key j visible iff j <= i + Skv_b - Sq_b (per sequence) */
+  ATTN_MASK_BAND = 3               /* attn_fwd_masked only: i - pre_tokens <= j <= i + next_tokens */
 } attn_mask;
 
 /*
@@ -86,7 +88,8 @@ typedef enum {
  * dtype: ATTN_BF16 or ATTN_F16 (q, k, v, out bfloat16 or float16; tensor cores with fp32
  *        accumulation; D = 64 or 128), or ATTN_F32 (float32 throughout, CUDA-core FMA;
  *        1 <= D <= 256).
- * softmax_max / softmax_sum may both be NULL to skip the statistics.
+ * softmax_max / softmax_sum may both be NULL to skip the statistics. mask_mode is 0, 1 or 2
+ * (the band needs attn_fwd_masked).
  * Limits (from the constraints): 1 <= Nq <= 256, D <= 768 (larger D is ATTN_ERR_INVALID;
  * sizes this build does not run are ATTN_ERR_UNSUPPORTED), Tq, Tkv <= 1M tokens and
  * B <= 2048 for TND; scale must be finite and > 0. Empty problems (B = 0, Sq = 0 or a total
@@ -126,6 +129,44 @@ ATTN_API int attn_fwd_accumulate(const void* q, const void* k, const void* v,
                                  int B, int Sq, int Skv, int Nq, int Nkv, int D,
                                  float scale, int mask_mode, int dtype, int layout, int first,
                                  void* acc_out, float* acc_max, float* acc_sum, void* stream);
+
+/*
+ * attn_fwd_masked -- attn_fwd with a band (preTokens / nextTokens), an optional explicit mask
+ * and a value head size of its own.
+ *
+ * Defined by: the attn_fwd definition above, restricted to the keys that pass both the mode
+ * and the mask; "aclnnFlashAttentionVarLenScore" (CANN 8.5 API doc), 约束说明, which lists
+ * preTokens / nextTokens, attenMaskOptional and the head-size rule qD == kD >= vD. The page
+ * does not carry the table that defines the sparse modes, so this call takes these readings:
+ *   mask_mode ATTN_MASK_BAND: key j is visible to query row i iff
+ *     i - pre_tokens <= j <= i + next_tokens, with i and j positions within the sequence
+ *     (top-left aligned); pre_tokens + next_tokens must be >= 0 (the band is not empty).
+ *     pre_tokens and next_tokens are ignored by the other modes. Values beyond +-2^30 act as
+ *     unbounded.
+ *   atten_mask (may be NULL): uint8, 1 = the key is masked out, 0 = it may be attended; the
+ *     entry for (sequence b, query position i, key position j) is
+ *     atten_mask[b * mask_batch_stride + i * mask_row_stride + j] (positions within the
+ *     sequence for TND; mask_batch_stride = 0 shares one mask across the batch). The caller
+ *     guarantees that every addressed entry lies inside its buffer: for BHSD,
+ *     mask_row_stride >= Skv; for TND, the mask must cover each sequence's lengths.
+ *     A key must pass both the mode and the mask.
+ *   Dv: v is [B, Nkv, Skv, Dv] (BHSD) or [Tkv, Nkv, Dv] (TND) and out is [B, Nq, Sq, Dv] or
+ *     [Tq, Nq, Dv]; 1 <= Dv <= Dqk. q and k have head size Dqk.
+ * Other arguments, statistics, limits and errors are those of attn_fwd (D there is Dqk).
+ * Supported: ATTN_F32 with Dv <= Dqk <= 256; ATTN_BF16 and ATTN_F16 with Dqk = Dv = 64 or 128
+ * (other Dv are ATTN_ERR_UNSUPPORTED there). On the tensor-core path a mask given with
+ * atten_mask, mask_row_stride and mask_batch_stride all 16-byte aligned is read 16 bytes at a
+ * time, otherwise byte by byte.
+ * Errors: mask_mode outside 0..3, pre_tokens + next_tokens < 0 with the band, negative
+ * strides, Dv outside 1..Dqk, or a BHSD mask_row_stride < Skv give ATTN_ERR_INVALID.
+ */
+ATTN_API int attn_fwd_masked(const void* q, const void* k, const void* v,
+                             const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_kv,
+                             int B, int Sq, int Skv, int Nq, int Nkv, int Dqk, int Dv,
+                             float scale, int mask_mode, int64_t pre_tokens, int64_t next_tokens,
+                             const uint8_t* atten_mask, int64_t mask_batch_stride,
+                             int64_t mask_row_stride, int dtype, int layout,
+                             void* out, float* softmax_max, float* softmax_sum, void* stream);
 
 /*
  * attn_sparse_csr -- CSR-sparse attention forward, float32.

@@ -18,13 +18,14 @@ from typing import Optional
 __all__ = [
     "attn_fwd", "attn_fwd_accumulate", "attn_sparse_csr", "attn_merge", "attn_get_last_error", "AttnError",
     "ATTN_BF16", "ATTN_F32", "ATTN_F16", "ATTN_BHSD", "ATTN_TND", "ATTN_MASK_NONE",
-    "ATTN_MASK_CAUSAL_TOPLEFT", "ATTN_MASK_CAUSAL_BOTTOMRIGHT", "lib_path", "load_library",
+    "ATTN_MASK_CAUSAL_TOPLEFT", "ATTN_MASK_CAUSAL_BOTTOMRIGHT", "ATTN_MASK_BAND", "lib_path",
+    "load_library", "attn_fwd_masked",
 ]
 
 ATTN_OK, ATTN_ERR_INVALID, ATTN_ERR_UNSUPPORTED, ATTN_ERR_CUDA, ATTN_ERR_DATA, ATTN_ERR_TIMEOUT = range(6)
 ATTN_BF16, ATTN_F32, ATTN_F16 = 0, 1, 2
 ATTN_BHSD, ATTN_TND = 0, 1
-ATTN_MASK_NONE, ATTN_MASK_CAUSAL_TOPLEFT, ATTN_MASK_CAUSAL_BOTTOMRIGHT = 0, 1, 2
+ATTN_MASK_NONE, ATTN_MASK_CAUSAL_TOPLEFT, ATTN_MASK_CAUSAL_BOTTOMRIGHT, ATTN_MASK_BAND = 0, 1, 2, 3
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _lock = threading.Lock()
@@ -57,6 +58,9 @@ def load_library():
         lib.attn_fwd.restype = I
         lib.attn_fwd_accumulate.argtypes = [P, P, P, P, P, I, I, I, I, I, I, F, I, I, I, I, P, P, P, P]
         lib.attn_fwd_accumulate.restype = I
+        lib.attn_fwd_masked.argtypes = [P, P, P, P, P, I, I, I, I, I, I, I, F, I, I64, I64, P, I64,
+                                        I64, I, I, P, P, P, P]
+        lib.attn_fwd_masked.restype = I
         lib.attn_sparse_csr.argtypes = [P, P, P, P, P, I, I, I, I, I64, P, P]
         lib.attn_sparse_csr.restype = I
         lib.attn_merge.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, P, P, P, P, P]
@@ -123,6 +127,22 @@ def attn_fwd_accumulate(q, k, v, *, cu_seqlens_q=None, cu_seqlens_kv=None, B: in
                                    int(D), float(scale), int(mask_mode), int(dtype), int(layout),
                                    1 if first else 0, _ptr(acc_out), _ptr(acc_max), _ptr(acc_sum),
                                    _stream(stream)), "attn_fwd_accumulate")
+
+
+def attn_fwd_masked(q, k, v, *, cu_seqlens_q=None, cu_seqlens_kv=None, B: int, Sq: int, Skv: int,
+                    Nq: int, Nkv: int, Dqk: int, Dv: int, scale: float, mask_mode: int,
+                    pre_tokens: int = 0, next_tokens: int = 0, atten_mask=None,
+                    mask_batch_stride: int = 0, mask_row_stride: int = 0, dtype: int, layout: int,
+                    out, softmax_max=None, softmax_sum=None, stream=None) -> None:
+    """attn_fwd with a band, an optional uint8 mask (1 = excluded) and a value head size Dv
+    (see ``attn_fwd_masked`` in include/attn.h)."""
+    lib = load_library()
+    _check(lib.attn_fwd_masked(_ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens_q), _ptr(cu_seqlens_kv),
+                               int(B), int(Sq), int(Skv), int(Nq), int(Nkv), int(Dqk), int(Dv),
+                               float(scale), int(mask_mode), int(pre_tokens), int(next_tokens),
+                               _ptr(atten_mask), int(mask_batch_stride), int(mask_row_stride),
+                               int(dtype), int(layout), _ptr(out), _ptr(softmax_max),
+                               _ptr(softmax_sum), _stream(stream)), "attn_fwd_masked")
 
 
 def attn_sparse_csr(q, k, v, csr_offset, csr_columns, *, B: int, H: int, S: int, D: int,

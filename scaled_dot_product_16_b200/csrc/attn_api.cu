@@ -70,13 +70,33 @@ const char* attn_status_string(int s) {
 
 namespace {
 
+// The masked-call extras of fwd_impl (band limits, explicit mask, value head size).
+struct Extras {
+  bool allow_band = false;
+  int Dv = -1;  // -1: same as D
+  int64_t pre = 0, next = 0;
+  const uint8_t* mask = nullptr;
+  int64_t mask_bs = 0, mask_rs = 0;
+};
+
+int clamp30(int64_t x) {
+  const int64_t lim = int64_t(1) << 30;
+  return (int)(x < -lim ? -lim : (x > lim ? lim : x));
+}
+
 int fwd_impl(const void* q, const void* k, const void* v, const int32_t* cu_seqlens_q,
              const int32_t* cu_seqlens_kv, int B, int Sq, int Skv, int Nq, int Nkv, int D,
              float scale, int mask_mode, int dtype, int layout, void* out, float* softmax_max,
-             float* softmax_sum, int acc_mode, void* stream) {
+             float* softmax_sum, int acc_mode, void* stream, const Extras& x = Extras()) {
   if (layout != ATTN_BHSD && layout != ATTN_TND) return ATTN_ERR_INVALID;
   if (dtype != ATTN_BF16 && dtype != ATTN_F32 && dtype != ATTN_F16) return ATTN_ERR_INVALID;
-  if (mask_mode < ATTN_MASK_NONE || mask_mode > ATTN_MASK_CAUSAL_BOTTOMRIGHT) return ATTN_ERR_INVALID;
+  const int max_mode = x.allow_band ? ATTN_MASK_BAND : ATTN_MASK_CAUSAL_BOTTOMRIGHT;
+  if (mask_mode < ATTN_MASK_NONE || mask_mode > max_mode) return ATTN_ERR_INVALID;
+  if (mask_mode == ATTN_MASK_BAND && clamp30(x.pre) + clamp30(x.next) < 0) return ATTN_ERR_INVALID;
+  const int Dv = x.Dv < 0 ? D : x.Dv;
+  if (Dv < 1 || Dv > D) return ATTN_ERR_INVALID;
+  if (x.mask != nullptr && (x.mask_bs < 0 || x.mask_rs < 0)) return ATTN_ERR_INVALID;
+  if (x.mask != nullptr && layout == ATTN_BHSD && x.mask_rs < Skv) return ATTN_ERR_INVALID;
   if (B < 0 || Sq < 0 || Skv < 0) return ATTN_ERR_INVALID;
   if (Nq < 1 || Nq > 256 || Nkv < 1 || Nq % Nkv != 0) return ATTN_ERR_INVALID;
   if (D < 1 || D > 768) return ATTN_ERR_INVALID;
@@ -96,6 +116,7 @@ int fwd_impl(const void* q, const void* k, const void* v, const int32_t* cu_seql
   if (dtype == ATTN_F32 && D > 256) return ATTN_ERR_UNSUPPORTED;
   if (dtype == ATTN_BF16 || dtype == ATTN_F16) {
     if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
+    if (Dv != D) return ATTN_ERR_UNSUPPORTED;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return ATTN_ERR_INVALID;
   }
 
@@ -111,8 +132,15 @@ int fwd_impl(const void* q, const void* k, const void* v, const int32_t* cu_seql
   a.Nq = Nq;
   a.Nkv = Nkv;
   a.D = D;
+  a.Dv = Dv;
   a.scale = scale;
   a.mask_mode = mask_mode;
+  a.pre = clamp30(x.pre);
+  a.next = clamp30(x.next);
+  a.mask = x.mask;
+  a.mask_bs = x.mask_bs;
+  a.mask_rs = x.mask_rs;
+  a.mask_vec = x.mask != nullptr && aligned16(x.mask) && (x.mask_bs & 15) == 0 && (x.mask_rs & 15) == 0;
   a.layout = layout;
   a.dtype = dtype;
   a.acc_mode = acc_mode;
@@ -146,6 +174,24 @@ int attn_fwd_accumulate(const void* q, const void* k, const void* v, const int32
   if (first != 0 && first != 1) return ATTN_ERR_INVALID;
   return fwd_impl(q, k, v, cu_seqlens_q, cu_seqlens_kv, B, Sq, Skv, Nq, Nkv, D, scale, mask_mode,
                   dtype, layout, acc_out, acc_max, acc_sum, first ? 1 : 2, stream);
+}
+
+int attn_fwd_masked(const void* q, const void* k, const void* v, const int32_t* cu_seqlens_q,
+                    const int32_t* cu_seqlens_kv, int B, int Sq, int Skv, int Nq, int Nkv, int Dqk,
+                    int Dv, float scale, int mask_mode, int64_t pre_tokens, int64_t next_tokens,
+                    const uint8_t* atten_mask, int64_t mask_batch_stride, int64_t mask_row_stride,
+                    int dtype, int layout, void* out, float* softmax_max, float* softmax_sum,
+                    void* stream) {
+  Extras x;
+  x.allow_band = true;
+  x.Dv = Dv < 1 ? 0 : Dv;  // 0 is rejected as out of range
+  x.pre = pre_tokens;
+  x.next = next_tokens;
+  x.mask = atten_mask;
+  x.mask_bs = mask_batch_stride;
+  x.mask_rs = mask_row_stride;
+  return fwd_impl(q, k, v, cu_seqlens_q, cu_seqlens_kv, B, Sq, Skv, Nq, Nkv, Dqk, scale, mask_mode,
+                  dtype, layout, out, softmax_max, softmax_sum, 0, stream, x);
 }
 
 int attn_sparse_csr(const float* q, const float* k, const float* v, const int32_t* csr_offset,

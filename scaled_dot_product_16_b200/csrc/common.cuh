@@ -22,11 +22,19 @@ __device__ __forceinline__ void seq_span(const int32_t* cu, int b, int* start, i
   *len = __ldg(cu + b) - lo;
 }
 
-// Keys visible to query row i are 0 .. visible_end(i) - 1 (every mask here is a prefix).
-__device__ __forceinline__ int visible_end(int mask_mode, int i, int sq, int sk) {
+// Keys visible to query row i under the mode are visible_begin(i) .. visible_end(i) - 1: a
+// prefix for the causal modes, a window i - pre .. i + next for the band (both limits within
+// +-2^30, so the sums below stay in int range).
+__device__ __forceinline__ int visible_end(int mask_mode, int i, int sq, int sk, int next = 0) {
   if (mask_mode == ATTN_MASK_NONE) return sk;
-  const int last = mask_mode == ATTN_MASK_CAUSAL_TOPLEFT ? i : i + sk - sq;
+  const int last = mask_mode == ATTN_MASK_CAUSAL_TOPLEFT ? i
+                   : mask_mode == ATTN_MASK_BAND         ? i + next
+                                                         : i + sk - sq;
   return last < 0 ? 0 : (last + 1 < sk ? last + 1 : sk);
+}
+__device__ __forceinline__ int visible_begin(int mask_mode, int i, int pre) {
+  if (mask_mode != ATTN_MASK_BAND) return 0;
+  return i - pre > 0 ? i - pre : 0;
 }
 
 // Find which query tile of a packed batch this block owns. Sequence b contributes

@@ -187,7 +187,7 @@ struct Work {
   int row0;         // first row (within the sequence) of this block's 256 rows
 };
 
-template <int HD, bool F16>
+template <int HD, bool F16, bool MASKED>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, FwdArgs a, int units_per_seq,
@@ -256,10 +256,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int rows0 = min(kBM, w.sq - w.row0);
   const int rows1 = min(kBM, w.sq - w.row0 - kBM);  // <= 0: no second tile
   const bool has1 = rows1 > 0;
-  const int kv_end0 = visible_end(a.mask_mode, w.row0 + rows0 - 1, w.sq, w.sk);
-  const int kv_end1 = has1 ? visible_end(a.mask_mode, w.row0 + kBM + rows1 - 1, w.sq, w.sk) : 0;
-  const int n0 = (kv_end0 + kBN - 1) / kBN;
-  const int n1 = has1 ? (kv_end1 + kBN - 1) / kBN : n0;  // tiles loaded (n1 >= n0)
+  // Key tiles run from jlo (the band's first tile for the block's first row; 0 otherwise) to
+  // the tile holding each Q tile's last visible key; n0 and n1 count tiles from jlo.
+  const int jlo = visible_begin(a.mask_mode, w.row0, a.pre) / kBN;
+  const int kv_end0 = visible_end(a.mask_mode, w.row0 + rows0 - 1, w.sq, w.sk, a.next);
+  const int kv_end1 = has1 ? visible_end(a.mask_mode, w.row0 + kBM + rows1 - 1, w.sq, w.sk, a.next) : 0;
+  const int n0 = max((kv_end0 + kBN - 1) / kBN, jlo) - jlo;
+  const int n1 = has1 ? max((kv_end1 + kBN - 1) / kBN, jlo) - jlo : n0;  // tiles loaded (n1 >= n0)
 
   const uint32_t bar_base = smem_u32(bars);
   auto bar_addr = [&](const uint64_t* p) { return smem_u32(p); };
@@ -323,7 +326,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t fb = bar_addr(&bars->kv_full[s]);
         mbar_arrive_expect_tx(fb, C::kTileBytes);
         const int j = i >> 1;
-        load_tile((i & 1) ? &tm_v : &tm_k, sKV + s * C::kTileBytes, fb, w.k0 + j * kBN, khead);
+        load_tile((i & 1) ? &tm_v : &tm_k, sKV + s * C::kTileBytes, fb, w.k0 + (jlo + j) * kBN, khead);
       }
       // drain: every stage this thread filled must have landed before the block exits
       for (int i = max(0, issued - C::kStages); i < issued; ++i) {
@@ -426,7 +429,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     const uint32_t S = tmem + lane_off + q * 128;
     const uint32_t O = tmem + lane_off + 256 + q * HD;
-    const int lim = i < w.sq ? visible_end(a.mask_mode, i, w.sq, w.sk) : w.sk;
+    const int lim = i < w.sq ? visible_end(a.mask_mode, i, w.sq, w.sk, a.next) : w.sk;
+    const int lo = i < w.sq ? visible_begin(a.mask_mode, i, a.pre) : 0;
+    // explicit mask row of this query (rows past the sequence read none)
+    const uint8_t* mrow = nullptr;
+    if constexpr (MASKED)
+      if (i < w.sq) mrow = a.mask + (int64_t)w.b * a.mask_bs + (int64_t)i * a.mask_rs;
 
     float m = -INFINITY;        // running max used for P (log2 units, lazily updated)
     float mraw = -INFINITY;     // true max of the raw scores q.k
@@ -437,15 +445,51 @@ __global__ void __launch_bounds__(kThreads, 1)
         ok = __all_sync(0xffffffffu, wait_bar(bar_addr(&bars->s_full[q]), j & 1, abort, a.status));
         if (!ok) break;
         tc_fence_after();
+        const int kbase = (jlo + j) * kBN;
+        uint4 mk[MASKED ? 8 : 1];
+        if constexpr (MASKED) {
+          // the mask bytes of this row's 128 keys (16 at a time when aligned and whole);
+          // issued before the TMEM loads so the two latencies overlap
+          if (mrow != nullptr && a.mask_vec && kbase + kBN <= w.sk) {
+            const uint4* src = reinterpret_cast<const uint4*>(mrow + kbase);
+#pragma unroll
+            for (int x = 0; x < 8; ++x) mk[x] = __ldg(src + x);
+          } else {
+#pragma unroll
+            for (int x = 0; x < 8; ++x) {
+              uint32_t wd[4];
+#pragma unroll
+              for (int y = 0; y < 4; ++y) {
+                uint32_t word = 0;
+#pragma unroll
+                for (int z = 0; z < 4; ++z) {
+                  const int c = x * 16 + y * 4 + z;
+                  const uint32_t byte = (mrow != nullptr && kbase + c < w.sk) ? mrow[kbase + c] : 0u;
+                  word |= (byte != 0u ? 1u : 0u) << (8 * z);
+                }
+                wd[y] = word;
+              }
+              mk[x] = make_uint4(wd[0], wd[1], wd[2], wd[3]);
+            }
+          }
+        }
         float s[4][32];
 #pragma unroll
         for (int c = 0; c < 4; ++c) tmem_ld32f(S + c * 32, s[c]);
         tmem_wait_ld();
-        const int kbase = j * kBN;
-        if (kbase + kBN > lim) {
+        if (kbase + kBN > lim || kbase < lo) {
 #pragma unroll
           for (int c = 0; c < kBN; ++c)
-            if (kbase + c >= lim) s[c >> 5][c & 31] = -INFINITY;
+            if (kbase + c >= lim || kbase + c < lo) s[c >> 5][c & 31] = -INFINITY;
+        }
+        if constexpr (MASKED) {
+#pragma unroll
+          for (int c = 0; c < kBN; ++c) {
+            const uint4 v4 = mk[c >> 4];
+            const uint32_t wd = ((c >> 2) & 3) == 0 ? v4.x : ((c >> 2) & 3) == 1 ? v4.y
+                              : ((c >> 2) & 3) == 2 ? v4.z : v4.w;
+            if ((wd >> (8 * (c & 3))) & 0xffu) s[c >> 5][c & 31] = -INFINITY;
+          }
         }
         // row max: a tree of 3-input maxima over the 128 scores
         float mx[8];
@@ -649,8 +693,8 @@ cudaError_t launch_hd(const FwdArgs& a, cudaStream_t st) {
          make_map(&tv, a.v, D, a.Nkv, tk_rows, D * 2, (uint64_t)a.Nkv * D * 2, 1, kBN, F16);
   }
   if (!ok) return cudaErrorInvalidValue;
-  cudaError_t e = cudaFuncSetAttribute(fwd_bf16_kernel<HD, F16>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+  auto kernel = a.mask != nullptr ? fwd_bf16_kernel<HD, F16, true> : fwd_bf16_kernel<HD, F16, false>;
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return e;
   int units_per_seq = 0;
   int64_t units;
@@ -664,8 +708,7 @@ cudaError_t launch_hd(const FwdArgs& a, cudaStream_t st) {
   if (blocks <= 0) return cudaSuccess;
   if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
   const float scale_log2 = a.scale * 1.4426950408889634f;
-  fwd_bf16_kernel<HD, F16><<<(unsigned)blocks, kThreads, C::kSmemBytes, st>>>(tq, tk, tv, a,
-                                                                           units_per_seq, scale_log2);
+  kernel<<<(unsigned)blocks, kThreads, C::kSmemBytes, st>>>(tq, tk, tv, a, units_per_seq, scale_log2);
   return cudaGetLastError();
 }
 

@@ -26,12 +26,12 @@ constexpr int kRowsPerWarp = kBM / kWarps;
 template <int DMAX>
 __global__ void __launch_bounds__(kWarps * 32) fwd_f32_kernel(FwdArgs a, int tiles_per_seq) {
   extern __shared__ float smem[];
-  const int D = a.D;
+  const int D = a.D, Dv = a.Dv;
   const int ldk = D + 1;  // padded row of the K tile: lane-strided reads avoid bank conflicts
   float* sQ = smem;                       // [kBM][D]
   float* sK = sQ + kBM * D;               // [kBN][D+1]
-  float* sV = sK + kBN * ldk;             // [kBN][D]
-  float* sP = sV + kBN * D;               // [kWarps][kRowsPerWarp][kBN]
+  float* sV = sK + kBN * ldk;             // [kBN][Dv]
+  float* sP = sV + kBN * Dv;              // [kWarps][kRowsPerWarp][kBN]
   __shared__ int s_info[4];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -91,6 +91,16 @@ __global__ void __launch_bounds__(kWarps * 32) fwd_f32_kernel(FwdArgs a, int til
     return a.layout == ATTN_BHSD ? (((int64_t)b * a.Nkv + g) * a.Skv + j) * D
                                  : ((int64_t)(k0 + j) * a.Nkv + g) * D;
   };
+  // value rows and output rows have Dv columns
+  auto voff = [&](int j) -> int64_t {
+    return a.layout == ATTN_BHSD ? (((int64_t)b * a.Nkv + g) * a.Skv + j) * Dv
+                                 : ((int64_t)(k0 + j) * a.Nkv + g) * Dv;
+  };
+  auto ooff = [&](int i) -> int64_t {
+    return a.layout == ATTN_BHSD ? (((int64_t)b * a.Nq + h) * a.Sq + i) * Dv
+                                 : ((int64_t)(q0 + i) * a.Nq + h) * Dv;
+  };
+  const uint8_t* mrow0 = a.mask != nullptr ? a.mask + (int64_t)b * a.mask_bs : nullptr;
 
   const int row0 = qt * kBM;
   const int nrows = min(kBM, sq - row0);
@@ -100,30 +110,35 @@ __global__ void __launch_bounds__(kWarps * 32) fwd_f32_kernel(FwdArgs a, int til
     sQ[x] = r < nrows ? Q[qoff(row0 + r) + d] : 0.f;
   }
 
-  // keys needed by the last row of the tile
-  const int kv_end = visible_end(a.mask_mode, row0 + nrows - 1, sq, sk);
+  // keys needed by the tile: from the first row's first visible key to the last row's last
+  const int kv_end = visible_end(a.mask_mode, row0 + nrows - 1, sq, sk, a.next);
+  const int kv_begin = visible_begin(a.mask_mode, row0, a.pre) / kBN * kBN;
 
   constexpr int DT = DMAX / 32;  // head-dim columns per lane
   float acc[kRowsPerWarp][DT];
   float m[kRowsPerWarp], l[kRowsPerWarp];
-  int vend[kRowsPerWarp];
+  int vbeg[kRowsPerWarp], vend[kRowsPerWarp];
 #pragma unroll
   for (int r = 0; r < kRowsPerWarp; ++r) {
     m[r] = -INFINITY;
     l[r] = 0.f;
     const int i = row0 + warp * kRowsPerWarp + r;
-    vend[r] = i < sq ? visible_end(a.mask_mode, i, sq, sk) : 0;
+    vend[r] = i < sq ? visible_end(a.mask_mode, i, sq, sk, a.next) : 0;
+    vbeg[r] = visible_begin(a.mask_mode, i, a.pre);
 #pragma unroll
     for (int t = 0; t < DT; ++t) acc[r][t] = 0.f;
   }
 
-  for (int j0 = 0; j0 < kv_end; j0 += kBN) {
+  for (int j0 = kv_begin; j0 < kv_end; j0 += kBN) {
     __syncthreads();  // previous tile fully consumed (and Q staged on the first pass)
     for (int x = threadIdx.x; x < kBN * D; x += blockDim.x) {
       const int r = x / D, d = x - r * D;
       const bool in = j0 + r < sk;
       sK[r * ldk + d] = in ? K[kvoff(j0 + r) + d] : 0.f;
-      sV[x] = in ? V[kvoff(j0 + r) + d] : 0.f;
+    }
+    for (int x = threadIdx.x; x < kBN * Dv; x += blockDim.x) {
+      const int r = x / Dv, d = x - r * Dv;
+      sV[x] = j0 + r < sk ? V[voff(j0 + r) + d] : 0.f;
     }
     __syncthreads();
 
@@ -142,7 +157,9 @@ __global__ void __launch_bounds__(kWarps * 32) fwd_f32_kernel(FwdArgs a, int til
     float* pw = sP + warp * kRowsPerWarp * kBN;
 #pragma unroll
     for (int r = 0; r < kRowsPerWarp; ++r) {
-      const bool vis = j < vend[r];
+      const int i = row0 + warp * kRowsPerWarp + r;
+      bool vis = j >= vbeg[r] && j < vend[r];
+      if (vis && mrow0 != nullptr) vis = mrow0[(int64_t)i * a.mask_rs + j] == 0;
       const float sc = vis ? s[r] * a.scale : -INFINITY;
       float mx = sc;
 #pragma unroll
@@ -165,10 +182,10 @@ __global__ void __launch_bounds__(kWarps * 32) fwd_f32_kernel(FwdArgs a, int til
     __syncwarp();
     // P.V: lane owns head-dim columns lane, lane+32, ...
     for (int jj = 0; jj < kBN; ++jj) {
-      const float* vr = sV + jj * D;
+      const float* vr = sV + jj * Dv;
       float vv[DT];
 #pragma unroll
-      for (int t = 0; t < DT; ++t) vv[t] = (lane + 32 * t) < D ? vr[lane + 32 * t] : 0.f;
+      for (int t = 0; t < DT; ++t) vv[t] = (lane + 32 * t) < Dv ? vr[lane + 32 * t] : 0.f;
 #pragma unroll
       for (int r = 0; r < kRowsPerWarp; ++r) {
         const float p = pw[r * kBN + jj];
@@ -192,7 +209,7 @@ __global__ void __launch_bounds__(kWarps * 32) fwd_f32_kernel(FwdArgs a, int til
     float f_prev = 0.f;
     int64_t o;
     if (a.acc_mode == 0) {
-      o = qoff(i);
+      o = ooff(i);
       if (lane == 0 && a.smax != nullptr) {
         const int64_t so = a.layout == ATTN_BHSD ? ((int64_t)b * a.Nq + h) * a.Sq + i
                                                  : (int64_t)(q0 + i) * a.Nq + h;
@@ -236,7 +253,7 @@ __global__ void __launch_bounds__(kWarps * 32) fwd_f32_kernel(FwdArgs a, int til
 #pragma unroll
     for (int t = 0; t < DT; ++t) {
       const int d = lane + 32 * t;
-      if (d < D) {
+      if (d < Dv) {
         float v = acc[r][t] * f_o;
         if (a.acc_mode == 2) v = fmaf(O[o + d], f_prev, v);
         O[o + d] = v;
@@ -247,7 +264,7 @@ __global__ void __launch_bounds__(kWarps * 32) fwd_f32_kernel(FwdArgs a, int til
 
 template <int DMAX>
 cudaError_t launch_dmax(const FwdArgs& a, cudaStream_t st) {
-  const size_t smem = sizeof(float) * (size_t)(kBM * a.D + kBN * (a.D + 1) + kBN * a.D +
+  const size_t smem = sizeof(float) * (size_t)(kBM * a.D + kBN * (a.D + 1) + kBN * a.Dv +
                                               kWarps * kRowsPerWarp * kBN);
   cudaError_t e = cudaFuncSetAttribute(fwd_f32_kernel<DMAX>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

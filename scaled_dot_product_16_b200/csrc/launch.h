@@ -13,8 +13,13 @@ struct FwdArgs {
   const int32_t* cu_q;   // TND only
   const int32_t* cu_kv;  // TND only
   int B, Sq, Skv, Nq, Nkv, D;
+  int Dv;  // value / output head size (== D except through attn_fwd_masked)
   float scale;
   int mask_mode, layout, dtype;
+  int pre, next;               // band limits (mask_mode ATTN_MASK_BAND), clamped to +-2^30
+  const uint8_t* mask;         // explicit mask, 1 = excluded (null: none)
+  int64_t mask_bs, mask_rs;    // its batch and row strides in bytes
+  bool mask_vec;               // mask, mask_bs and mask_rs all 16-byte aligned
   int acc_mode;  // 0: plain output; 1: overwrite an accumulator; 2: merge into it
   void* out;     // output, or the accumulator's output (merge layouts) when acc_mode != 0
   float* smax;   // statistics (may be null with ssum when acc_mode == 0), or the accumulator's

@@ -97,6 +97,32 @@ def test_host_validation_without_gpu(lib):
     assert _fwd(lib, layout=1, B=0) == OK
 
 
+def _masked(lib, **kw):
+    a = dict(q=16, k=16, v=16, cq=None, ck=None, B=1, Sq=8, Skv=8, Nq=2, Nkv=1, Dqk=64, Dv=64,
+             scale=0.125, mask=3, pre=4, nxt=0, am=None, bs=0, rs=0, dtype=1, layout=0, out=16,
+             m=None, l=None, stream=None)
+    a.update(kw)
+    return lib.attn_fwd_masked(a["q"], a["k"], a["v"], a["cq"], a["ck"], a["B"], a["Sq"], a["Skv"],
+                               a["Nq"], a["Nkv"], a["Dqk"], a["Dv"], a["scale"], a["mask"], a["pre"],
+                               a["nxt"], a["am"], a["bs"], a["rs"], a["dtype"], a["layout"],
+                               a["out"], a["m"], a["l"], a["stream"])
+
+
+def test_masked_validation_without_gpu(lib):
+    INVALID, UNSUP, OK = sdpa.ATTN_ERR_INVALID, sdpa.ATTN_ERR_UNSUPPORTED, sdpa.ATTN_OK
+    assert _fwd(lib, mask=3) == INVALID                 # the band needs attn_fwd_masked
+    assert _masked(lib, mask=4) == INVALID
+    assert _masked(lib, pre=-5, nxt=4) == INVALID       # empty band
+    assert _masked(lib, pre=-(1 << 62), nxt=-(1 << 62)) == INVALID
+    assert _masked(lib, Dv=65) == INVALID               # Dv <= Dqk
+    assert _masked(lib, Dv=0) == INVALID
+    assert _masked(lib, am=16, rs=7) == INVALID         # BHSD rows shorter than Skv
+    assert _masked(lib, am=16, rs=8, bs=-1) == INVALID
+    assert _masked(lib, dtype=0, Dv=32) == UNSUP        # tensor-core path: Dv == Dqk
+    assert _masked(lib, B=0) == OK                      # empty problem, no launch
+    assert _masked(lib, layout=1, B=0, Sq=0, Skv=0) == OK
+
+
 def test_merge_and_csr_validation_without_gpu(lib):
     P = 16
     args = [P] * 6
