@@ -116,7 +116,7 @@ int fwd_impl(const void* q, const void* k, const void* v, const int32_t* cu_seql
   if (dtype == ATTN_F32 && D > 256) return ATTN_ERR_UNSUPPORTED;
   if (dtype == ATTN_BF16 || dtype == ATTN_F16) {
     if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
-    if (Dv != D) return ATTN_ERR_UNSUPPORTED;
+    if (Dv != D && !(D == 128 && Dv == 64)) return ATTN_ERR_UNSUPPORTED;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return ATTN_ERR_INVALID;
   }
 

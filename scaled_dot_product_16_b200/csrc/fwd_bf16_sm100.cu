@@ -87,10 +87,13 @@ __device__ __forceinline__ void exp2_poly2(float x0, float x1, float& p0, float&
   p1 = __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23));
 }
 
-template <int HD, bool F16>
+// HD: head size of Q and K; HDV: head size of V and the output (HDV <= HD).
+template <int HD, int HDV, bool F16>
 struct Cfg {
   static constexpr int kBoxes = HD / 64;                 // 64-element (128-byte) TMA boxes
-  static constexpr int kTileBytes = kBM * HD * 2;        // one Q, K or V tile
+  static constexpr int kBoxesV = HDV / 64;
+  static constexpr int kTileBytes = kBM * HD * 2;        // one Q or K tile; a K/V ring slot
+  static constexpr int kTileBytesV = kBN * HDV * 2;      // one V tile
   static constexpr int kStages = HD == 128 ? SDPA_STAGES_D128 : 6;  // K/V ring depth
   static constexpr int kQOff = 0;
   static constexpr int kKVOff = 2 * kTileBytes;
@@ -100,7 +103,8 @@ struct Cfg {
   static_assert(kSmemBytes <= 232448, "227 KB of shared memory per block");
   static constexpr uint32_t kFmt = F16 ? 0u : 1u;  // instruction-descriptor operand format
   static constexpr uint32_t kIdescQK = idesc_f16_f32(kBM, kBN, 0, 0, kFmt);
-  static constexpr uint32_t kIdescPV = idesc_f16_f32(kBM, HD, 0, 1, kFmt);
+  static constexpr uint32_t kIdescPV = idesc_f16_f32(kBM, HDV, 0, 1, kFmt);
+  static_assert(HDV <= HD && HDV % 64 == 0, "value head size");
 };
 
 struct Barriers {
@@ -187,12 +191,14 @@ struct Work {
   int row0;         // first row (within the sequence) of this block's 256 rows
 };
 
-template <int HD, bool F16, bool MASKED>
+// EXT: the masked-call features (band lower edge, explicit mask). Plain calls use the EXT = false
+// instantiation, whose softmax loop carries none of their code.
+template <int HD, int HDV, bool F16, bool EXT>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, FwdArgs a, int units_per_seq,
                     float scale_log2) {
-  using C = Cfg<HD, F16>;
+  using C = Cfg<HD, HDV, F16>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   Barriers* bars = reinterpret_cast<Barriers*>(smem + C::kBarOff);
@@ -258,7 +264,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const bool has1 = rows1 > 0;
   // Key tiles run from jlo (the band's first tile for the block's first row; 0 otherwise) to
   // the tile holding each Q tile's last visible key; n0 and n1 count tiles from jlo.
-  const int jlo = visible_begin(a.mask_mode, w.row0, a.pre) / kBN;
+  const int jlo = EXT ? visible_begin(a.mask_mode, w.row0, a.pre) / kBN : 0;
   const int kv_end0 = visible_end(a.mask_mode, w.row0 + rows0 - 1, w.sq, w.sk, a.next);
   const int kv_end1 = has1 ? visible_end(a.mask_mode, w.row0 + kBM + rows1 - 1, w.sq, w.sk, a.next) : 0;
   const int n0 = max((kv_end0 + kBN - 1) / kBN, jlo) - jlo;
@@ -303,8 +309,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool bhsd = a.layout == ATTN_BHSD;
       const int qhead = bhsd ? w.b * a.Nq + w.h : w.h;
       const int khead = bhsd ? w.b * a.Nkv + w.g : w.g;
-      auto load_tile = [&](const CUtensorMap* map, uint32_t dst, uint32_t bar, int tok, int head) {
-        for (int x = 0; x < C::kBoxes; ++x) {
+      auto load_tile = [&](const CUtensorMap* map, uint32_t dst, uint32_t bar, int tok, int head,
+                           int boxes) {
+        for (int x = 0; x < boxes; ++x) {
           if (bhsd)
             tma_load_3d(dst + x * (kBM * 128), map, bar, x * 64, tok, head);
           else
@@ -316,17 +323,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_prefetch_desc(&tm_v);
       const uint32_t qbar = bar_addr(&bars->q_full);
       mbar_arrive_expect_tx(qbar, (has1 ? 2 : 1) * C::kTileBytes);
-      load_tile(&tm_q, sQ, qbar, w.q0 + w.row0, qhead);
-      if (has1) load_tile(&tm_q, sQ + C::kTileBytes, qbar, w.q0 + w.row0 + kBM, qhead);
+      load_tile(&tm_q, sQ, qbar, w.q0 + w.row0, qhead, C::kBoxes);
+      if (has1) load_tile(&tm_q, sQ + C::kTileBytes, qbar, w.q0 + w.row0 + kBM, qhead, C::kBoxes);
       // K0, V0, K1, V1, ... through the ring
       int issued = 0;
       for (int i = 0; i < 2 * n1; ++i, ++issued) {
         const int s = i % C::kStages, r = i / C::kStages;
         if (r > 0 && !wait_bar(bar_addr(&bars->kv_empty[s]), (r - 1) & 1, abort, a.status)) break;
         const uint32_t fb = bar_addr(&bars->kv_full[s]);
-        mbar_arrive_expect_tx(fb, C::kTileBytes);
+        mbar_arrive_expect_tx(fb, (i & 1) ? C::kTileBytesV : C::kTileBytes);
         const int j = i >> 1;
-        load_tile((i & 1) ? &tm_v : &tm_k, sKV + s * C::kTileBytes, fb, w.k0 + (jlo + j) * kBN, khead);
+        load_tile((i & 1) ? &tm_v : &tm_k, sKV + s * C::kTileBytes, fb, w.k0 + (jlo + j) * kBN, khead,
+                  (i & 1) ? C::kBoxesV : C::kBoxes);
       }
       // drain: every stage this thread filled must have landed before the block exits
       for (int i = max(0, issued - C::kStages); i < issued; ++i) {
@@ -338,7 +346,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == kMmaWarp) {
     // =============================== MMA issue ==========================================
     if (lane == 0) {
-      const uint32_t S0 = tmem, S1 = tmem + 128, O0 = tmem + 256, O1 = tmem + 256 + HD;
+      const uint32_t S0 = tmem, S1 = tmem + 128, O0 = tmem + 256, O1 = tmem + 256 + HDV;
       // Descriptors are built once. K-step kk of an operand adds a constant to the start
       // address field (shared-memory addresses stay below 256 KB, so the 14-bit field never
       // carries), which keeps the issue loop at a few instructions per MMA.
@@ -428,13 +436,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int i = w.row0 + q * kBM + r;            // row within the sequence
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     const uint32_t S = tmem + lane_off + q * 128;
-    const uint32_t O = tmem + lane_off + 256 + q * HD;
+    const uint32_t O = tmem + lane_off + 256 + q * HDV;
     const int lim = i < w.sq ? visible_end(a.mask_mode, i, w.sq, w.sk, a.next) : w.sk;
-    const int lo = i < w.sq ? visible_begin(a.mask_mode, i, a.pre) : 0;
+    const int lo = EXT && i < w.sq ? visible_begin(a.mask_mode, i, a.pre) : 0;
     // explicit mask row of this query (rows past the sequence read none)
     const uint8_t* mrow = nullptr;
-    if constexpr (MASKED)
-      if (i < w.sq) mrow = a.mask + (int64_t)w.b * a.mask_bs + (int64_t)i * a.mask_rs;
+    if constexpr (EXT)
+      if (i < w.sq && a.mask != nullptr) mrow = a.mask + (int64_t)w.b * a.mask_bs + (int64_t)i * a.mask_rs;
 
     float m = -INFINITY;        // running max used for P (log2 units, lazily updated)
     float mraw = -INFINITY;     // true max of the raw scores q.k
@@ -446,11 +454,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
         tc_fence_after();
         const int kbase = (jlo + j) * kBN;
-        uint4 mk[MASKED ? 8 : 1];
-        if constexpr (MASKED) {
+        uint4 mk[EXT ? 8 : 1];
+        if constexpr (EXT) {
           // the mask bytes of this row's 128 keys (16 at a time when aligned and whole);
           // issued before the TMEM loads so the two latencies overlap
-          if (mrow != nullptr && a.mask_vec && kbase + kBN <= w.sk) {
+          if (mrow == nullptr) {
+            // band only, or a row past the sequence: nothing to read
+          } else if (a.mask_vec && kbase + kBN <= w.sk) {
             const uint4* src = reinterpret_cast<const uint4*>(mrow + kbase);
 #pragma unroll
             for (int x = 0; x < 8; ++x) mk[x] = __ldg(src + x);
@@ -464,7 +474,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int z = 0; z < 4; ++z) {
                   const int c = x * 16 + y * 4 + z;
-                  const uint32_t byte = (mrow != nullptr && kbase + c < w.sk) ? mrow[kbase + c] : 0u;
+                  const uint32_t byte = kbase + c < w.sk ? mrow[kbase + c] : 0u;
                   word |= (byte != 0u ? 1u : 0u) << (8 * z);
                 }
                 wd[y] = word;
@@ -477,18 +487,26 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int c = 0; c < 4; ++c) tmem_ld32f(S + c * 32, s[c]);
         tmem_wait_ld();
-        if (kbase + kBN > lim || kbase < lo) {
+        if constexpr (!EXT) {
+          if (kbase + kBN > lim) {
 #pragma unroll
-          for (int c = 0; c < kBN; ++c)
-            if (kbase + c >= lim || kbase + c < lo) s[c >> 5][c & 31] = -INFINITY;
-        }
-        if constexpr (MASKED) {
+            for (int c = 0; c < kBN; ++c)
+              if (kbase + c >= lim) s[c >> 5][c & 31] = -INFINITY;
+          }
+        } else {
+          if (kbase + kBN > lim || kbase < lo) {
+#pragma unroll
+            for (int c = 0; c < kBN; ++c)
+              if (kbase + c >= lim || kbase + c < lo) s[c >> 5][c & 31] = -INFINITY;
+          }
+          if (mrow != nullptr) {
 #pragma unroll
           for (int c = 0; c < kBN; ++c) {
             const uint4 v4 = mk[c >> 4];
             const uint32_t wd = ((c >> 2) & 3) == 0 ? v4.x : ((c >> 2) & 3) == 1 ? v4.y
                               : ((c >> 2) & 3) == 2 ? v4.z : v4.w;
             if ((wd >> (8 * (c & 3))) & 0xffu) s[c >> 5][c & 31] = -INFINITY;
+          }
           }
         }
         // row max: a tree of 3-input maxima over the 128 scores
@@ -536,7 +554,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (__any_sync(0xffffffffu, bump && j > 0)) {
           const float f = (bump && j > 0) ? corr : 1.f;
 #pragma unroll
-          for (int c = 0; c < HD / 32; ++c) {
+          for (int c = 0; c < HDV / 32; ++c) {
             uint32_t o[32];
             tmem_ld32(O + c * 32, o);
             tmem_wait_ld();
@@ -571,7 +589,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       float f_prev = 0.f;               // factor on the accumulator's previous output row
       int64_t orow, so;
       if (a.acc_mode == kAccNone) {
-        orow = bhsd ? (((int64_t)w.b * a.Nq + w.h) * a.Sq + i) * HD : ((int64_t)(w.q0 + i) * a.Nq + w.h) * HD;
+        orow = bhsd ? (((int64_t)w.b * a.Nq + w.h) * a.Sq + i) * HDV : ((int64_t)(w.q0 + i) * a.Nq + w.h) * HDV;
         so = bhsd ? ((int64_t)w.b * a.Nq + w.h) * a.Sq + i : (int64_t)(w.q0 + i) * a.Nq + w.h;
         if (store && a.smax != nullptr) {
           a.smax[so] = m_loc;
@@ -580,12 +598,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       } else {
         // accumulator in the merge layouts: BHSD -> output [Sq, B, Nq*D] (SBH), statistics
         // [B, Nq, Sq, 8]; TND -> output [T, Nq*D], statistics [T, Nq, 8]
-        orow = bhsd ? (((int64_t)i * a.B + w.b) * a.Nq + w.h) * HD : ((int64_t)(w.q0 + i) * a.Nq + w.h) * HD;
+        orow = bhsd ? (((int64_t)i * a.B + w.b) * a.Nq + w.h) * HDV : ((int64_t)(w.q0 + i) * a.Nq + w.h) * HDV;
         so = (bhsd ? ((int64_t)w.b * a.Nq + w.h) * a.Sq + i : (int64_t)(w.q0 + i) * a.Nq + w.h) * 8;
         if (store) merge_into_stats(a, so, m_loc, l_loc, &f_prev, &f_o);
       }
 #pragma unroll
-      for (int c = 0; c < HD / 32; ++c) {
+      for (int c = 0; c < HDV / 32; ++c) {
         uint32_t o[32];
         if (have_o && ok) {
           tmem_ld32(O + c * 32, o);
@@ -674,26 +692,27 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t D, uint64_t dim1, uint6
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int HD, bool F16>
+template <int HD, int HDV, bool F16>
 cudaError_t launch_hd(const FwdArgs& a, cudaStream_t st) {
-  using C = Cfg<HD, F16>;
+  using C = Cfg<HD, HDV, F16>;
   CUtensorMap tq, tk, tv;
-  const uint64_t D = HD;
+  const uint64_t D = HD, Dv = HDV;
   bool ok;
   if (a.layout == ATTN_BHSD) {
     // (d, s, b*h): rows of a head are contiguous
     ok = make_map(&tq, a.q, D, a.Sq, (uint64_t)a.B * a.Nq, D * 2, (uint64_t)a.Sq * D * 2, kBM, 1, F16) &&
          make_map(&tk, a.k, D, a.Skv, (uint64_t)a.B * a.Nkv, D * 2, (uint64_t)a.Skv * D * 2, kBN, 1, F16) &&
-         make_map(&tv, a.v, D, a.Skv, (uint64_t)a.B * a.Nkv, D * 2, (uint64_t)a.Skv * D * 2, kBN, 1, F16);
+         make_map(&tv, a.v, Dv, a.Skv, (uint64_t)a.B * a.Nkv, Dv * 2, (uint64_t)a.Skv * Dv * 2, kBN, 1, F16);
   } else {
     // (d, head, token): a tile is 128 tokens of one head
     const uint64_t tq_rows = a.Sq > 0 ? a.Sq : 1, tk_rows = a.Skv > 0 ? a.Skv : 1;
     ok = make_map(&tq, a.q, D, a.Nq, tq_rows, D * 2, (uint64_t)a.Nq * D * 2, 1, kBM, F16) &&
          make_map(&tk, a.k, D, a.Nkv, tk_rows, D * 2, (uint64_t)a.Nkv * D * 2, 1, kBN, F16) &&
-         make_map(&tv, a.v, D, a.Nkv, tk_rows, D * 2, (uint64_t)a.Nkv * D * 2, 1, kBN, F16);
+         make_map(&tv, a.v, Dv, a.Nkv, tk_rows, Dv * 2, (uint64_t)a.Nkv * Dv * 2, 1, kBN, F16);
   }
   if (!ok) return cudaErrorInvalidValue;
-  auto kernel = a.mask != nullptr ? fwd_bf16_kernel<HD, F16, true> : fwd_bf16_kernel<HD, F16, false>;
+  const bool ext = a.mask != nullptr || a.mask_mode == ATTN_MASK_BAND;
+  auto kernel = ext ? fwd_bf16_kernel<HD, HDV, F16, true> : fwd_bf16_kernel<HD, HDV, F16, false>;
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return e;
   int units_per_seq = 0;
@@ -716,8 +735,9 @@ cudaError_t launch_hd(const FwdArgs& a, cudaStream_t st) {
 
 cudaError_t launch_fwd_bf16(const FwdArgs& a, cudaStream_t st) {
   const bool f16 = a.dtype == ATTN_F16;
-  if (a.D == 128) return f16 ? launch_hd<128, true>(a, st) : launch_hd<128, false>(a, st);
-  return f16 ? launch_hd<64, true>(a, st) : launch_hd<64, false>(a, st);
+  if (a.D == 128 && a.Dv == 64) return f16 ? launch_hd<128, 64, true>(a, st) : launch_hd<128, 64, false>(a, st);
+  if (a.D == 128) return f16 ? launch_hd<128, 128, true>(a, st) : launch_hd<128, 128, false>(a, st);
+  return f16 ? launch_hd<64, 64, true>(a, st) : launch_hd<64, 64, false>(a, st);
 }
 
 }  // namespace sdpa

@@ -166,8 +166,30 @@ def test_band_full_size_sampled():
     assert torch.isfinite(out.float()).all()
 
 
+@pytest.mark.parametrize("dtype", [BF, F16], ids=["bf16", "f16"])
+@pytest.mark.parametrize("mode", [W.MASK_NONE, W.MASK_CAUSAL_TOPLEFT, BAND])
+def test_value_head_size_tensor_cores(dtype, mode):
+    """Dqk = 128, Dv = 64 on the tcgen05 path (qD == kD >= vD)."""
+    base = W.dense_bhsd(2, 4, 300, 128, causal=False, dtype=dtype, seed=2, cfg=41, Hkv=2, Skv=333)
+    inp = W.AttnInputs(base.q, base.k, base.v[..., :64].contiguous(), W.BHSD, mode, W.dtype_code(dtype),
+                       2, 300, 333, 4, 2, 128, base.scale)
+    _check(inp, mode=mode, pre=90, nxt=40, Dv=64)
+
+
+def test_value_head_size_tensor_cores_varlen_masked():
+    rng = np.random.default_rng(10)
+    base = W.varlen_tnd([0, 700, 1, 257], 8, 2, 128, causal=False, dtype=BF, seed=6, cfg=42)
+    inp = W.AttnInputs(base.q, base.k, base.v[..., :64].contiguous(), W.TND, W.MASK_CAUSAL_TOPLEFT,
+                       W.BF16, base.B, base.Sq, base.Skv, 8, 2, 128, base.scale, cu_q=base.cu_q,
+                       cu_kv=base.cu_kv)
+    rs, bs = 704, 704 * 704
+    mask = _random_mask(rng, 4, 704, 704, rs, bs, p=0.2)
+    _check(inp, mode=W.MASK_CAUSAL_TOPLEFT, mask=mask, bs=bs, rs=rs, Dv=64)
+
+
 def test_tensor_core_path_rejects_other_value_sizes():
     inp = W.dense_bhsd(1, 2, 64, 128, causal=False, dtype=BF, seed=1, cfg=40)
-    with pytest.raises(sdpa.AttnError) as e:
-        _run(inp, mode=W.MASK_NONE, Dv=64)
-    assert e.value.status == sdpa.ATTN_ERR_UNSUPPORTED
+    for Dv in (32, 96):
+        with pytest.raises(sdpa.AttnError) as e:
+            _run(inp, mode=W.MASK_NONE, Dv=Dv)
+        assert e.value.status == sdpa.ATTN_ERR_UNSUPPORTED
