@@ -8,6 +8,7 @@
  *   attn_merge       merge of two partial attention results from their max/sum statistics.
  *   attn_fwd_accumulate  attn_fwd over one chunk of keys folded into a running merge result.
  *   attn_fwd_masked  attn_fwd with band limits, an explicit mask and a value head size Dv.
+ *   attn_sparse_csr_tc  attn_sparse_csr in bf16 / fp16 on the tensor cores.
  *
  * Conventions shared by every call
  *   - All tensor pointers are DEVICE pointers owned by the caller. The library allocates no
@@ -189,6 +190,28 @@ ATTN_API int attn_sparse_csr(const float* q, const float* k, const float* v,
                     const int32_t* csr_offset, const int32_t* csr_columns,
                     int B, int H, int S, int D, int64_t nnz_cap,
                     float* out, void* stream);
+
+/*
+ * attn_sparse_csr_tc -- CSR-sparse attention forward in bf16 or fp16 on the tensor cores.
+ *
+ * Defined by: the attn_sparse_csr definition above ("paddle.nn.functional.sparse_attention",
+ * formula and 参数), with 16-bit inputs and output and fp32 accumulation. Each block of 128
+ * query rows gathers the union of its rows' columns into tiles of 128 keys and multiplies
+ * those on the tensor cores; each row's softmax keeps exactly its own stored entries.
+ *
+ *   q, k, v, out   dtype (ATTN_BF16 or ATTN_F16) [B, H, S, D], 16-byte aligned; D = 64 or 128
+ *   csr_offset     int32 [B, H, S+1], as for attn_sparse_csr
+ *   csr_columns    int32 [B, H, nnz_cap]: column of each stored entry, 0 <= j < S, order free;
+ *                  the columns of one row must be distinct
+ * Scale 1/sqrt(D). An empty row gives zeros. S <= 32768 (larger is ATTN_ERR_UNSUPPORTED).
+ * Data errors: a column outside [0, S), a row pointer that starts above 0, decreases or passes
+ * nnz_cap, or a column stored twice in one row, set ATTN_ERR_DATA; those rows are written as
+ * zeros. Other dtypes are ATTN_ERR_INVALID.
+ */
+ATTN_API int attn_sparse_csr_tc(const void* q, const void* k, const void* v,
+                                const int32_t* csr_offset, const int32_t* csr_columns,
+                                int B, int H, int S, int D, int64_t nnz_cap, int dtype,
+                                void* out, void* stream);
 
 /*
  * attn_merge -- merge two partial attention results (the ring-attention update).

@@ -19,7 +19,7 @@ __all__ = [
     "attn_fwd", "attn_fwd_accumulate", "attn_sparse_csr", "attn_merge", "attn_get_last_error", "AttnError",
     "ATTN_BF16", "ATTN_F32", "ATTN_F16", "ATTN_BHSD", "ATTN_TND", "ATTN_MASK_NONE",
     "ATTN_MASK_CAUSAL_TOPLEFT", "ATTN_MASK_CAUSAL_BOTTOMRIGHT", "ATTN_MASK_BAND", "lib_path",
-    "load_library", "attn_fwd_masked",
+    "load_library", "attn_fwd_masked", "attn_sparse_csr_tc",
 ]
 
 ATTN_OK, ATTN_ERR_INVALID, ATTN_ERR_UNSUPPORTED, ATTN_ERR_CUDA, ATTN_ERR_DATA, ATTN_ERR_TIMEOUT = range(6)
@@ -62,6 +62,8 @@ def load_library():
                                         I64, I, I, P, P, P, P]
         lib.attn_fwd_masked.restype = I
         lib.attn_sparse_csr.argtypes = [P, P, P, P, P, I, I, I, I, I64, P, P]
+        lib.attn_sparse_csr_tc.argtypes = [P, P, P, P, P, I, I, I, I, I64, I, P, P]
+        lib.attn_sparse_csr_tc.restype = I
         lib.attn_sparse_csr.restype = I
         lib.attn_merge.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, P, P, P, P, P]
         lib.attn_merge.restype = I
@@ -152,6 +154,16 @@ def attn_sparse_csr(q, k, v, csr_offset, csr_columns, *, B: int, H: int, S: int,
     _check(lib.attn_sparse_csr(_ptr(q), _ptr(k), _ptr(v), _ptr(csr_offset), _ptr(csr_columns),
                                int(B), int(H), int(S), int(D), int(nnz_cap), _ptr(out),
                                _stream(stream)), "attn_sparse_csr")
+
+
+def attn_sparse_csr_tc(q, k, v, csr_offset, csr_columns, *, B: int, H: int, S: int, D: int,
+                       nnz_cap: int, dtype: int, out, stream=None) -> None:
+    """CSR-sparse attention forward in bf16/fp16 on the tensor cores (see
+    ``attn_sparse_csr_tc`` in include/attn.h)."""
+    lib = load_library()
+    _check(lib.attn_sparse_csr_tc(_ptr(q), _ptr(k), _ptr(v), _ptr(csr_offset), _ptr(csr_columns),
+                                  int(B), int(H), int(S), int(D), int(nnz_cap), int(dtype),
+                                  _ptr(out), _stream(stream)), "attn_sparse_csr_tc")
 
 
 def attn_merge(prev_out, prev_max, prev_sum, cur_out, cur_max, cur_sum, *, S: int, B: int, N: int,

@@ -223,6 +223,40 @@ int attn_sparse_csr(const float* q, const float* k, const float* v, const int32_
   return e == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
+int attn_sparse_csr_tc(const void* q, const void* k, const void* v, const int32_t* csr_offset,
+                       const int32_t* csr_columns, int B, int H, int S, int D, int64_t nnz_cap,
+                       int dtype, void* out, void* stream) {
+  if (dtype != ATTN_BF16 && dtype != ATTN_F16) return ATTN_ERR_INVALID;
+  if (B < 0 || H < 0 || S < 0 || nnz_cap < 0) return ATTN_ERR_INVALID;
+  if (D < 1) return ATTN_ERR_INVALID;
+  if ((int64_t)B * H * S == 0) return ATTN_OK;
+  if (q == nullptr || k == nullptr || v == nullptr || out == nullptr || csr_offset == nullptr)
+    return ATTN_ERR_INVALID;
+  if (nnz_cap > 0 && csr_columns == nullptr) return ATTN_ERR_INVALID;
+  if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
+  if (S > 32768) return ATTN_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return ATTN_ERR_INVALID;
+  sdpa::CsrTcArgs a{};
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.offset = csr_offset;
+  a.columns = csr_columns;
+  a.B = B;
+  a.H = H;
+  a.S = S;
+  a.D = D;
+  a.dtype = dtype;
+  a.nnz_cap = nnz_cap;
+  a.cols_vec = csr_columns != nullptr && aligned16(csr_columns) && nnz_cap % 4 == 0;
+  a.out = out;
+  int sms = 0;
+  int rc = device_state(&a.status, &sms);
+  if (rc != ATTN_OK) return rc;
+  const cudaError_t e = sdpa::launch_sparse_csr_tc(a, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
 int attn_merge(const void* prev_out, const float* prev_max, const float* prev_sum,
                const void* cur_out, const float* cur_max, const float* cur_sum, int S, int B,
                int N, int D, int dtype, int layout, const int64_t* actual_seq_qlen, void* out,

@@ -40,6 +40,19 @@ struct CsrArgs {
   int* status;
 };
 
+struct CsrTcArgs {  // attn_sparse_csr_tc: 16-bit q, k, v, out [B, H, S, D]
+  const void* q;
+  const void* k;
+  const void* v;
+  const int32_t* offset;
+  const int32_t* columns;
+  int B, H, S, D, dtype;
+  int64_t nnz_cap;
+  bool cols_vec;  // columns 16-byte aligned and nnz_cap % 4 == 0: read 4 indices at a time
+  void* out;
+  int* status;
+};
+
 struct MergeArgs {
   const void* prev_out;
   const float* prev_max;
@@ -59,5 +72,6 @@ cudaError_t launch_merge(const MergeArgs& a, cudaStream_t st);
 cudaError_t launch_fwd_f32(const FwdArgs& a, cudaStream_t st);
 cudaError_t launch_fwd_bf16(const FwdArgs& a, cudaStream_t st);
 cudaError_t launch_sparse_csr(const CsrArgs& a, cudaStream_t st);
+cudaError_t launch_sparse_csr_tc(const CsrTcArgs& a, cudaStream_t st);
 
 }  // namespace sdpa

@@ -135,6 +135,12 @@ def test_merge_and_csr_validation_without_gpu(lib):
     assert lib.attn_sparse_csr(P, P, P, P, P, 1, 1, 4, 0, 4, P, None) == sdpa.ATTN_ERR_INVALID
     assert lib.attn_sparse_csr(P, P, P, P, P, 1, 1, 4, 300, 4, P, None) == sdpa.ATTN_ERR_UNSUPPORTED
     assert lib.attn_sparse_csr(P, P, P, P, P, 0, 1, 4, 64, 4, P, None) == sdpa.ATTN_OK
+    tc = lib.attn_sparse_csr_tc
+    assert tc(P, P, P, P, P, 1, 1, 4, 64, 4, sdpa.ATTN_F32, P, None) == sdpa.ATTN_ERR_INVALID
+    assert tc(P, P, P, P, P, 1, 1, 4, 96, 4, sdpa.ATTN_BF16, P, None) == sdpa.ATTN_ERR_UNSUPPORTED
+    assert tc(P, P, P, P, P, 1, 1, 32769, 64, 4, sdpa.ATTN_BF16, P, None) == sdpa.ATTN_ERR_UNSUPPORTED
+    assert tc(18, P, P, P, P, 1, 1, 4, 64, 4, sdpa.ATTN_BF16, P, None) == sdpa.ATTN_ERR_INVALID
+    assert tc(P, P, P, P, P, 0, 1, 4, 64, 4, sdpa.ATTN_F16, P, None) == sdpa.ATTN_OK
 
 
 def test_missing_library_fails_loudly(monkeypatch, tmp_path):

@@ -1,0 +1,129 @@
+"""attn_sparse_csr_tc (bf16 / fp16 on the tensor cores) on the GPU against the float64 oracle.
+
+The oracle takes the same 16-bit input values, widened exactly; the output is compared with
+the bf16/fp16 tolerance of the other parity tests."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import scaled_dot_product_16_b200 as sdpa
+from scaled_dot_product_16_b200 import workloads as W
+from tests import gpu_util as G
+
+pytestmark = pytest.mark.gpu
+
+BF, F16 = torch.bfloat16, torch.float16
+
+
+def _run(q, k, v, off, cols, B, H, S, D):
+    dq, dk, dv = (torch.as_tensor(x).cuda().contiguous() for x in (q, k, v))
+    doff = torch.from_numpy(np.ascontiguousarray(off, np.int32)).cuda()
+    dcol = torch.from_numpy(np.ascontiguousarray(cols, np.int32)).cuda()
+    out = torch.full_like(dq, float("nan"))
+    sdpa.attn_sparse_csr_tc(dq, dk, dv, doff, dcol, B=B, H=H, S=S, D=D, nnz_cap=cols.shape[-1],
+                            dtype=W.dtype_code(dq.dtype), out=out)
+    return out.cpu(), sdpa.attn_get_last_error()
+
+
+def _inputs(B, H, S, D, dtype, seed):
+    return [W.randn((B, H, S, D), 300 + 7 * seed + i).to(dtype) for i in range(3)]
+
+
+def _distinct_pattern(rng, B, H, S, max_per_row, empty_every=0):
+    """Random rows of distinct, unsorted columns; every empty_every-th row empty."""
+    offs = np.zeros((B * H, S + 1), np.int32)
+    rows = []
+    for bh in range(B * H):
+        cnt = rng.integers(0, max_per_row + 1, size=S)
+        if empty_every:
+            cnt[::empty_every] = 0
+        offs[bh, 1:] = np.cumsum(cnt)
+        rows.append(np.concatenate([rng.permutation(S)[:c] for c in cnt]) if cnt.sum() else np.zeros(0, int))
+    cap = max(1, max(len(r) for r in rows))
+    cols = np.zeros((B * H, cap), np.int32)
+    for bh, r in enumerate(rows):
+        cols[bh, :len(r)] = r
+    return offs.reshape(B, H, S + 1), cols.reshape(B, H, cap)
+
+
+def _check(q, k, v, off, cols, B, H, S, D):
+    out, st = _run(q, k, v, off, cols, B, H, S, D)
+    assert st == 0
+    ref = oracle.sparse_csr(q, k, v, off, cols, B=B, H=H, S=S, D=D)
+    G.check_out(G.f64(out), ref, W.dtype_code(q.dtype), "csr_tc out")
+
+
+@pytest.mark.parametrize("dtype", [BF, F16], ids=["bf16", "f16"])
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("S", [300, 640])
+def test_window_stride_pattern(dtype, D, S):
+    offs, c = W.window_stride_pattern(S)
+    B, H = 1, 2
+    off = np.broadcast_to(offs, (B, H, S + 1)).copy()
+    cols = np.broadcast_to(c, (B, H, c.shape[0])).copy()
+    _check(*_inputs(B, H, S, D, dtype, S + D), off, cols, B, H, S, D)
+
+
+@pytest.mark.parametrize("dtype", [BF, F16], ids=["bf16", "f16"])
+@pytest.mark.parametrize("D", [64, 128])
+def test_random_patterns(dtype, D):
+    rng = np.random.default_rng(D)
+    B, H, S = 2, 3, 333
+    off, cols = _distinct_pattern(rng, B, H, S, 60, empty_every=7)
+    _check(*_inputs(B, H, S, D, dtype, D), off, cols, B, H, S, D)
+
+
+def test_union_wider_than_one_pass():
+    """Rows of 150 random columns over 2,560 keys: each 128-row block's union spans about 2,000
+    columns, so the per-row masks are rebuilt window after window (256 union columns each)."""
+    rng = np.random.default_rng(5)
+    B, H, S, D = 1, 2, 2560, 64
+    off, cols = _distinct_pattern(rng, B, H, S, 150)
+    _check(*_inputs(B, H, S, D, BF, 5), off, cols, B, H, S, D)
+
+
+def test_full_pattern_equals_dense():
+    B, H, S, D = 1, 2, 200, 128
+    q, k, v = _inputs(B, H, S, D, BF, 9)
+    cols = np.broadcast_to(np.tile(np.arange(S, dtype=np.int32), S), (B, H, S * S)).copy()
+    off = np.broadcast_to(np.arange(0, S * S + 1, S, dtype=np.int32), (B, H, S + 1)).copy()
+    _check(q, k, v, off, cols, B, H, S, D)
+
+
+def test_cfg4_full_size_bf16():
+    """Configuration 4's shape and pattern (B=2, H=8, S=4096, D=64, window 256 + every 64th
+    column) with the inputs rounded to bf16; every row against the oracle."""
+    inp = W.cfg4_csr(seed=0)
+    q, k, v = (x.to(BF) for x in (inp.q, inp.k, inp.v))
+    _check(q, k, v, inp.offset, inp.columns, inp.B, inp.H, inp.S, inp.D)
+
+
+def test_data_errors_zero_only_the_bad_rows():
+    B, H, S, D = 1, 1, 300, 64
+    q, k, v = _inputs(B, H, S, D, BF, 11)
+    offs, c = W.window_stride_pattern(S, half_window=8, stride=100)
+    off = offs.reshape(1, 1, -1).copy()
+    cols = c.reshape(1, 1, -1).copy()
+    ref = oracle.sparse_csr(q, k, v, off, cols, B=B, H=H, S=S, D=D)
+    bad = cols.copy()
+    bad[0, 0, off[0, 0, 20]] = S                       # row 20: a column out of range
+    bad[0, 0, off[0, 0, 150] + 1] = bad[0, 0, off[0, 0, 150]]  # row 150: a column stored twice
+    out, st = _run(q, k, v, off, bad, B, H, S, D)
+    assert st == sdpa.ATTN_ERR_DATA
+    assert torch.all(out[0, 0, 20] == 0) and torch.all(out[0, 0, 150] == 0)
+    keep = np.ones(S, bool)
+    keep[[20, 150]] = False
+    G.check_out(G.f64(out)[0, 0, keep], ref[0, 0, keep], W.BF16, "other rows")
+
+
+def test_validation():
+    q = torch.zeros((1, 1, 8, 96), dtype=BF, device="cuda")
+    off = torch.zeros((1, 1, 9), dtype=torch.int32, device="cuda")
+    cols = torch.zeros((1, 1, 1), dtype=torch.int32, device="cuda")
+    with pytest.raises(sdpa.AttnError) as e:
+        sdpa.attn_sparse_csr_tc(q, q, q, off, cols, B=1, H=1, S=8, D=96, nnz_cap=1, dtype=W.BF16, out=q)
+    assert e.value.status == sdpa.ATTN_ERR_UNSUPPORTED
+    with pytest.raises(sdpa.AttnError) as e:
+        sdpa.attn_sparse_csr_tc(q, q, q, off, cols, B=1, H=1, S=8, D=96, nnz_cap=1, dtype=W.F32, out=q)
+    assert e.value.status == sdpa.ATTN_ERR_INVALID
