@@ -45,7 +45,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one attn_fwd launch on the
 # full varlen workload, from a one-pass ncu capture (profiles/attn_fwd_bf16_varlen.md); it is
 # reported only while the kernel source still has the hash it was measured on.
-TRAFFIC = {"kernel_sha": "22e5c2d45f4a957d", "bytes_per_launch": 938_170_000 + 601_440_000}
+TRAFFIC = {"kernel_sha": "eefbe2f34578ff23", "bytes_per_launch": 937_251_840 + 602_236_928}
 
 
 def kernel_sha() -> str:
@@ -206,6 +206,81 @@ class MergeCase:
         a, p = self.acc, self.parts[c]
         sdpa.attn_merge(a[0], a[1], a[2], p[0], p[1], p[2], S=self.S, B=self.B, N=self.N, D=self.D,
                         dtype=W.BF16, out=a[0], out_max=a[1], out_sum=a[2])
+
+
+def _device_ms(fn, iters: int, stream) -> float:
+    """Mean device time of fn() over iters calls (CUDA events on the launching stream)."""
+    for _ in range(2):
+        fn()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(iters):
+        fn()
+    b.record(stream)
+    torch.cuda.synchronize()
+    if sdpa.attn_get_last_error() != 0:
+        raise RuntimeError("device status set while timing a later-row operation")
+    return a.elapsed_time(b) / iters
+
+
+def next_rows(fwd: "FwdCase", csr: "CsrCase", rank: int, stream) -> dict:
+    """The operations built beyond the step's own rows, each timed on its own: the fused
+    ring fold, the band (sliding window) and the tensor-core CSR variant."""
+    res = {}
+    # ring attention, B=4, N=32, S=8192, D=128, keys in 4 chunks of 2048 folded by
+    # attn_fwd_accumulate into one accumulator (SBH output, [B,N,S,8] statistics)
+    inp = W.dense_bhsd(4, 32, 8192, 128, causal=False, dtype=torch.bfloat16, seed=rank, cfg=5)
+    q = inp.q.cuda()
+    kc = [inp.k[:, :, c * 2048:(c + 1) * 2048].contiguous().cuda() for c in range(4)]
+    vc = [inp.v[:, :, c * 2048:(c + 1) * 2048].contiguous().cuda() for c in range(4)]
+    acc = torch.empty((8192, 4, 32 * 128), dtype=torch.bfloat16, device="cuda")
+    am = torch.empty((4, 32, 8192, 8), device="cuda")
+    al = torch.empty_like(am)
+
+    def ring():
+        for c in range(4):
+            sdpa.attn_fwd_accumulate(q, kc[c], vc[c], B=4, Sq=8192, Skv=2048, Nq=32, Nkv=32, D=128,
+                                     scale=inp.scale, mask_mode=W.MASK_NONE, dtype=W.BF16,
+                                     layout=W.BHSD, first=c == 0, acc_out=acc, acc_max=am, acc_sum=al)
+
+    ms = _device_ms(ring, 5, stream)
+    fl = M.attn_fwd_flops(inp)
+    res["attn_fwd_accumulate"] = {"workload": "ring: dense 4x32x8192x128 bf16, 4 key chunks of 2048",
+                                  "ms_per_ring": ms, "tflops": fl / (ms / 1e3) / 1e12, "launches": 4}
+    del q, kc, vc, acc, am, al
+    # sliding window: 1024 keys back, none ahead, on the step's varlen workload
+    i = fwd.inp
+    ob = torch.empty_like(fwd.out)
+    mb, lb = torch.empty_like(fwd.m), torch.empty_like(fwd.l)
+
+    def band():
+        sdpa.attn_fwd_masked(fwd.q, fwd.k, fwd.v, cu_seqlens_q=fwd.cq, cu_seqlens_kv=fwd.ck, B=i.B,
+                             Sq=i.Sq, Skv=i.Skv, Nq=i.Nq, Nkv=i.Nkv, Dqk=i.D, Dv=i.D, scale=i.scale,
+                             mask_mode=sdpa.ATTN_MASK_BAND, pre_tokens=1023, next_tokens=0,
+                             dtype=i.dtype, layout=i.layout, out=ob, softmax_max=mb, softmax_sum=lb)
+
+    ms = _device_ms(band, 20, stream)
+    fl = 4 * i.Nq * i.D * M.band_pairs(i, 1023, 0)
+    res["attn_fwd_masked"] = {"workload": "band pre=1023 next=0 (sliding window) on the varlen GQA "
+                                          "batch of the step (Nq=32 Nkv=8 D=128 bf16)",
+                              "ms": ms, "tflops": fl / (ms / 1e3) / 1e12, "flops_per_call": fl}
+    # CSR on the tensor cores: the fp32 CSR workload's pattern with bf16 inputs
+    c = csr if csr is not None else CsrCase(W.cfg4_csr(seed=rank))
+    qb, kb, vb = (t.to(torch.bfloat16) for t in (c.q, c.k, c.v))
+    outb = torch.empty_like(qb)
+    ci = c.inp
+
+    def csr_tc():
+        sdpa.attn_sparse_csr_tc(qb, kb, vb, c.off, c.col, B=ci.B, H=ci.H, S=ci.S, D=ci.D,
+                                nnz_cap=ci.nnz_cap, dtype=W.BF16, out=outb)
+
+    ms = _device_ms(csr_tc, 20, stream)
+    ms32 = _device_ms(c.run, 20, stream)
+    res["attn_sparse_csr_tc"] = {"workload": "2x8x4096x64 bf16, window 256 + every 64th column",
+                                 "ms": ms, "tflops": c.flops / (ms / 1e3) / 1e12,
+                                 "fp32_kernel_ms": ms32, "speedup_vs_fp32": ms32 / ms}
+    return res
 
 
 # ---------------------------------------------------------------------------------------------
@@ -403,6 +478,8 @@ def run_ours(args, rank: int, world: int, local: int):
                        "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                        "steps": args.e2e_steps, "what": "attn_fwd with pinned-host inputs copied in "
                        "and outputs + statistics copied back, per step"}
+    if not args.no_next_rows:
+        line["next_rows"] = next_rows(fwd, csr, rank, stream)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(fwd.inp, args.cpu_budget)
     if rank == 0:
@@ -419,6 +496,8 @@ def main(argv=None):
     ap.add_argument("--parts", default="fwd,csr,merge", help="operations in a step (fwd always runs)")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-next-rows", action="store_true",
+                    help="skip timing the ring fold, the band and the tensor-core CSR")
     ap.add_argument("--cpu-budget", type=float, default=20.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--ref-rows", type=int, default=2048, help="oracle rows per reference step")
     args = ap.parse_args(argv)

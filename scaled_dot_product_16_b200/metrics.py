@@ -36,6 +36,18 @@ def attn_fwd_flops(inp: W.AttnInputs) -> int:
     return 4 * inp.Nq * inp.D * visible_pairs(inp)
 
 
+def band_pairs(inp: W.AttnInputs, pre: int, nxt: int) -> int:
+    """(query, key) pairs with i - pre <= j <= i + nxt (in-sequence positions), summed over the
+    sequences: the visible pairs of the band mode."""
+    tot = 0
+    for sq, sk in zip(*seq_lengths(inp)):
+        i = np.arange(sq, dtype=np.int64)
+        lo = np.clip(i - pre, 0, sk)
+        hi = np.clip(i + nxt + 1, 0, sk)
+        tot += int(np.maximum(hi - lo, 0).sum())
+    return int(tot)
+
+
 def attn_fwd_min_bytes(inp: W.AttnInputs) -> int:
     """Compulsory HBM traffic: read Q, K, V once, write O and the two statistics."""
     e = 2 if inp.dtype == W.BF16 else 4
