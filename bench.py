@@ -64,10 +64,15 @@ def load_peaks():
 # ---------------------------------------------------------------------------------------------
 # distributed plumbing
 # ---------------------------------------------------------------------------------------------
-def dist_setup():
+def dist_setup(use_gpu: bool = True):
+    """Rank, world size and local rank from the launcher's environment. The GPU arm binds a
+    device and, for N > 1, an NCCL process group; the reference arm (CPU oracle, rank 0 only,
+    no collective) touches neither."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    if not use_gpu:
+        return rank, world, local
     if world > 1:
         import datetime
 
@@ -329,8 +334,7 @@ def cpu_baseline(inp: W.AttnInputs, budget_s: float = 20.0) -> dict:
 
 
 # ---------------------------------------------------------------------------------------------
-def config_dict(fwd: FwdCase, world: int) -> dict:
-    i = fwd.inp
+def config_dict(i: W.AttnInputs, world: int) -> dict:
     return {"workload": "varlen TND causal GQA bf16: 16 seqs U{0..8192} (idx 7 empty), Nq=32 Nkv=8 D=128; "
                         "plus CSR fp32 2x8x4096x64 (window 256 + every 64th) and 3 SBH merges 8192x4x32x128 bf16",
             "tokens_per_rank": int(i.Sq), "n_seq": int(i.B), "Nq": i.Nq, "Nkv": i.Nkv, "D": i.D,
@@ -354,9 +358,9 @@ def run_reference(args, rank: int, world: int):
     line = {"impl": "reference", "metric": METRIC, "value": val, "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": {"workload": "varlen TND causal GQA (oracle rows)", "max_len": args.max_len},
+            "data": "synthetic", "config": config_dict(inp, world),
             "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": oracle_threads(), "kind": "oracle",
-                             "sample": f"{rows} random (head, token) rows per step"},
+                             "sample": f"{rows} random (head, query-token) rows of the varlen batch per step, all their visible keys"},
             "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -421,7 +425,7 @@ def run_ours(args, rank: int, world: int, local: int):
     line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": total_ms_max / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": config_dict(fwd, world),
+            "config": config_dict(fwd.inp, world),
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                          "frac": achieved / peak, "traffic": traffic,
                          "kernel": "attn_fwd bf16 (tcgen05)",
@@ -533,14 +537,14 @@ def main(argv=None):
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
-    rank, world, local = dist_setup()
+    rank, world, local = dist_setup(use_gpu=args.impl != "reference")
     try:
         if args.impl == "reference":
             run_reference(args, rank, world)
         else:
             run_ours(args, rank, world, local)
     finally:
-        if world > 1:
+        if world > 1 and args.impl != "reference":
             import torch.distributed as dist
             dist.destroy_process_group()
 
