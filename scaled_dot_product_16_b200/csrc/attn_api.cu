@@ -52,7 +52,7 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 extern "C" {
 
-int attn_abi_version(void) { return (1 << 16) | 0; }
+int attn_abi_version(void) { return (1 << 16) | 2; }  // 1.2: attn_fwd_masked, attn_sparse_csr_tc
 
 const char* attn_status_string(int s) {
   switch (s) {

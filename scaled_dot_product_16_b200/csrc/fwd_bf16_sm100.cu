@@ -191,9 +191,10 @@ struct Work {
   int row0;         // first row (within the sequence) of this block's 256 rows
 };
 
-// EXT: the masked-call features (band lower edge, explicit mask). Plain calls use the EXT = false
-// instantiation, whose softmax loop carries none of their code.
-template <int HD, int HDV, bool F16, bool EXT>
+// EXT: the masked-call features. 0: plain calls, whose softmax loop carries none of their code;
+// 1: the band's lower edge; 2: the band and an explicit mask (its bytes take registers that the
+// band alone does not need).
+template <int HD, int HDV, bool F16, int EXT>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, FwdArgs a, int units_per_seq,
@@ -264,7 +265,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const bool has1 = rows1 > 0;
   // Key tiles run from jlo (the band's first tile for the block's first row; 0 otherwise) to
   // the tile holding each Q tile's last visible key; n0 and n1 count tiles from jlo.
-  const int jlo = EXT ? visible_begin(a.mask_mode, w.row0, a.pre) / kBN : 0;
+  const int jlo = EXT >= 1 ? visible_begin(a.mask_mode, w.row0, a.pre) / kBN : 0;
   const int kv_end0 = visible_end(a.mask_mode, w.row0 + rows0 - 1, w.sq, w.sk, a.next);
   const int kv_end1 = has1 ? visible_end(a.mask_mode, w.row0 + kBM + rows1 - 1, w.sq, w.sk, a.next) : 0;
   const int n0 = max((kv_end0 + kBN - 1) / kBN, jlo) - jlo;
@@ -438,10 +439,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t S = tmem + lane_off + q * 128;
     const uint32_t O = tmem + lane_off + 256 + q * HDV;
     const int lim = i < w.sq ? visible_end(a.mask_mode, i, w.sq, w.sk, a.next) : w.sk;
-    const int lo = EXT && i < w.sq ? visible_begin(a.mask_mode, i, a.pre) : 0;
+    const int lo = EXT >= 1 && i < w.sq ? visible_begin(a.mask_mode, i, a.pre) : 0;
     // explicit mask row of this query (rows past the sequence read none)
     const uint8_t* mrow = nullptr;
-    if constexpr (EXT)
+    if constexpr (EXT == 2)
       if (i < w.sq && a.mask != nullptr) mrow = a.mask + (int64_t)w.b * a.mask_bs + (int64_t)i * a.mask_rs;
 
     float m = -INFINITY;        // running max used for P (log2 units, lazily updated)
@@ -454,8 +455,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
         tc_fence_after();
         const int kbase = (jlo + j) * kBN;
-        uint4 mk[EXT ? 8 : 1];
-        if constexpr (EXT) {
+        uint4 mk[EXT == 2 ? 8 : 1];
+        if constexpr (EXT == 2) {
           // the mask bytes of this row's 128 keys (16 at a time when aligned and whole);
           // issued before the TMEM loads so the two latencies overlap
           if (mrow == nullptr) {
@@ -487,7 +488,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int c = 0; c < 4; ++c) tmem_ld32f(S + c * 32, s[c]);
         tmem_wait_ld();
-        if constexpr (!EXT) {
+        if constexpr (EXT == 0) {
           if (kbase + kBN > lim) {
 #pragma unroll
             for (int c = 0; c < kBN; ++c)
@@ -499,7 +500,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int c = 0; c < kBN; ++c)
               if (kbase + c >= lim || kbase + c < lo) s[c >> 5][c & 31] = -INFINITY;
           }
-          if (mrow != nullptr) {
+          if (EXT == 2 && mrow != nullptr) {
 #pragma unroll
           for (int c = 0; c < kBN; ++c) {
             const uint4 v4 = mk[c >> 4];
@@ -711,8 +712,9 @@ cudaError_t launch_hd(const FwdArgs& a, cudaStream_t st) {
          make_map(&tv, a.v, Dv, a.Nkv, tk_rows, Dv * 2, (uint64_t)a.Nkv * Dv * 2, 1, kBN, F16);
   }
   if (!ok) return cudaErrorInvalidValue;
-  const bool ext = a.mask != nullptr || a.mask_mode == ATTN_MASK_BAND;
-  auto kernel = ext ? fwd_bf16_kernel<HD, HDV, F16, true> : fwd_bf16_kernel<HD, HDV, F16, false>;
+  auto kernel = a.mask != nullptr                 ? fwd_bf16_kernel<HD, HDV, F16, 2>
+                : a.mask_mode == ATTN_MASK_BAND ? fwd_bf16_kernel<HD, HDV, F16, 1>
+                                                : fwd_bf16_kernel<HD, HDV, F16, 0>;
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return e;
   int units_per_seq = 0;
