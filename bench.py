@@ -45,7 +45,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one attn_fwd launch on the
 # full varlen workload, from a one-pass ncu capture (profiles/attn_fwd_bf16_varlen.md); it is
 # reported only while the kernel source still has the hash it was measured on.
-TRAFFIC = {"kernel_sha": "eefbe2f34578ff23", "bytes_per_launch": 937_251_840 + 602_236_928}
+TRAFFIC = {"kernel_sha": "3612f886071302b1", "bytes_per_launch": 937_927_936 + 600_918_272}
 
 
 def kernel_sha() -> str:
@@ -229,7 +229,7 @@ def _device_ms(fn, iters: int, stream) -> float:
     return a.elapsed_time(b) / iters
 
 
-def next_rows(fwd: "FwdCase", csr: "CsrCase", rank: int, stream) -> dict:
+def next_rows(fwd: "FwdCase", csr: "CsrCase", rank: int, stream, peaks: dict) -> dict:
     """The operations built beyond the step's own rows, each timed on its own: the fused
     ring fold, the band (sliding window) and the tensor-core CSR variant."""
     res = {}
@@ -251,8 +251,11 @@ def next_rows(fwd: "FwdCase", csr: "CsrCase", rank: int, stream) -> dict:
 
     ms = _device_ms(ring, 5, stream)
     fl = M.attn_fwd_flops(inp)
+    tensor = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
     res["attn_fwd_accumulate"] = {"workload": "ring: dense 4x32x8192x128 bf16, 4 key chunks of 2048",
-                                  "ms_per_ring": ms, "tflops": fl / (ms / 1e3) / 1e12, "launches": 4}
+                                  "ms_per_ring": ms, "tflops": fl / (ms / 1e3) / 1e12, "launches": 4,
+                                  "frac_of_sustained_bf16": fl / (ms / 1e3) / 1e12 / tensor}
     del q, kc, vc, acc, am, al
     # sliding window: 1024 keys back, none ahead, on the step's varlen workload
     i = fwd.inp
@@ -269,7 +272,8 @@ def next_rows(fwd: "FwdCase", csr: "CsrCase", rank: int, stream) -> dict:
     fl = 4 * i.Nq * i.D * M.band_pairs(i, 1023, 0)
     res["attn_fwd_masked"] = {"workload": "band pre=1023 next=0 (sliding window) on the varlen GQA "
                                           "batch of the step (Nq=32 Nkv=8 D=128 bf16)",
-                              "ms": ms, "tflops": fl / (ms / 1e3) / 1e12, "flops_per_call": fl}
+                              "ms": ms, "tflops": fl / (ms / 1e3) / 1e12, "flops_per_call": fl,
+                              "frac_of_sustained_bf16": fl / (ms / 1e3) / 1e12 / tensor}
     # CSR on the tensor cores: the fp32 CSR workload's pattern with bf16 inputs
     c = csr if csr is not None else CsrCase(W.cfg4_csr(seed=rank))
     qb, kb, vb = (t.to(torch.bfloat16) for t in (c.q, c.k, c.v))
@@ -284,7 +288,30 @@ def next_rows(fwd: "FwdCase", csr: "CsrCase", rank: int, stream) -> dict:
     ms32 = _device_ms(c.run, 20, stream)
     res["attn_sparse_csr_tc"] = {"workload": "2x8x4096x64 bf16, window 256 + every 64th column",
                                  "ms": ms, "tflops": c.flops / (ms / 1e3) / 1e12,
+                                 "frac_of_sustained_bf16": c.flops / (ms / 1e3) / 1e12 / tensor,
                                  "fp32_kernel_ms": ms32, "speedup_vs_fp32": ms32 / ms}
+    del qb, kb, vb, outb
+    # merge in the TND layout (ring-attention update of a packed batch): T = 65,536 tokens,
+    # N = 32, D = 128, bf16 outputs, [T, N, 8] statistics, with actual_seq_qlen checked
+    T, N, D = 65536, 32, 128
+    po = W.randn((T, N * D), W.mix_seed(6, rank, 1), torch.bfloat16).cuda()
+    co = W.randn((T, N * D), W.mix_seed(6, rank, 2), torch.bfloat16).cuda()
+    pm, ps = (x.reshape(1, N, T, 8).permute(0, 2, 1, 3).reshape(T, N, 8).contiguous().cuda()
+              for x in W.merge_stats_random(1, N, T, W.mix_seed(6, rank, 3)))
+    cm, cs = (x.reshape(1, N, T, 8).permute(0, 2, 1, 3).reshape(T, N, 8).contiguous().cuda()
+              for x in W.merge_stats_random(1, N, T, W.mix_seed(6, rank, 4)))
+    seq = torch.tensor([T // 4, T // 2, 3 * T // 4, T], dtype=torch.int64, device="cuda")
+    mo, mm, ml = torch.empty_like(po), torch.empty_like(pm), torch.empty_like(ps)
+
+    def merge_tnd():
+        sdpa.attn_merge(po, pm, ps, co, cm, cs, S=T, B=4, N=N, D=D, dtype=W.BF16, layout=W.TND,
+                        actual_seq_qlen=seq, out=mo, out_max=mm, out_sum=ml)
+
+    ms = _device_ms(merge_tnd, 20, stream)
+    by = M.merge_bytes(T, 1, N, D, 2)
+    res["attn_merge_tnd"] = {"workload": "TND T=65536 N=32 D=128 bf16, [T,N,8] statistics, 4 sequences",
+                             "ms": ms, "gbs": by / (ms / 1e3) / 1e9,
+                             "frac_of_hbm": by / (ms / 1e3) / 1e9 / hbm, "bytes_per_call": by}
     return res
 
 
@@ -513,7 +540,7 @@ def run_ours(args, rank: int, world: int, local: int):
                        "and outputs + statistics copied back, every step; steps pipelined over two "
                        "buffer sets and three streams (copy in, compute, copy out)"}
     if not args.no_next_rows:
-        line["next_rows"] = next_rows(fwd, csr, rank, stream)
+        line["next_rows"] = next_rows(fwd, csr, rank, stream, peaks)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(fwd.inp, args.cpu_budget)
     if rank == 0:
