@@ -50,7 +50,7 @@ extern "C" {
 typedef enum {
   ATTN_OK = 0,
   ATTN_ERR_INVALID = 1,     /* bad shape, null pointer, inconsistent sizes              */
-  ATTN_ERR_UNSUPPORTED = 2, /* valid request this build does not run (e.g. bf16, D=96)  */
+  ATTN_ERR_UNSUPPORTED = 2, /* valid request this library does not run (e.g. bf16, D=96) */
   ATTN_ERR_CUDA = 3,        /* a CUDA runtime call failed (launch, device query)        */
   ATTN_ERR_DATA = 4,        /* device-side: bad cumulative lengths or CSR indices       */
   ATTN_ERR_TIMEOUT = 5      /* device-side: a pipeline wait exceeded its bound          */
@@ -92,7 +92,7 @@ typedef enum {
  * softmax_max / softmax_sum may both be NULL to skip the statistics. mask_mode is 0, 1 or 2
  * (the band needs attn_fwd_masked).
  * Limits (from the constraints): 1 <= Nq <= 256, D <= 768 (larger D is ATTN_ERR_INVALID;
- * sizes this build does not run are ATTN_ERR_UNSUPPORTED), Tq, Tkv <= 1M tokens and
+ * sizes this library does not run are ATTN_ERR_UNSUPPORTED), Tq, Tkv <= 1M tokens and
  * B <= 2048 for TND; scale must be finite and > 0. Empty problems (B = 0, Sq = 0 or a total
  * of 0 tokens) return ATTN_OK without a launch. For ATTN_BF16 and ATTN_F16, q, k, v and out
  * must be 16-byte aligned.

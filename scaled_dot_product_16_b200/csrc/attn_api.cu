@@ -58,7 +58,7 @@ const char* attn_status_string(int s) {
   switch (s) {
     case ATTN_OK: return "ok";
     case ATTN_ERR_INVALID: return "invalid argument";
-    case ATTN_ERR_UNSUPPORTED: return "unsupported by this build";
+    case ATTN_ERR_UNSUPPORTED: return "unsupported by this library";
     case ATTN_ERR_CUDA: return "CUDA runtime error";
     case ATTN_ERR_DATA: return "bad device data (cumulative lengths or CSR indices)";
     case ATTN_ERR_TIMEOUT: return "pipeline wait timed out";
