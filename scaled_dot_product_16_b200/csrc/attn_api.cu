@@ -215,11 +215,16 @@ int attn_sparse_csr(const float* q, const float* k, const float* v, const int32_
   a.S = S;
   a.D = D;
   a.nnz_cap = nnz_cap;
+  a.cols_vec = csr_columns != nullptr && aligned16(csr_columns) && nnz_cap % 4 == 0;
   a.out = out;
   int sms = 0;
   int rc = device_state(&a.status, &sms);
   if (rc != ATTN_OK) return rc;
-  const cudaError_t e = sdpa::launch_sparse_csr(a, static_cast<cudaStream_t>(stream));
+  // D = 64 or 128 with 16-byte aligned tensors: tiled over each block's union of columns;
+  // otherwise a warp per row gathering its own entries
+  const cudaError_t e = sdpa::sparse_csr_tiled_supported(a)
+                            ? sdpa::launch_sparse_csr_tiled(a, static_cast<cudaStream_t>(stream))
+                            : sdpa::launch_sparse_csr(a, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 

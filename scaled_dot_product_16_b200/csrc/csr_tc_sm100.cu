@@ -17,10 +17,9 @@
 //   * each row keeps a byte per union column of the current 512-column window (256 at D = 128:
 //     "is this column one of my entries"); the softmax sets the other scores to -inf, so every row sums over
 //     exactly its own entries, with the online (streaming) update and a lazy rescale;
-//   * the union pass streams the block's entries (one contiguous span when the row pointers are
-//     good) with 16-byte loads, writing a plain byte per column that is packed into the bitmap
-//     afterwards, so no update is a read-modify-write; each softmax thread then builds its own
-//     row's bytes from its own columns, 16 loads deep, with no other thread involved;
+//   * the union is built as csr_union.cuh describes (one streamed pass over the block's span of
+//     column indices); each softmax thread then builds its own row's bytes from its own
+//     columns, 16 loads deep, with no other thread involved;
 //   * P is written to TMEM as a 16-bit high part and a 16-bit remainder, and O accumulates both
 //     (two MMAs per key step): rows with few entries put large weights on few values, where a
 //     single 16-bit P would cost up to 2^-9 of |v| on top of the output's own rounding;
@@ -30,6 +29,7 @@
 #include <math.h>
 
 #include "common.cuh"
+#include "csr_union.cuh"
 #include "launch.h"
 #include "sm100.cuh"
 
@@ -102,7 +102,6 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile
   }
 }
 
-constexpr int kSpanBatch = 16;  // column indices each thread loads before using any (union pass)
 constexpr int kRowBatch = 16;   // a row's column indices its thread loads before using any
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool valid) {
@@ -185,129 +184,11 @@ __global__ void __launch_bounds__(kThreads, 1) csr_tc_kernel(CsrTcArgs a, float 
   const uint32_t tmem = bars->tmem_base;
   volatile int* abort = &bars->abort;
 
-  // ---- row pointers and the union of the block's columns ------------------------------------
-  // Thread x checks row r0 + x. When every row pointer is good, the block's entries are one
-  // contiguous span of the column array and all threads stream it in 16-deep batches, writing
-  // a byte per column. Otherwise (or when a column is out of range) a slow pass goes a row per
-  // warp at a time and flags the offending rows, which are written as zeros.
+  // ---- the union of the block's rows' columns (csr_union.cuh) ---------------------------------
   const int r = warp * 32 + lane;
   const int i = r0 + r;
-  const int nrows = min(kRows, S - r0);
-  bool good_x = true;
-  if (threadIdx.x < kRows) {
-    const int x = threadIdx.x, ii = r0 + x;
-    int c0 = 0, c1 = 0;
-    if (ii < S) {
-      c0 = __ldg(off + ii);
-      c1 = __ldg(off + ii + 1);
-      good_x = !(c0 < 0 || c1 < c0 || (int64_t)c1 > a.nnz_cap || (ii == 0 && c0 != 0));
-    } else {
-      c0 = c1 = __ldg(off + S);  // past the end: empty rows at the span's end
-    }
-    row_c0[x] = good_x ? c0 : 0;
-    row_c1[x] = good_x ? c1 : 0;
-    if (!good_x) {
-      row_bad[x] = 1;
-      report(a.status, ATTN_ERR_DATA);
-    }
-  }
-  if (threadIdx.x == 0) misc[1] = 0;
-  const bool all_good = __syncthreads_and(good_x) != 0;
-  if (all_good) {
-    const int E0 = row_c0[0], E1 = row_c1[kRows - 1];
-    bool col_bad = false;
-    if (a.cols_vec) {
-      // 16 bytes (4 indices) per load from the aligned quad holding E0 on; quads end at
-      // nnz_cap, a multiple of 4, so none reads past this (b, h)'s columns
-      for (int q0 = E0 >> 2; q0 * 4 < E1; q0 += kThreads * (kSpanBatch / 4)) {
-        int4 jj[kSpanBatch / 4];
-#pragma unroll
-        for (int b = 0; b < kSpanBatch / 4; ++b) {
-          const int q = q0 + b * kThreads + (int)threadIdx.x;
-          jj[b] = q * 4 < E1 ? __ldg(reinterpret_cast<const int4*>(cols) + q) : make_int4(0, 0, 0, 0);
-        }
-#pragma unroll
-        for (int b = 0; b < kSpanBatch / 4; ++b) {
-          const int e = (q0 + b * kThreads + (int)threadIdx.x) * 4;
-          const int js[4] = {jj[b].x, jj[b].y, jj[b].z, jj[b].w};
-#pragma unroll
-          for (int z = 0; z < 4; ++z) {
-            if (e + z >= E0 && e + z < E1) {
-              if (js[z] >= 0 && js[z] < S) bytes[js[z]] = 1;
-              else col_bad = true;
-            }
-          }
-        }
-      }
-    } else {
-      for (int base = E0; base < E1; base += kThreads * kSpanBatch) {
-        int jj[kSpanBatch];
-#pragma unroll
-        for (int b = 0; b < kSpanBatch; ++b) {
-          const int e = base + b * kThreads + (int)threadIdx.x;
-          jj[b] = e < E1 ? __ldg(cols + e) : 0;
-        }
-#pragma unroll
-        for (int b = 0; b < kSpanBatch; ++b) {
-          const int e = base + b * kThreads + (int)threadIdx.x, j = jj[b];
-          if (e < E1) {
-            if (j >= 0 && j < S) bytes[j] = 1;
-            else col_bad = true;
-          }
-        }
-      }
-    }
-    if (col_bad) misc[1] = 1;
-  }
-  __syncthreads();
-  if (!all_good || misc[1] != 0) {
-    // slow pass: a row per warp, good rows only; rows holding a bad column are flagged
-    for (int rr = warp; rr < nrows; rr += kThreads / 32) {
-      const int c0 = row_c0[rr], c1 = row_c1[rr];
-      bool col_bad = false;
-      for (int e = (row_bad[rr] ? c1 : c0) + lane; e < c1; e += 32) {
-        const int j = __ldg(cols + e);
-        if (j >= 0 && j < S) bytes[j] = 1;
-        else col_bad = true;
-      }
-      if (__any_sync(0xffffffffu, col_bad) && lane == 0) {
-        row_bad[rr] = 1;
-        report(a.status, ATTN_ERR_DATA);
-      }
-    }
-  }
-  __syncthreads();
-  // pack the column bytes into bitmap words (byte b of a 32-bit group -> bit b)
-  for (int w = threadIdx.x; w < nw; w += kThreads) {
-    const uint32_t* g = reinterpret_cast<const uint32_t*>(bytes) + w * 8;
-    uint32_t bits = 0;
-#pragma unroll
-    for (int x = 0; x < 8; ++x) {
-      const uint32_t v = g[x];
-      bits |= ((v & 1u) | ((v >> 7) & 2u) | ((v >> 14) & 4u) | ((v >> 21) & 8u)) << (4 * x);
-    }
-    bitmap[w] = bits;
-  }
-  __syncthreads();
-  if (warp == kMmaWarp) {
-    // exclusive prefix of the popcounts, 32 words at a time
-    uint32_t carry = 0;
-    for (int w0 = 0; w0 < nw; w0 += 32) {
-      const int w = w0 + lane;
-      const uint32_t c = w < nw ? (uint32_t)__popc(bitmap[w]) : 0u;
-      uint32_t x = c;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
-        if (lane >= o) x += y;
-      }
-      if (w < nw) wpre[w] = carry + x - c;
-      carry += __shfl_sync(0xffffffffu, x, 31);
-    }
-    if (lane == 0) misc[0] = (int)carry;
-  }
-  __syncthreads();
-  const int U = misc[0];
+  const CsrUnion un{bitmap, wpre, bytes, row_c0, row_c1, row_bad, misc};
+  const int U = csr_block_union<kThreads, kRows>(un, off, cols, S, r0, a.nnz_cap, a.cols_vec, a.status);
   const int T = (U + kKeys - 1) / kKeys;  // gathered key tiles
 
   const uint32_t sQ = smem_u32(smem + C::kQOff);
@@ -317,19 +198,7 @@ __global__ void __launch_bounds__(kThreads, 1) csr_tc_kernel(CsrTcArgs a, float 
   if (warp >= kProdWarp) {
     // =============================== gather producers ====================================
     const int p = warp - kProdWarp;
-    // union column u: the word holding the u-th set bit (largest w with wpre[w] <= u), then
-    // the bit of that rank inside it
-    auto union_col = [&](int u) -> int {
-      int lo = 0, hi = nw - 1;
-      while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if ((int)wpre[mid] <= u) lo = mid;
-        else hi = mid - 1;
-      }
-      uint32_t bits = bitmap[lo];
-      for (int z = (int)(u - (int)wpre[lo]); z > 0; --z) bits &= bits - 1;
-      return lo * 32 + (__ffs(bits) - 1);
-    };
+    auto union_col = [&](int u) { return csr_union_col(bitmap, wpre, nw, u); };
     bool ok = true;
     if (p == 0 && T > 0) {
       gather_tile<HD>(sQ, [&](int k) { return r0 + k < S ? Qb + (int64_t)(r0 + k) * HD : nullptr; }, Qb, lane);
@@ -426,7 +295,7 @@ __global__ void __launch_bounds__(kThreads, 1) csr_tc_kernel(CsrTcArgs a, float 
           for (int b = 0; b < kRowBatch; ++b) {
             const int j = jj[b];
             if (j >= 0 && j < S) {  // bad columns are already flagged; the row is zeroed
-              const int u = (int)wpre[j >> 5] + __popc(bitmap[j >> 5] & ((1u << (j & 31)) - 1u));
+              const int u = csr_union_index(bitmap, wpre, j);
               if (u >= base && u < base + C::kWin) {
                 row[u - base] = 1;
                 ++hits;

@@ -36,6 +36,7 @@ struct CsrArgs {
   const int32_t* columns;
   int B, H, S, D;
   int64_t nnz_cap;
+  bool cols_vec;  // columns 16-byte aligned and nnz_cap % 4 == 0: read 4 indices at a time
   float* out;
   int* status;
 };
@@ -72,6 +73,8 @@ cudaError_t launch_merge(const MergeArgs& a, cudaStream_t st);
 cudaError_t launch_fwd_f32(const FwdArgs& a, cudaStream_t st);
 cudaError_t launch_fwd_bf16(const FwdArgs& a, cudaStream_t st);
 cudaError_t launch_sparse_csr(const CsrArgs& a, cudaStream_t st);
+bool sparse_csr_tiled_supported(const CsrArgs& a);
+cudaError_t launch_sparse_csr_tiled(const CsrArgs& a, cudaStream_t st);
 cudaError_t launch_sparse_csr_tc(const CsrTcArgs& a, cudaStream_t st);
 
 }  // namespace sdpa

@@ -96,3 +96,65 @@ def test_bad_columns_report_data_error():
     cols[0, 0, 3] = 3
     out, st = _run(q, q, q, off2, cols, B, H, S, D)
     assert st == sdpa.ATTN_ERR_DATA
+
+
+# ---- the tiled path (D = 64 or 128, 16-byte aligned tensors) and the row-per-warp path ---------
+def test_repeated_columns_count_per_entry_tiled():
+    """A column stored c times in a row weighs c times (reading of the row pointer), including
+    a column stored 300 times, past what a byte of the tiled kernel's counts holds."""
+    B, H, S, D = 1, 2, 200, 64
+    q, k, v = (W.randn((B, H, S, D), 400 + i) for i in range(3))
+    rng = np.random.default_rng(3)
+    rows = []
+    for i in range(S):
+        base = rng.integers(0, S, size=int(rng.integers(0, 12)))
+        if i % 7 == 0:
+            base = np.concatenate([base, np.full(3, i)])      # a few repeats
+        if i == 100:
+            base = np.concatenate([base, np.full(300, 5)])    # 300 copies of one column
+        rows.append(base.astype(np.int32))
+    cnt = np.array([len(r) for r in rows])
+    off1 = np.concatenate([[0], np.cumsum(cnt)]).astype(np.int32)
+    col1 = np.concatenate(rows).astype(np.int32)
+    off = np.broadcast_to(off1, (B, H, S + 1)).copy()
+    cols = np.broadcast_to(col1, (B, H, col1.size)).copy()
+    out, st = _run(q, k, v, off, cols, B, H, S, D)
+    assert st == 0
+    ref = oracle.sparse_csr(q, k, v, off, cols, B=B, H=H, S=S, D=D)
+    G.check_out(out.numpy(), ref, W.F32, "repeats")
+
+
+@pytest.mark.parametrize("D", [64, 128])
+def test_union_wider_than_one_window_tiled(D):
+    """Rows of 150 random columns over 2,560 keys: each 128-row block's union spans about 2,000
+    columns, so the per-row counts are rebuilt window after window."""
+    rng = np.random.default_rng(D)
+    B, H, S = 1, 2, 2560
+    q, k, v = (W.randn((B, H, S, D), 500 + i) for i in range(3))
+    off, cols = _random_pattern(rng, B, H, S, 150)
+    out, st = _run(q, k, v, off, cols, B, H, S, D)
+    assert st == 0
+    ref = oracle.sparse_csr(q, k, v, off, cols, B=B, H=H, S=S, D=D)
+    G.check_out(out.numpy(), ref, W.F32, "wide union")
+
+
+def test_row_per_warp_path_on_misaligned_tensors():
+    """A q view that starts 4 bytes into its buffer is not 16-byte aligned, so the call takes the
+    row-per-warp kernel; both paths agree with the oracle on the same data."""
+    B, H, S, D = 1, 2, 130, 64
+    rng = np.random.default_rng(11)
+    q, k, v = (W.randn((B, H, S, D), 600 + i) for i in range(3))
+    off, cols = _random_pattern(rng, B, H, S, 30)
+    ref = oracle.sparse_csr(q, k, v, off, cols, B=B, H=H, S=S, D=D)
+    buf = torch.zeros(B * H * S * D + 1, device="cuda")
+    dq = buf[1:].view(B, H, S, D)
+    dq.copy_(q.cuda())
+    dk, dv = k.cuda(), v.cuda()
+    out = torch.full_like(dk, float("nan"))
+    sdpa.attn_sparse_csr(dq, dk, dv, torch.from_numpy(off).cuda(), torch.from_numpy(cols).cuda(),
+                         B=B, H=H, S=S, D=D, nnz_cap=cols.shape[-1], out=out)
+    assert sdpa.attn_get_last_error() == 0
+    G.check_out(out.cpu().numpy(), ref, W.F32, "row-per-warp path")
+    out2, st = _run(q, k, v, off, cols, B, H, S, D)
+    assert st == 0
+    G.check_out(out2.numpy(), ref, W.F32, "tiled path")
