@@ -172,8 +172,8 @@ __global__ void __launch_bounds__(kThreads) merge_sbh_kernel(
         if (idx[u] < total) {
           const int r = idx[u] / vpr, c = idx[u] - r * vpr;
           const int64_t off = row0 + r * row_stride + (int64_t)c * V;
-          pv[u] = __ldcs(reinterpret_cast<const uint4*>(prev_out + off));
-          cv[u] = __ldcs(reinterpret_cast<const uint4*>(cur_out + off));
+          pv[u] = *reinterpret_cast<const uint4*>(prev_out + off);
+          cv[u] = *reinterpret_cast<const uint4*>(cur_out + off);
         }
       }
 #pragma unroll
@@ -187,7 +187,7 @@ __global__ void __launch_bounds__(kThreads) merge_sbh_kernel(
           const float po = s_po[r], co = s_co[r];
 #pragma unroll
           for (int i = 0; i < V; ++i) o[i] = fmaf(a[i], po, bb[i] * co);
-          __stcs(reinterpret_cast<uint4*>(out + off), pack(o, (T*)nullptr));
+          *reinterpret_cast<uint4*>(out + off) = pack(o, (T*)nullptr);
         }
       }
     }
@@ -236,8 +236,8 @@ __global__ void __launch_bounds__(THREADS) merge_sbh_vec_kernel(
     if (idx < total) {
       const int r = idx / vpr, c = idx - r * vpr;
       const int64_t off = row0 + r * row_stride + (int64_t)c * V;
-      pv[u] = __ldcs(reinterpret_cast<const uint4*>(prev_out + off));
-      cv[u] = __ldcs(reinterpret_cast<const uint4*>(cur_out + off));
+      pv[u] = *reinterpret_cast<const uint4*>(prev_out + off);
+      cv[u] = *reinterpret_cast<const uint4*>(cur_out + off);
     }
   }
   // 2. lane-wise statistics, one (row, lane) element per thread
@@ -270,7 +270,7 @@ __global__ void __launch_bounds__(THREADS) merge_sbh_vec_kernel(
       const float po = s_po[r], co = s_co[r];
 #pragma unroll
       for (int i = 0; i < V; ++i) o[i] = fmaf(a[i], po, bb[i] * co);
-      __stcs(reinterpret_cast<uint4*>(out + off), pack(o, (T*)nullptr));
+      *reinterpret_cast<uint4*>(out + off) = pack(o, (T*)nullptr);
     }
   }
 }
