@@ -182,7 +182,9 @@ ATTN_API int attn_fwd_masked(const void* q, const void* k, const void* v,
  *                  offset[S] <= nnz_cap
  *   csr_columns    int32 [B, H, nnz_cap]: column of each stored entry, 0 <= j < S; order
  *                  within a row is free and a repeated column counts once per entry
- * An empty row gives an output row of zeros. 1 <= D <= 256.
+ * An empty row gives an output row of zeros. 1 <= D <= 256. D = 64 or 128 with 16-byte aligned
+ * q, k, v, out and S <= 32768 run a kernel tiled over each block's union of columns; other
+ * shapes run a warp per row. Both compute in float32 with the same definition.
  * Data errors: a column outside [0, S), or a row pointer that starts above 0, decreases or
  * passes nnz_cap, set ATTN_ERR_DATA; the affected rows are written as zeros.
  */
