@@ -45,7 +45,9 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one attn_fwd launch on the
 # full varlen workload, from a one-pass ncu capture (profiles/attn_fwd_bf16_varlen.md); it is
 # reported only while the kernel source still has the hash it was measured on.
-TRAFFIC = {"kernel_sha": "3612f886071302b1", "bytes_per_launch": 937_927_936 + 600_918_272}
+# DRAM bytes per attn_fwd launch from an ncu capture, valid only for this kernel source and this
+# workload (the default varlen batch of 75,336 tokens)
+TRAFFIC = {"kernel_sha": "3612f886071302b1", "tokens": 75_336, "bytes_per_launch": 937_927_936 + 600_918_272}
 
 
 def kernel_sha() -> str:
@@ -448,7 +450,8 @@ def run_ours(args, rank: int, world: int, local: int):
     # dominant kernel roofline (attn_fwd, timed inside a long step: sustained peak)
     achieved = fwd.flops / (fwd_ms / args.steps / 1e3) / 1e12
     peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
-    traffic = TRAFFIC["bytes_per_launch"] if TRAFFIC["kernel_sha"] == kernel_sha() else None
+    traffic = (TRAFFIC["bytes_per_launch"]
+               if TRAFFIC["kernel_sha"] == kernel_sha() and int(fwd.inp.Sq) == TRAFFIC["tokens"] else None)
     line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": total_ms_max / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",

@@ -151,17 +151,21 @@ __global__ void __launch_bounds__(kThreads, D == 64 ? 2 : 1) csr_f32_tiled_kerne
       kcol[lane] = u < U ? csr_union_col(bitmap, wpre, nw, u) : -1;
     }
     __syncthreads();
+    // key rows: lane = key, so the transposed stores of a warp fall in 32 different banks
     for (int x = tid; x < kKeys * (D / 4); x += kThreads) {
-      const int k = x / (D / 4), c4 = x % (D / 4), col = kcol[k];
-      float4 kv = make_float4(0.f, 0.f, 0.f, 0.f), vv = kv;
-      if (col >= 0) {
-        kv = __ldg(reinterpret_cast<const float4*>(Kb + (int64_t)col * D) + c4);
-        vv = __ldg(reinterpret_cast<const float4*>(Vb + (int64_t)col * D) + c4);
-      }
+      const int k = x % kKeys, c4 = x / kKeys, col = kcol[k];
+      float4 kv = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (col >= 0) kv = __ldg(reinterpret_cast<const float4*>(Kb + (int64_t)col * D) + c4);
       Kt[(4 * c4 + 0) * kKeys + k] = kv.x;
       Kt[(4 * c4 + 1) * kKeys + k] = kv.y;
       Kt[(4 * c4 + 2) * kKeys + k] = kv.z;
       Kt[(4 * c4 + 3) * kKeys + k] = kv.w;
+    }
+    // value rows: lanes along the row, so every row is one contiguous 16-byte-per-lane store
+    for (int x = tid; x < kKeys * (D / 4); x += kThreads) {
+      const int k = x / (D / 4), c4 = x % (D / 4), col = kcol[k];
+      float4 vv = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (col >= 0) vv = __ldg(reinterpret_cast<const float4*>(Vb + (int64_t)col * D) + c4);
       reinterpret_cast<float4*>(Vs + k * D)[c4] = vv;
     }
     __syncthreads();
