@@ -6,25 +6,25 @@
 //
 // Design (tiles of the CSR pattern, gathered):
 //   * a block owns 128 query rows of one (b, h); row r is TMEM lane r and softmax thread r;
-//   * the block first takes the union of the columns its rows store: a bitmap over the S keys
-//     in shared memory, then an exclusive prefix of the words' popcounts. Union column u is the
-//     u-th set bit, so the union is sorted and each key appears once;
+//   * the block first takes the union of the columns its rows store (csr_union.cuh): a bitmap
+//     over the S keys with an exclusive prefix of its words' popcounts, built from one streamed
+//     pass over the block's column indices. Union column u is the u-th set bit, so the union
+//     is sorted and each key appears once;
 //   * two producer warps gather the union's key and value rows, 128 per tile, with 16-byte
 //     cp.async into the 128-byte-swizzled K-major layout the MMA descriptors expect (the same
 //     layout a TMA load with 128-byte swizzle gives), zero-filling past the union's end;
 //   * one thread issues S = Q K_t^T (both operands in shared memory) into one of two TMEM score
 //     buffers, and O += P_t V_t with P read from TMEM; S_{t+1} overlaps the softmax of tile t;
-//   * each row keeps a byte per union column of the current 512-column window (256 at D = 128:
-//     "is this column one of my entries"); the softmax sets the other scores to -inf, so every row sums over
-//     exactly its own entries, with the online (streaming) update and a lazy rescale;
-//   * the union is built as csr_union.cuh describes (one streamed pass over the block's span of
-//     column indices); each softmax thread then builds its own row's bytes from its own
-//     columns, 16 loads deep, with no other thread involved;
+//   * each row keeps a byte per union column of the current window (512 columns at D = 64, 256
+//     at D = 128) that says whether the column is one of its entries, built by the row's own
+//     softmax thread from its own columns, 16 loads deep; the softmax sets the other scores to
+//     -inf, so every row sums over exactly its own entries, with the online (streaming) update
+//     and a lazy rescale;
 //   * P is written to TMEM as a 16-bit high part and a 16-bit remainder, and O accumulates both
 //     (two MMAs per key step): rows with few entries put large weights on few values, where a
 //     single 16-bit P would cost up to 2^-9 of |v| on top of the output's own rounding;
 //   * every wait is bounded; a timeout records ATTN_ERR_TIMEOUT and the block drains and exits.
-// A column stored twice in one row would be counted once by the bit mask, so a repeated
+// A column stored twice in one row would be counted once by the byte mask, so a repeated
 // column is reported as ATTN_ERR_DATA and that row is written as zeros.
 #include <math.h>
 
