@@ -193,3 +193,31 @@ def test_tensor_core_path_rejects_other_value_sizes():
         with pytest.raises(sdpa.AttnError) as e:
             _run(inp, mode=W.MASK_NONE, Dv=Dv)
         assert e.value.status == sdpa.ATTN_ERR_UNSUPPORTED
+
+
+def test_causal_attention_from_band_masked_key_chunks():
+    """Causal attention over 512 keys assembled from 4 chunks of 128 keys, as a ring of devices
+    would: chunk c sees key j' (its own index) iff j' <= i - 128c, a band with unbounded
+    look-back and look-ahead -128c. Each chunk's result (with rows that see none of its keys
+    giving out 0, max -inf, sum 0) is merged in turn; the end result equals causal attention."""
+    B, N, S, D, L = 1, 2, 512, 128, 128
+    full = W.dense_bhsd(B, N, S, D, causal=True, dtype=BF, seed=7, cfg=43)
+    acc = None
+    for c in range(S // L):
+        kc = full.k[:, :, c * L:(c + 1) * L].contiguous()
+        vc = full.v[:, :, c * L:(c + 1) * L].contiguous()
+        chunk = W.AttnInputs(full.q, kc, vc, W.BHSD, W.MASK_NONE, W.BF16, B, S, L, N, N, D, full.scale)
+        out, m, l = _run(chunk, mode=BAND, pre=1 << 40, nxt=-c * L)
+        part = [out.permute(2, 0, 1, 3).reshape(S, B, N * D).contiguous().cuda(),
+                m.unsqueeze(-1).expand(B, N, S, 8).contiguous().cuda(),
+                l.unsqueeze(-1).expand(B, N, S, 8).contiguous().cuda()]
+        if acc is None:
+            acc = part
+            continue
+        sdpa.attn_merge(acc[0], acc[1], acc[2], *part, S=S, B=B, N=N, D=D, dtype=W.BF16,
+                        out=acc[0], out_max=acc[1], out_sum=acc[2])
+        assert sdpa.attn_get_last_error() == 0
+    got = acc[0].cpu().reshape(S, B, N, D).permute(1, 2, 0, 3)
+    ref, rm, rl = G.oracle_fwd(full)
+    G.check_out(G.f64(got), ref, W.BF16, "causal from chunks")
+    G.check_stats(acc[1][..., 0].cpu().numpy(), acc[2][..., 0].cpu().numpy(), rm, rl, "causal stats")
