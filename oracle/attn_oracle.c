@@ -19,6 +19,9 @@
  *               columns [B,H,nnz]; softmax over the stored entries of each row only.
  *   merge       "npu_ring_attention_update" (MindSpeed op doc), 小算子等价计算逻辑: lane-wise
  *               max/sum update over [B,N,S,8] statistics, output rescaled with lane 0.
+ *   masked      "aclnnFlashAttentionVarLenScore", 约束说明: band limits (preTokens/nextTokens),
+ *               an explicit mask (attenMaskOptional) and a value head size with qD == kD >= vD;
+ *               the readings are stated above oracle_attn_fwd_ext.
  *
  * Statistics convention (the pages only imply it through the merge, which takes exp of
  * differences of maxima): softmax_max = max_j of the scaled score in natural-log units and
