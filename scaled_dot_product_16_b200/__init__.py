@@ -85,11 +85,16 @@ def _status_string(status: int) -> str:
 
 
 def _ptr(x) -> Optional[int]:
-    """Data pointer of a tensor (or an int address, or None)."""
+    """Device data pointer of a tensor (or an int address, or None). Tensors must be on a CUDA
+    device and dense: the C ABI reads them as contiguous device arrays."""
     if x is None:
         return None
     if isinstance(x, int):
         return x
+    if getattr(x, "is_cuda", True) is False:
+        raise ValueError("tensor arguments must be on a CUDA device")
+    if hasattr(x, "is_contiguous") and not x.is_contiguous():
+        raise ValueError("tensor arguments must be contiguous")
     return int(x.data_ptr())
 
 

@@ -151,6 +151,28 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
                         out=None, out_max=None, out_sum=None, stream=0)
 
 
+def test_binding_rejects_host_and_strided_tensors(lib):
+    """The C ABI reads device arrays; the binding refuses host tensors (whose addresses a kernel
+    cannot read) and non-contiguous views before anything is called."""
+    import torch
+    host = torch.zeros(4, 8)
+    with pytest.raises(ValueError, match="CUDA device"):
+        sdpa.attn_merge(host, host, host, host, host, host, S=1, B=1, N=1, D=8, dtype=sdpa.ATTN_F32,
+                        out=host, out_max=host, out_sum=host, stream=0)
+
+    class Strided:  # stands in for a strided CUDA tensor on a machine without a GPU
+        is_cuda = True
+
+        def is_contiguous(self):
+            return False
+
+        def data_ptr(self):
+            return 16
+
+    with pytest.raises(ValueError, match="contiguous"):
+        sdpa._ptr(Strided())
+
+
 def test_product_never_touches_the_oracle():
     pkg = os.path.join(ROOT, "scaled_dot_product_16_b200")
     for dirpath, _, files in os.walk(pkg):

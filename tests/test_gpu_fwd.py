@@ -157,9 +157,16 @@ def test_host_validation():
     with pytest.raises(sdpa.AttnError) as e:
         sdpa.attn_fwd(q, k, v, **{**kw, "D": 96})
     assert e.value.status == sdpa.ATTN_ERR_UNSUPPORTED
+    # a contiguous view that starts 2 bytes into its buffer: the library's alignment check
+    buf = torch.empty(q.numel() + 1, dtype=q.dtype, device=q.device)
+    qm = buf[1:].view(q.shape)
+    qm.copy_(q)
     with pytest.raises(sdpa.AttnError) as e:
-        sdpa.attn_fwd(q[..., 1:], k, v, **kw)  # misaligned base pointer
+        sdpa.attn_fwd(qm, k, v, **kw)
     assert e.value.status == sdpa.ATTN_ERR_INVALID
+    # a strided view is refused by the binding before the library is called
+    with pytest.raises(ValueError):
+        sdpa.attn_fwd(q[..., 1:], k, v, **kw)
 
 
 # ---- fp16 on the tensor-core path ---------------------------------------------------------------
