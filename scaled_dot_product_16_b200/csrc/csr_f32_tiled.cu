@@ -8,15 +8,21 @@
 // Design: a block owns 128 query rows of one (b, h) (256 threads). It takes the union of its
 // rows' columns (csr_union.cuh), then walks the union 32 keys at a time: the key and value rows
 // are gathered once into shared memory and serve all 128 rows, instead of every row gathering
-// its own ~300 key/value rows through L1/L2 (which bounds the row-per-warp kernel). Scores are
-// a 128x32 register-tiled product on the FMA pipe (4 rows x 4 keys per thread, Q transposed and
-// pre-scaled in shared memory); each row counts how often it stores each union column (a byte
-// per row and union column, 256-column windows, built by the row's own thread), so a score
-// enters the online softmax with weight count * exp(s - m), or not at all. P goes through
-// shared memory to the P.V product (4 rows x D/8 columns per thread). All arithmetic is fp32
-// FMA with expf, as the row-per-warp kernel does. A row that stores one column more than 255
-// times in a window (a count a byte cannot hold) is recomputed exactly by a row-per-warp pass
-// at the end.
+// its own ~300 key/value rows through L1/L2 (which bounds the row-per-warp kernel).
+//  * The gathers are cp.async copies into two buffers: tile t+1's rows are in flight while
+//    tile t is multiplied, and a tile costs two block barriers.
+//  * For each window of 512 union columns, every row's thread marks which of them its row
+//    stores (a bit per row and union column) from its own column list, merging runs of
+//    neighbouring columns in registers. The window's union columns are listed once, a thread
+//    per bitmap word, so no tile searches for its columns.
+//  * Scores are a 128x32 register-tiled product on the FMA pipe (4 rows x 4 keys per thread,
+//    keys kg, kg+8, kg+16, kg+24, so the 16-byte reads of 8 neighbouring threads fall in 8
+//    different bank groups); an unmarked score is left out of the online softmax.
+//  * P goes through shared memory to the P.V product (4 rows x D/8 columns per thread, columns
+//    4kg + 32c, so 8 neighbouring threads read 128 contiguous bytes of a value row).
+// All arithmetic is fp32 FMA with expf, as the row-per-warp kernel does. A row that stores some
+// column more than once (each copy weighs once, which a bit cannot hold) is recomputed exactly
+// by a row-per-warp pass at the end.
 #include <math.h>
 
 #include "common.cuh"
@@ -29,40 +35,136 @@ namespace {
 constexpr int kRows = 128;                   // query rows per block
 constexpr int kKeys = 32;                    // union keys per tile
 constexpr int kThreads = 256;
-constexpr int kWin = 256;                    // union columns whose per-row counts are held at once
-constexpr int kWinStride = kWin + 16;        // padded row of the counts
+constexpr int kWin = 512;                    // union columns whose row marks are held at once
+constexpr int kWinTiles = kWin / kKeys;
+constexpr int kWinWords = kWin / 32;         // mark words per row
+constexpr int kMaskStride = kWinWords + 1;   // padded row of the marks: a warp's 4 rows, 4 banks apart
 constexpr int kMaxS = 32768;
-constexpr int kPStride = kKeys + 1;          // padded row of P
+constexpr int kPStride = kKeys + 2;          // padded row of P: a warp's 4 rows, 8 banks apart
 
 template <int D>
 struct F32Cfg {
-  static constexpr int kQtOff = 0;                                  // float Qt[D][kRows]
-  static constexpr int kKtOff = kQtOff + D * kRows * 4;             // float Kt[D][kKeys]
-  static constexpr int kVsOff = kKtOff + D * kKeys * 4;             // float Vs[kKeys][D]
-  static constexpr int kPsOff = kVsOff + kKeys * D * 4;             // float Ps[kRows][kPStride]
-  static constexpr int kBitmapOff = kPsOff + kRows * kPStride * 4;
+  static constexpr int kKStride = D + 4;  // floats per staged key row (16-byte groups: key k -> k mod 8)
+  static constexpr int kQsOff = 0;                                    // float Qs[kRows][D], scaled
+  static constexpr int kKsOff = kQsOff + kRows * D * 4;               // float Ks[2][kKeys][kKStride]
+  static constexpr int kVsOff = kKsOff + 2 * kKeys * kKStride * 4;    // float Vs[2][kKeys][D]
+  static constexpr int kPsOff = kVsOff + 2 * kKeys * D * 4;           // float Ps[kRows][kPStride]
+  static constexpr int kMaskOff = kPsOff + kRows * kPStride * 4;      // uint32 marks[kRows][kMaskStride]
+  static constexpr int kKcolOff = kMaskOff + kRows * kMaskStride * 4; // int kcol[kWin]
+  static constexpr int kBitmapOff = kKcolOff + kWin * 4;
   static constexpr int kPrefixOff = kBitmapOff + kMaxS / 8;
-  static constexpr int kBytesOff = kPrefixOff + kMaxS / 8;
-  static constexpr int kBytesSize = kMaxS > kRows * kWinStride ? kMaxS : kRows * kWinStride;
-  static constexpr int kColOff = kBytesOff + kBytesSize;
-  static constexpr int kRowOff = kColOff + kKeys * 4;               // c0, c1, bad, heavy per row
+  static constexpr int kRowOff = kPrefixOff + kMaxS / 8;              // c0, c1, bad, heavy per row
   static constexpr int kMiscOff = kRowOff + 4 * kRows * 4;
   static constexpr int kSmemBytes = kMiscOff + 16;
+  // the union's byte per column lives in the K/V buffers until the union is packed
+  static_assert(kPsOff - kKsOff >= kMaxS, "the union's column bytes fit the K/V buffers");
   static_assert(kSmemBytes <= 232448, "227 KB of shared memory per block");
+  static_assert(D != 64 || kSmemBytes <= 112 * 1024, "two blocks per SM at D = 64");
 };
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool valid) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(valid ? 16 : 0)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+// Starts the copies of the key and value rows of kcol[0 .. nk) into one buffer pair (key row k
+// at ks + k * kKStride floats, value row k at vs + k * D floats); rows nk .. kKeys-1 are zeroed.
+template <int D>
+__device__ __forceinline__ void stage_tile(uint32_t ks, uint32_t vs, const int* kcol, int nk, const float* Kb,
+                                           const float* Vb) {
+  constexpr int kChunks = D / 4;  // 16-byte chunks per row
+  for (int x = threadIdx.x; x < kKeys * kChunks; x += kThreads) {
+    const int k = x / kChunks, c = x % kChunks;
+    const bool valid = k < nk;
+    const int64_t col = valid ? kcol[k] : 0;  // row 0 is a readable address for a zero fill
+    cp_async16(ks + (uint32_t)(k * F32Cfg<D>::kKStride + 4 * c) * 4u, Kb + col * D + 4 * c, valid);
+    cp_async16(vs + (uint32_t)(k * D + 4 * c) * 4u, Vb + col * D + 4 * c, valid);
+  }
+}
+
+// Marks for rows of the block: bit u - W0 of row x's words is set when row x stores union column
+// u (W0 <= u < W0 + kWin). Thread x < kRows does row x; a column stored twice marks the row heavy.
+__device__ __forceinline__ void build_marks(uint32_t* marks, const CsrUnion& un, int* row_heavy,
+                                            const int32_t* cols, int S, int W0) {
+  const int x = threadIdx.x;
+  if (x >= kRows) return;
+  uint32_t* mrow = marks + x * kMaskStride;
+#pragma unroll
+  for (int w = 0; w < kWinWords; ++w) mrow[w] = 0u;
+  bool dup = false;
+  int cur_w = -1;     // the mark word being gathered in registers
+  uint32_t cur = 0u;  // its bits so far
+  const int e1 = un.row_c1[x];
+  for (int e0 = un.row_c0[x]; e0 < e1; e0 += kUnionBatch) {
+    int uu[kUnionBatch];
+#pragma unroll
+    for (int b = 0; b < kUnionBatch; ++b) uu[b] = e0 + b < e1 ? __ldg(cols + e0 + b) : -1;
+#pragma unroll
+    for (int b = 0; b < kUnionBatch; ++b) {
+      const int j = uu[b];  // bad columns are already flagged; the row is zeroed
+      uu[b] = (j >= 0 && j < S) ? csr_union_index(un.bitmap, un.wpre, j) - W0 : -1;
+    }
+#pragma unroll
+    for (int b = 0; b < kUnionBatch; ++b) {
+      const int u = uu[b];
+      if (u >= 0 && u < kWin) {
+        const int w = u >> 5;
+        const uint32_t bit = 1u << (u & 31);
+        if (w != cur_w) {
+          if (cur_w >= 0) {
+            const uint32_t old = mrow[cur_w];
+            dup |= (old & cur) != 0u;
+            mrow[cur_w] = old | cur;
+          }
+          cur_w = w;
+          cur = 0u;
+        }
+        dup |= (cur & bit) != 0u;
+        cur |= bit;
+      }
+    }
+  }
+  if (cur_w >= 0) {
+    const uint32_t old = mrow[cur_w];
+    dup |= (old & cur) != 0u;
+    mrow[cur_w] = old | cur;
+  }
+  if (dup) row_heavy[x] = 1;
+}
+
+// kcol[u - W0] = the column of union index u, for W0 <= u < min(U, W0 + kWin): a thread per
+// bitmap word walks its set bits.
+__device__ __forceinline__ void list_window_columns(int* kcol, const CsrUnion& un, int nw, int W0) {
+  for (int w = threadIdx.x; w < nw; w += kThreads) {
+    uint32_t bits = un.bitmap[w];
+    int u = (int)un.wpre[w];
+    if (u >= W0 + kWin || u + __popc(bits) <= W0) continue;
+    while (bits != 0u) {
+      const int pos = __ffs(bits) - 1;
+      bits &= bits - 1u;
+      if (u >= W0 && u < W0 + kWin) kcol[u - W0] = w * 32 + pos;
+      ++u;
+    }
+  }
+}
 
 template <int D>
 __global__ void __launch_bounds__(kThreads, D == 64 ? 2 : 1) csr_f32_tiled_kernel(CsrArgs a) {
   using C = F32Cfg<D>;
   extern __shared__ __align__(16) uint8_t smem[];
-  float* Qt = reinterpret_cast<float*>(smem + C::kQtOff);
-  float* Kt = reinterpret_cast<float*>(smem + C::kKtOff);
+  float* Qs = reinterpret_cast<float*>(smem + C::kQsOff);
+  float* Ks = reinterpret_cast<float*>(smem + C::kKsOff);
   float* Vs = reinterpret_cast<float*>(smem + C::kVsOff);
   float* Ps = reinterpret_cast<float*>(smem + C::kPsOff);
+  uint32_t* marks = reinterpret_cast<uint32_t*>(smem + C::kMaskOff);
+  int* kcol = reinterpret_cast<int*>(smem + C::kKcolOff);
   uint32_t* bitmap = reinterpret_cast<uint32_t*>(smem + C::kBitmapOff);
   uint32_t* wpre = reinterpret_cast<uint32_t*>(smem + C::kPrefixOff);
-  uint8_t* bytes = smem + C::kBytesOff;
-  int* kcol = reinterpret_cast<int*>(smem + C::kColOff);
+  uint8_t* bytes = smem + C::kKsOff;  // the union's byte per column, before any K/V row lands
   int* row_c0 = reinterpret_cast<int*>(smem + C::kRowOff);
   int* row_c1 = row_c0 + kRows;
   int* row_bad = row_c1 + kRows;
@@ -92,111 +194,81 @@ __global__ void __launch_bounds__(kThreads, D == 64 ? 2 : 1) csr_f32_tiled_kerne
   const int U = csr_block_union<kThreads, kRows>(un, off, cols, S, r0, a.nnz_cap, a.cols_vec, a.status);
   const int T = (U + kKeys - 1) / kKeys;
 
-  // Q, transposed and scaled: Qt[d][r] = q[r0 + r][d] / sqrt(D); rows past S are zero
+  // Q, scaled: Qs[r][d] = q[r0 + r][d] / sqrt(D); rows past S are zero
   for (int x = tid; x < kRows * (D / 4); x += kThreads) {
-    const int rr = x % kRows, c4 = x / kRows;
+    const int rr = x / (D / 4), c4 = x % (D / 4);
     float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
     if (r0 + rr < S) v = __ldg(reinterpret_cast<const float4*>(Qb + (int64_t)(r0 + rr) * D) + c4);
-    Qt[(4 * c4 + 0) * kRows + rr] = v.x * scale;
-    Qt[(4 * c4 + 1) * kRows + rr] = v.y * scale;
-    Qt[(4 * c4 + 2) * kRows + rr] = v.z * scale;
-    Qt[(4 * c4 + 3) * kRows + rr] = v.w * scale;
+    reinterpret_cast<float4*>(Qs + rr * D)[c4] = make_float4(v.x * scale, v.y * scale, v.z * scale, v.w * scale);
   }
 
   const int rg = tid >> 3;  // rows 4rg .. 4rg+3
-  const int kg = tid & 7;   // keys 4kg .. 4kg+3 of a tile; columns kg*D/8 .. of the output
-  constexpr int kCols = D / 8;
-  float m[4], l[4], o[4][kCols];
+  const int kg = tid & 7;   // keys kg + 8j of a tile; output columns 4kg + 32c .. +3
+  constexpr int kV4 = D / 32;
+  constexpr uint32_t kKsBuf = kKeys * C::kKStride * 4, kVsBuf = kKeys * D * 4;
+  const uint32_t ks0 = smem_addr(Ks), vs0 = smem_addr(Vs);
+  float m[4], l[4], o[4][kV4 * 4];
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     m[i] = -INFINITY;
     l[i] = 0.f;
 #pragma unroll
-    for (int c = 0; c < kCols; ++c) o[i][c] = 0.f;
+    for (int c = 0; c < kV4 * 4; ++c) o[i][c] = 0.f;
   }
 
+  int W0 = 0;
   for (int t = 0; t < T; ++t) {
-    if ((t * kKeys) % kWin == 0) {
-      // each row's counts for union columns [t*32, t*32 + kWin), built by the row's thread
+    const int b = t & 1;
+    if (t % kWinTiles == 0) {
+      __syncthreads();  // the last window's marks, columns and buffers are read no more
+      W0 = t * kKeys;
+      build_marks(marks, un, row_heavy, cols, S, W0);
+      list_window_columns(kcol, un, nw, W0);
       __syncthreads();
-      if (tid < kRows) {
-        const int base = t * kKeys;
-        uint8_t* row = bytes + tid * kWinStride;
-#pragma unroll
-        for (int x = 0; x < kWin / 16; ++x) reinterpret_cast<uint4*>(row)[x] = make_uint4(0u, 0u, 0u, 0u);
-        const int e1 = row_c1[tid];
-        for (int e0 = row_c0[tid]; e0 < e1; e0 += kUnionBatch) {
-          int jj[kUnionBatch];
-#pragma unroll
-          for (int b = 0; b < kUnionBatch; ++b) jj[b] = e0 + b < e1 ? __ldg(cols + e0 + b) : -1;
-#pragma unroll
-          for (int b = 0; b < kUnionBatch; ++b) {
-            const int j = jj[b];
-            if (j >= 0 && j < S) {  // bad columns are already flagged; the row is zeroed
-              const int u = csr_union_index(bitmap, wpre, j);
-              if (u >= base && u < base + kWin) {
-                const uint8_t c = row[u - base];
-                if (c == 255) row_heavy[tid] = 1;
-                else row[u - base] = (uint8_t)(c + 1);
-              }
-            }
-          }
-        }
-      }
-      __syncthreads();
+      stage_tile<D>(ks0 + b * kKsBuf, vs0 + b * kVsBuf, kcol, min(kKeys, U - W0), Kb, Vb);
     }
-    // the tile's union columns, then their key rows (transposed) and value rows
-    if (warp == 0) {
-      const int u = t * kKeys + lane;
-      kcol[lane] = u < U ? csr_union_col(bitmap, wpre, nw, u) : -1;
-    }
-    __syncthreads();
-    // key rows: lane = key, so the transposed stores of a warp fall in 32 different banks
-    for (int x = tid; x < kKeys * (D / 4); x += kThreads) {
-      const int k = x % kKeys, c4 = x / kKeys, col = kcol[k];
-      float4 kv = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (col >= 0) kv = __ldg(reinterpret_cast<const float4*>(Kb + (int64_t)col * D) + c4);
-      Kt[(4 * c4 + 0) * kKeys + k] = kv.x;
-      Kt[(4 * c4 + 1) * kKeys + k] = kv.y;
-      Kt[(4 * c4 + 2) * kKeys + k] = kv.z;
-      Kt[(4 * c4 + 3) * kKeys + k] = kv.w;
-    }
-    // value rows: lanes along the row, so every row is one contiguous 16-byte-per-lane store
-    for (int x = tid; x < kKeys * (D / 4); x += kThreads) {
-      const int k = x / (D / 4), c4 = x % (D / 4), col = kcol[k];
-      float4 vv = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (col >= 0) vv = __ldg(reinterpret_cast<const float4*>(Vb + (int64_t)col * D) + c4);
-      reinterpret_cast<float4*>(Vs + k * D)[c4] = vv;
-    }
-    __syncthreads();
+    cp_async_wait_all();
+    __syncthreads();  // tile t has landed for every thread; tile t-1's reads of P and V are done
+    if (t + 1 < T && (t + 1) % kWinTiles != 0)
+      stage_tile<D>(ks0 + (b ^ 1) * kKsBuf, vs0 + (b ^ 1) * kVsBuf, kcol + (t + 1) * kKeys - W0,
+                    min(kKeys, U - (t + 1) * kKeys), Kb, Vb);
+    const float* Kt = Ks + b * (kKeys * C::kKStride);
+    const float* Vt = Vs + b * (kKeys * D);
 
-    // scores of rows 4rg.. against keys 4kg..
+    // scores of rows 4rg.. against keys kg + 8j
     float sc[4][4];
 #pragma unroll
     for (int i = 0; i < 4; ++i)
 #pragma unroll
       for (int j = 0; j < 4; ++j) sc[i][j] = 0.f;
-#pragma unroll 8
-    for (int d = 0; d < D; ++d) {
-      const float4 qa = *reinterpret_cast<const float4*>(Qt + d * kRows + 4 * rg);
-      const float4 kb = *reinterpret_cast<const float4*>(Kt + d * kKeys + 4 * kg);
-      const float qv[4] = {qa.x, qa.y, qa.z, qa.w}, kvv[4] = {kb.x, kb.y, kb.z, kb.w};
+#pragma unroll 4
+    for (int d = 0; d < D; d += 4) {
+      float4 kk[4];
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
+      for (int j = 0; j < 4; ++j) kk[j] = *reinterpret_cast<const float4*>(Kt + (kg + 8 * j) * C::kKStride + d);
 #pragma unroll
-        for (int j = 0; j < 4; ++j) sc[i][j] = fmaf(qv[i], kvv[j], sc[i][j]);
+      for (int i = 0; i < 4; ++i) {
+        const float4 qq = *reinterpret_cast<const float4*>(Qs + (4 * rg + i) * D + d);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          sc[i][j] = fmaf(qq.x, kk[j].x, sc[i][j]);
+          sc[i][j] = fmaf(qq.y, kk[j].y, sc[i][j]);
+          sc[i][j] = fmaf(qq.z, kk[j].z, sc[i][j]);
+          sc[i][j] = fmaf(qq.w, kk[j].w, sc[i][j]);
+        }
+      }
     }
-    // online softmax per row over the 8 lanes that share it
+    // online softmax per row over the 8 threads that share it
     float corr[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const uint32_t cw = *reinterpret_cast<const uint32_t*>(bytes + (4 * rg + i) * kWinStride +
-                                                            (t * kKeys) % kWin + 4 * kg);
-      float cnt[4], tmax = -INFINITY;
+      const uint32_t mw = marks[(4 * rg + i) * kMaskStride + t % kWinTiles] >> kg;
+      bool has[4];
+      float tmax = -INFINITY;
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        cnt[j] = (float)((cw >> (8 * j)) & 0xffu);
-        if (cnt[j] > 0.f) tmax = fmaxf(tmax, sc[i][j]);
+        has[j] = ((mw >> (8 * j)) & 1u) != 0u;
+        if (has[j]) tmax = fmaxf(tmax, sc[i][j]);
       }
 #pragma unroll
       for (int x = 1; x < 8; x <<= 1) tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, x));
@@ -207,7 +279,7 @@ __global__ void __launch_bounds__(kThreads, D == 64 ? 2 : 1) csr_f32_tiled_kerne
         corr[i] = m[i] == -INFINITY ? 0.f : expf(m[i] - mnew);
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          p[j] = cnt[j] > 0.f ? cnt[j] * expf(sc[i][j] - mnew) : 0.f;
+          p[j] = has[j] ? expf(sc[i][j] - mnew) : 0.f;
           rs += p[j];
         }
       }
@@ -216,32 +288,31 @@ __global__ void __launch_bounds__(kThreads, D == 64 ? 2 : 1) csr_f32_tiled_kerne
       l[i] = l[i] * corr[i] + rs;
       m[i] = mnew;
 #pragma unroll
-      for (int j = 0; j < 4; ++j) Ps[(4 * rg + i) * kPStride + 4 * kg + j] = p[j];
+      for (int j = 0; j < 4; ++j) Ps[(4 * rg + i) * kPStride + kg + 8 * j] = p[j];
     }
     __syncthreads();
-    // O = O * corr + P V for rows 4rg.. and columns kg*D/8 ..
+    // O = O * corr + P V for rows 4rg.. and columns 4kg + 32c ..
 #pragma unroll
     for (int i = 0; i < 4; ++i)
 #pragma unroll
-      for (int c = 0; c < kCols; ++c) o[i][c] *= corr[i];
+      for (int c = 0; c < kV4 * 4; ++c) o[i][c] *= corr[i];
 #pragma unroll 4
     for (int k = 0; k < kKeys; ++k) {
       float pk[4];
 #pragma unroll
       for (int i = 0; i < 4; ++i) pk[i] = Ps[(4 * rg + i) * kPStride + k];
 #pragma unroll
-      for (int c4 = 0; c4 < kCols / 4; ++c4) {
-        const float4 vv = reinterpret_cast<const float4*>(Vs + k * D + kg * kCols)[c4];
+      for (int c = 0; c < kV4; ++c) {
+        const float4 vv = *reinterpret_cast<const float4*>(Vt + k * D + 4 * kg + 32 * c);
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          o[i][4 * c4 + 0] = fmaf(pk[i], vv.x, o[i][4 * c4 + 0]);
-          o[i][4 * c4 + 1] = fmaf(pk[i], vv.y, o[i][4 * c4 + 1]);
-          o[i][4 * c4 + 2] = fmaf(pk[i], vv.z, o[i][4 * c4 + 2]);
-          o[i][4 * c4 + 3] = fmaf(pk[i], vv.w, o[i][4 * c4 + 3]);
+          o[i][4 * c + 0] = fmaf(pk[i], vv.x, o[i][4 * c + 0]);
+          o[i][4 * c + 1] = fmaf(pk[i], vv.y, o[i][4 * c + 1]);
+          o[i][4 * c + 2] = fmaf(pk[i], vv.z, o[i][4 * c + 2]);
+          o[i][4 * c + 3] = fmaf(pk[i], vv.w, o[i][4 * c + 3]);
         }
       }
     }
-    __syncthreads();  // the next tile overwrites Kt, Vs and Ps
   }
   __syncthreads();
 
@@ -251,14 +322,14 @@ __global__ void __launch_bounds__(kThreads, D == 64 ? 2 : 1) csr_f32_tiled_kerne
     const int rr = 4 * rg + i, ii = r0 + rr;
     if (ii >= S || row_heavy[rr]) continue;
     const float f = (row_bad[rr] == 0 && l[i] > 0.f) ? 1.f / l[i] : 0.f;
-    float* dst = a.out + (bh * (int64_t)S + ii) * D + kg * kCols;
+    float* dst = a.out + (bh * (int64_t)S + ii) * D + 4 * kg;
 #pragma unroll
-    for (int c4 = 0; c4 < kCols / 4; ++c4)
-      reinterpret_cast<float4*>(dst)[c4] =
-          make_float4(o[i][4 * c4] * f, o[i][4 * c4 + 1] * f, o[i][4 * c4 + 2] * f, o[i][4 * c4 + 3] * f);
+    for (int c = 0; c < kV4; ++c)
+      reinterpret_cast<float4*>(dst + 32 * c)[0] =
+          make_float4(o[i][4 * c] * f, o[i][4 * c + 1] * f, o[i][4 * c + 2] * f, o[i][4 * c + 3] * f);
   }
 
-  // ---- rows that store a column more than 255 times: a row per warp, entry by entry ----------
+  // ---- rows that store a column more than once: a row per warp, entry by entry ---------------
   for (int rr = warp; rr < kRows; rr += kThreads / 32) {
     if (!row_heavy[rr] || r0 + rr >= S) continue;
     constexpr int kPer = D / 32;  // columns per lane

@@ -33,13 +33,17 @@ def test_paddle_worked_example():
     assert np.max(np.abs(out.numpy() - g["output"].reshape(shape))) <= 1e-6
 
 
-def _random_pattern(rng, B, H, S, max_per_row):
+def _random_pattern(rng, B, H, S, max_per_row, distinct=False):
+    """Random row lengths on [0, max_per_row]; columns unsorted, with repeats unless distinct."""
     offs = np.zeros((B, H, S + 1), np.int32)
     rows = []
     for bh in range(B * H):
         cnt = rng.integers(0, max_per_row + 1, size=S)
         offs.reshape(B * H, S + 1)[bh, 1:] = np.cumsum(cnt)
-        rows.append(rng.integers(0, S, size=int(cnt.sum())))  # unsorted, with repeats
+        if distinct:
+            rows.append(np.concatenate([rng.permutation(S)[:c] for c in cnt]))
+        else:
+            rows.append(rng.integers(0, S, size=int(cnt.sum())))
     cap = max(1, max(len(r) for r in rows))
     cols = np.zeros((B, H, cap), np.int32)
     for bh, r in enumerate(rows):
@@ -101,7 +105,7 @@ def test_bad_columns_report_data_error():
 # ---- the tiled path (D = 64 or 128, 16-byte aligned tensors) and the row-per-warp path ---------
 def test_repeated_columns_count_per_entry_tiled():
     """A column stored c times in a row weighs c times (reading of the row pointer), including
-    a column stored 300 times, past what a byte of the tiled kernel's counts holds."""
+    a column stored 300 times; such rows take the tiled kernel's exact row-per-warp pass."""
     B, H, S, D = 1, 2, 200, 64
     q, k, v = (W.randn((B, H, S, D), 400 + i) for i in range(3))
     rng = np.random.default_rng(3)
@@ -126,8 +130,8 @@ def test_repeated_columns_count_per_entry_tiled():
 
 @pytest.mark.parametrize("D", [64, 128])
 def test_union_wider_than_one_window_tiled(D):
-    """Rows of 150 random columns over 2,560 keys: each 128-row block's union spans about 2,000
-    columns, so the per-row counts are rebuilt window after window."""
+    """Rows of up to 150 random columns (with repeats) over 2,560 keys: each 128-row block's
+    union spans about 2,500 columns, so the per-row marks are rebuilt window after window."""
     rng = np.random.default_rng(D)
     B, H, S = 1, 2, 2560
     q, k, v = (W.randn((B, H, S, D), 500 + i) for i in range(3))
@@ -136,6 +140,36 @@ def test_union_wider_than_one_window_tiled(D):
     assert st == 0
     ref = oracle.sparse_csr(q, k, v, off, cols, B=B, H=H, S=S, D=D)
     G.check_out(out.numpy(), ref, W.F32, "wide union")
+
+
+@pytest.mark.parametrize("D", [64, 128])
+def test_distinct_columns_across_windows_tiled(D):
+    """Rows of up to 200 distinct unsorted columns over 3,000 keys: no row needs the exact pass,
+    every block's union spans six 512-column windows, and the last block and tile are ragged."""
+    rng = np.random.default_rng(700 + D)
+    B, H, S = 1, 2, 3000
+    q, k, v = (W.randn((B, H, S, D), 700 + i) for i in range(3))
+    off, cols = _random_pattern(rng, B, H, S, 200, distinct=True)
+    out, st = _run(q, k, v, off, cols, B, H, S, D)
+    assert st == 0
+    ref = oracle.sparse_csr(q, k, v, off, cols, B=B, H=H, S=S, D=D)
+    G.check_out(out.numpy(), ref, W.F32, "distinct, six windows")
+
+
+@pytest.mark.parametrize("U", [511, 512, 513, 544])
+def test_union_at_the_window_edge_tiled(U):
+    """Every row stores the same U distinct columns (reversed), so each block's union is exactly
+    U columns: one window short of, at, and just past 512 union columns."""
+    B, H, S, D = 1, 1, 1100, 64
+    q, k, v = (W.randn((B, H, S, D), 800 + i) for i in range(3))
+    row = (np.arange(U, dtype=np.int64) * 2 + 1)[::-1]  # U distinct odd columns, all below S
+    assert np.unique(row).size == U
+    off = (np.arange(S + 1, dtype=np.int64) * U).astype(np.int32).reshape(1, 1, -1)
+    cols = np.tile(row.astype(np.int32), S).reshape(1, 1, -1)
+    out, st = _run(q, k, v, off, cols, B, H, S, D)
+    assert st == 0
+    ref = oracle.sparse_csr(q, k, v, off, cols, B=B, H=H, S=S, D=D)
+    G.check_out(out.numpy(), ref, W.F32, f"union of {U}")
 
 
 def test_row_per_warp_path_on_misaligned_tensors():
