@@ -10,7 +10,8 @@
 // are gathered once into shared memory and serve all 128 rows, instead of every row gathering
 // its own ~300 key/value rows through L1/L2 (which bounds the row-per-warp kernel).
 //  * The gathers are cp.async copies into two buffers: tile t+1's rows are in flight while
-//    tile t is multiplied, and a tile costs two block barriers.
+//    tile t is multiplied, and a tile costs one block barrier (the P rows a thread's softmax
+//    writes are read back only by the 8 lanes of its own warp that share those rows).
 //  * For each window of 512 union columns, every row's thread marks which of them its row
 //    stores (a bit per row and union column) from its own column list, merging runs of
 //    neighbouring columns in registers. The window's union columns are listed once, a thread
@@ -228,7 +229,7 @@ __global__ void __launch_bounds__(kThreads, D == 64 ? 2 : 1) csr_f32_tiled_kerne
       stage_tile<D>(ks0 + b * kKsBuf, vs0 + b * kVsBuf, kcol, min(kKeys, U - W0), Kb, Vb);
     }
     cp_async_wait_all();
-    __syncthreads();  // tile t has landed for every thread; tile t-1's reads of P and V are done
+    __syncthreads();  // tile t has landed for every thread; tile t-1's reads of K, V and P are done
     if (t + 1 < T && (t + 1) % kWinTiles != 0)
       stage_tile<D>(ks0 + (b ^ 1) * kKsBuf, vs0 + (b ^ 1) * kVsBuf, kcol + (t + 1) * kKeys - W0,
                     min(kKeys, U - (t + 1) * kKeys), Kb, Vb);
@@ -290,7 +291,7 @@ __global__ void __launch_bounds__(kThreads, D == 64 ? 2 : 1) csr_f32_tiled_kerne
 #pragma unroll
       for (int j = 0; j < 4; ++j) Ps[(4 * rg + i) * kPStride + kg + 8 * j] = p[j];
     }
-    __syncthreads();
+    __syncwarp();  // rows 4rg.. of P are written and read by the same 8 lanes of this warp
     // O = O * corr + P V for rows 4rg.. and columns 4kg + 32c ..
 #pragma unroll
     for (int i = 0; i < 4; ++i)

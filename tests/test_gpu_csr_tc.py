@@ -83,6 +83,36 @@ def test_union_wider_than_one_pass():
     _check(*_inputs(B, H, S, D, BF, 5), off, cols, B, H, S, D)
 
 
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("aligned", [True, False], ids=["cols16", "cols_unaligned"])
+def test_narrow_union_marked_in_one_pass(D, aligned):
+    """A +-24 window plus every 100th column: each block's union (about 180 columns) fits one
+    mark window at both head sizes. The union is taken with 16-byte loads of the column array
+    or, from an array that starts 4 bytes off a 16-byte boundary, one index at a time. Some
+    rows are empty and the last block is ragged."""
+    B, H, S = 1, 2, 777
+    offs, c = W.window_stride_pattern(S, half_window=24, stride=100)
+    cnt = np.diff(offs)
+    cnt[::11] = 0                                      # empty every 11th row
+    keep = np.concatenate([np.arange(offs[i], offs[i + 1]) for i in range(S) if cnt[i]])
+    offs = np.concatenate([[0], np.cumsum(cnt)]).astype(np.int32)
+    c = c[keep]
+    off = np.broadcast_to(offs, (B, H, S + 1)).copy()
+    cols = np.broadcast_to(c, (B, H, c.shape[0])).copy()
+    q, k, v = _inputs(B, H, S, D, BF, 40 + D)
+    ref = oracle.sparse_csr(q, k, v, off, cols, B=B, H=H, S=S, D=D)
+    dq, dk, dv = (x.cuda() for x in (q, k, v))
+    doff = torch.from_numpy(off).cuda()
+    buf = torch.zeros(cols.size + 1, dtype=torch.int32, device="cuda")
+    dcol = (buf[:-1] if aligned else buf[1:]).view(cols.shape)
+    dcol.copy_(torch.from_numpy(cols))
+    out = torch.full_like(dq, float("nan"))
+    sdpa.attn_sparse_csr_tc(dq, dk, dv, doff, dcol, B=B, H=H, S=S, D=D, nnz_cap=cols.shape[-1],
+                            dtype=sdpa.ATTN_BF16, out=out)
+    assert sdpa.attn_get_last_error() == 0
+    G.check_out(G.f64(out.cpu()), ref, W.BF16, "one-pass marks")
+
+
 def test_full_pattern_equals_dense():
     B, H, S, D = 1, 2, 200, 128
     q, k, v = _inputs(B, H, S, D, BF, 9)
