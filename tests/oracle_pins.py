@@ -106,6 +106,28 @@ def pin_csr_single_and_empty_rows():
     assert np.max(np.abs(out[0, 0, 3] - (p[0] * v[0, 0, 0] + p[1] * v[0, 0, 1]))) <= 1e-14
 
 
+def pin_csr_repeated_columns_weigh_per_entry():
+    """A column stored c times in a row weighs c times (the row pointer counts entries): each
+    row equals torch's float64 attention of its query over the key/value rows gathered entry
+    by entry, repeats included."""
+    r = _rng(31)
+    B, H, S, D = 1, 1, 6, 4
+    q, k, v = (r.standard_normal((B, H, S, D)) for _ in range(3))
+    rows = [[1, 4, 1], [2, 2, 2, 5], [0, 3, 0, 3, 3], [5], [], [4, 0, 4, 0, 1, 4]]
+    off = np.concatenate([[0], np.cumsum([len(x) for x in rows])]).astype(np.int32).reshape(1, 1, -1)
+    cols = np.concatenate([np.array(x, np.int32) for x in rows]).reshape(1, 1, -1)
+    out = oracle.sparse_csr(q, k, v, off, cols, B=B, H=H, S=S, D=D)
+    for i, row in enumerate(rows):
+        if not row:
+            assert np.all(out[0, 0, i] == 0.0)
+            continue
+        kk = torch.from_numpy(k[0, 0, row]).view(1, 1, len(row), D)
+        vv = torch.from_numpy(v[0, 0, row]).view(1, 1, len(row), D)
+        qq = torch.from_numpy(q[0, 0, i:i + 1]).view(1, 1, 1, D)
+        ref = torch.nn.functional.scaled_dot_product_attention(qq, kk, vv).view(D).numpy()
+        assert np.max(np.abs(out[0, 0, i] - ref)) <= 1e-13
+
+
 def pin_csr_heads_independent():
     """Each (b, h) slice uses its own row pointer and columns."""
     r = _rng(4)

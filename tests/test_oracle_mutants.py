@@ -33,6 +33,9 @@ MUTANTS = [
     ("csr_first_slice_only", "base = bhi * (int64_t)S * D;", "base = 0;", 0),
     ("csr_query_transposed", "ld(q, rowq + d, et) * ld(k, base + j * D + d, et)",
      "ld(q, base + j * D + d, et) * ld(k, rowq + d, et)", 0),
+    ("csr_repeats_counted_once", "s[c - c0] = exp(s[c - c0] - mx);",
+     "{ int64_t cc; int seen = 0; for (cc = c0; cc < c; ++cc) seen |= cp[cc] == cp[c];"
+     " s[c - c0] = seen ? 0.0 : exp(s[c - c0] - mx); }", 0),
     ("csr_normalisation_dropped", "for (d = 0; d < D; ++d) o[d] /= sum;\n    }\n    free(s);",
      "for (d = 0; d < D; ++d) o[d] /= 1.0;\n    }\n    free(s);", 0),
     ("merge_exp_sign", "prev_sum[x] * exp(pm - m)", "prev_sum[x] * exp(m - pm)", 0),
