@@ -53,6 +53,12 @@ MUTANTS = [
     ("mask_row_stride_ignored", "mask[mrow + i * mask_rstride + j]", "mask[mrow + i * sk + j]", 0),
     ("mask_batch_stride_ignored", "b * mask_bstride, mask_rstride))", "0 * mask_bstride, mask_rstride))", 0),
     ("mask_key_shifted", "mask[mrow + i * mask_rstride + j]", "mask[mrow + i * mask_rstride + (j + 1) % sk]", 0),
+    ("ext_dropped_scale", "s[j] = scale * acc;", "s[j] = acc;", 1),
+    ("ext_max_not_subtracted", "s[j] == -INFINITY ? 0.0 : exp(s[j] - mx);", "s[j] == -INFINITY ? 0.0 : exp(s[j]);", 0),
+    ("ext_normalisation_dropped", "for (d = 0; d < Dv; ++d) o[d] /= sum;", "for (d = 0; d < Dv; ++d) o[d] /= 1.0;", 0),
+    ("empty_row_max_zero", "    *m = -INFINITY;\n    *l = 0.0;\n    return;", "    *m = 0.0;\n    *l = 0.0;\n    return;", 0),
+    ("ext_empty_row_max_zero", "    *m = -INFINITY;\n    *l = 0.0;\n    return;", "    *m = 0.0;\n    *l = 0.0;\n    return;", 1),
+    ("merge_max_is_min", "double m = pm > cm ? pm : cm;", "double m = pm < cm ? pm : cm;", 0),
     ("scores_over_value_dims", "for (d = 0; d < Dqk; ++d)\n      acc +=", "for (d = 0; d < Dv; ++d)\n      acc +=", 0),
 ]
 
