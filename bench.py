@@ -558,7 +558,7 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--max-len", type=int, default=8192, help="max sequence length of the varlen batch")
     ap.add_argument("--parts", default="fwd,csr,merge", help="operations in a step (fwd always runs)")
-    ap.add_argument("--e2e-steps", type=int, default=6)
+    ap.add_argument("--e2e-steps", type=int, default=24)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-next-rows", action="store_true",
                     help="skip timing the ring fold, the band and the tensor-core CSR")
