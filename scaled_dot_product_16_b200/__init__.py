@@ -1,8 +1,9 @@
 """Python binding of libattn.so: scaled-dot-product attention forward on B200 (sm_100a).
 
-The three operations are the C-ABI calls declared in ``include/attn.h``; the functions here
-carry the same names and only marshal arguments (tensor data pointers, sizes, the current
-CUDA stream) into them. Every step of the computation runs in the library's CUDA kernels.
+The operations (attn_fwd, attn_fwd_masked, attn_fwd_accumulate, attn_sparse_csr,
+attn_sparse_csr_tc, attn_merge, attn_get_last_error) are the C-ABI calls declared in
+``include/attn.h``; the functions here carry the same names and only marshal arguments (tensor
+data pointers, sizes, the current CUDA stream) into them. Every step of the computation runs in the library's CUDA kernels.
 There is no CPU path: if ``libattn.so`` is missing the first call raises.
 
 PyTorch is used for device memory and streams only: pass CUDA tensors (contiguous, in the
