@@ -345,11 +345,17 @@ def time_oracle(inp: W.AttnInputs, n_rows: int, seed: int):
 
 
 def oracle_threads() -> int:
-    return int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    """Gives the oracle every core this process may run on and returns that count. Only rank 0
+    runs the oracle (the other ranks do no CPU work), while a launcher such as torchrun sets
+    OMP_NUM_THREADS=1 for every rank; the oracle's OpenMP loops run in torch's OpenMP runtime,
+    so torch.set_num_threads sets their width."""
+    torch.set_num_threads(len(os.sched_getaffinity(0)))
+    return torch.get_num_threads()
 
 
 def cpu_baseline(inp: W.AttnInputs, budget_s: float = 20.0) -> dict:
     """The oracle as it stands on this host's cores, on a bounded row sample of the workload."""
+    cores = oracle_threads()
     n = 64
     flops, dt = time_oracle(inp, n, 1234)
     while dt < 1.0 and n < 1 << 20:  # calibrate on growing samples
@@ -357,7 +363,7 @@ def cpu_baseline(inp: W.AttnInputs, budget_s: float = 20.0) -> dict:
         flops, dt = time_oracle(inp, n, 1234)
     n = max(n, int(n * budget_s / dt))  # then one sample sized to about the budget
     flops, dt = time_oracle(inp, n, 4321)
-    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": oracle_threads(), "kind": "oracle",
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
             "sample": f"{n} random (head, query-token) rows of the varlen batch, all their visible keys; "
                       f"{flops / 1e9:.1f} GFLOP in {dt:.1f} s"}
 
@@ -376,6 +382,7 @@ def run_reference(args, rank: int, world: int):
         return
     inp = W.cfg3_varlen_gqa(seed=0, max_len=args.max_len)
     rows = args.ref_rows
+    cores = oracle_threads()
     for s in range(args.warmup):
         time_oracle(inp, max(8, rows // 8), 100 + s)
     fl, dt = 0, 0.0
@@ -388,7 +395,7 @@ def run_reference(args, rank: int, world: int):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "config": config_dict(inp, world),
-            "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": oracle_threads(), "kind": "oracle",
+            "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
                              "sample": f"{rows} random (head, query-token) rows of the varlen batch per step, all their visible keys"},
             "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
