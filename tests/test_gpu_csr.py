@@ -172,6 +172,36 @@ def test_union_at_the_window_edge_tiled(U):
     G.check_out(out.numpy(), ref, W.F32, f"union of {U}")
 
 
+def _sparse_distinct_pattern(rng, S, max_per_row):
+    """One (b, h) slice: row lengths on [0, max_per_row], distinct random columns per row
+    (drawn with replacement, rows holding a repeat drawn again)."""
+    cnt = rng.integers(0, max_per_row + 1, size=S)
+    rows = []
+    for c in cnt:
+        r = rng.integers(0, S, size=c)
+        while np.unique(r).size != c:
+            r = rng.integers(0, S, size=c)
+        rows.append(r)
+    off = np.concatenate([[0], np.cumsum(cnt)]).astype(np.int32).reshape(1, 1, -1)
+    cols = np.concatenate(rows).astype(np.int32).reshape(1, 1, -1)
+    return off, cols
+
+
+@pytest.mark.parametrize("S,D", [(32768, 64), (32767, 64), (32768, 128)])
+def test_longest_sequence_tiled(S, D):
+    """S at the tiled kernel's limit of 32,768 keys: the union's byte per column fills the 32 KB
+    it borrows from the K/V buffers and the bitmap holds 1,024 words; rows of up to 12 distinct
+    random columns, so each block's union (650 to 870 columns) spans two 512-column windows."""
+    rng = np.random.default_rng(S + D)
+    B, H = 1, 1
+    q, k, v = (W.randn((B, H, S, D), 900 + i) for i in range(3))
+    off, cols = _sparse_distinct_pattern(rng, S, 12)
+    out, st = _run(q, k, v, off, cols, B, H, S, D)
+    assert st == 0
+    ref = oracle.sparse_csr(q, k, v, off, cols, B=B, H=H, S=S, D=D)
+    G.check_out(out.numpy(), ref, W.F32, f"S={S}")
+
+
 def test_row_per_warp_path_on_misaligned_tensors():
     """A q view that starts 4 bytes into its buffer is not 16-byte aligned, so the call takes the
     row-per-warp kernel; both paths agree with the oracle on the same data."""

@@ -113,6 +113,24 @@ def test_narrow_union_marked_in_one_pass(D, aligned):
     G.check_out(G.f64(out.cpu()), ref, W.BF16, "one-pass marks")
 
 
+@pytest.mark.parametrize("S,D", [(32768, 64), (32767, 128)])
+def test_longest_sequence(S, D):
+    """S at the limit of 32,768 keys (a byte per column in shared memory while the union is
+    taken); rows of up to 12 distinct random columns, several mark windows per block."""
+    rng = np.random.default_rng(S + D)
+    B, H = 1, 1
+    cnt = rng.integers(0, 13, size=S)
+    rows = []
+    for c in cnt:
+        r = rng.integers(0, S, size=c)
+        while np.unique(r).size != c:
+            r = rng.integers(0, S, size=c)
+        rows.append(r)
+    off = np.concatenate([[0], np.cumsum(cnt)]).astype(np.int32).reshape(1, 1, -1)
+    cols = np.concatenate(rows).astype(np.int32).reshape(1, 1, -1)
+    _check(*_inputs(B, H, S, D, BF, 60 + D), off, cols, B, H, S, D)
+
+
 def test_full_pattern_equals_dense():
     B, H, S, D = 1, 2, 200, 128
     q, k, v = _inputs(B, H, S, D, BF, 9)
