@@ -43,10 +43,9 @@ METRIC = "attn fwd TFLOP/s & % of BF16 tensor peak; attn_merge HBM GB/s & % of p
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one attn_fwd launch on the
-# full varlen workload, from a one-pass ncu capture (profiles/attn_fwd_bf16_varlen.md); it is
-# reported only while the kernel source still has the hash it was measured on.
-# DRAM bytes per attn_fwd launch from an ncu capture, valid only for this kernel source and this
-# workload (the default varlen batch of 75,336 tokens)
+# default varlen batch (75,336 tokens), from a one-pass ncu capture of that launch. It is
+# reported only for that workload and while the kernel source still has the hash it was
+# measured on.
 TRAFFIC = {"kernel_sha": "3612f886071302b1", "tokens": 75_336, "bytes_per_launch": 937_927_936 + 600_918_272}
 
 
