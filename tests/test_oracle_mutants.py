@@ -59,6 +59,18 @@ MUTANTS = [
     ("empty_row_max_zero", "    *m = -INFINITY;\n    *l = 0.0;\n    return;", "    *m = 0.0;\n    *l = 0.0;\n    return;", 0),
     ("ext_empty_row_max_zero", "    *m = -INFINITY;\n    *l = 0.0;\n    return;", "    *m = 0.0;\n    *l = 0.0;\n    return;", 1),
     ("merge_max_is_min", "double m = pm > cm ? pm : cm;", "double m = pm < cm ? pm : cm;", 0),
+    ("kv_range_from_query_sequence", "seq_range(layout, cu_kv, b, Skv, &tk0, &lk);",
+     "seq_range(layout, cu_q, b, Sq, &tk0, &lk);", 0),
+    ("ext_gqa_divides_by_nkv", "h / group, lq, lk,", "h / Nkv, lq, lk,", 0),
+    ("mask_replaces_mode", "  if (mask_mode == ORC_MASK_TOPLEFT && j > i) return 0;",
+     "  if (mask != NULL) return mask[mrow + i * mask_rstride + j] == 0;\n"
+     "  if (mask_mode == ORC_MASK_TOPLEFT && j > i) return 0;", 0),
+    ("band_bottom_right_aligned", "(j < i - pre || j > i + next)",
+     "(j < i + sk - sq - pre || j > i + sk - sq + next)", 0),
+    ("csr_empty_row_divides", "      if (c1 <= c0) continue;\n", "", 0),
+    ("merge_stats_sum_from_lane_0", "out_sum[x] = l[lane];", "out_sum[x] = l[0];", 0),
+    ("merge_cur_scaled_by_prev_max", "cs_scaled[lane] = cur_sum[x] * exp(cm - m);",
+     "cs_scaled[lane] = cur_sum[x] * exp(pm - m);", 0),
     ("scores_over_value_dims", "for (d = 0; d < Dqk; ++d)\n      acc +=", "for (d = 0; d < Dv; ++d)\n      acc +=", 0),
 ]
 
