@@ -3,6 +3,8 @@
 Every case compiles a copy of oracle/attn_oracle.c with one plausible slip (a dropped term, a
 wrong sign, a wrong index, an off-by-one, a transposed operand) into a temporary library and
 runs the whole pin suite against it on the CPU. The built oracle itself is never modified.
+Every slip keeps the oracle's memory accesses inside its buffers, so a mutant fails by value,
+never by corrupting the test process.
 """
 import os
 import subprocess
@@ -20,7 +22,8 @@ MUTANTS = [
     ("dropped_scale", "s[j] = scale * acc;", "s[j] = acc;", 0),
     ("gqa_index_modulo", "h / group, nk, Nq, Nkv, Sq, Skv, D,\n                 scale, s, out + oo",
      "h % Nkv, nk, Nq, Nkv, Sq, Skv, D,\n                 scale, s, out + oo", 0),
-    ("keys_from_query_sequence", "ld(k, offs(layout, b, tk0, j, g, d", "ld(k, offs(layout, b, tq0, j, g, d", 0),
+    ("keys_from_next_sequence", "seq_range(layout, cu_kv, b, Skv, &tk0, &lk);",
+     "seq_range(layout, cu_kv, (b + 1) % B, Skv, &tk0, &lk);", 0),
     ("values_use_key_head_of_query", "ld(v, offs(layout, b, tk0, j, g, d", "ld(v, offs(layout, b, tk0, j, h % Nkv, d", 0),
     ("causal_off_by_one", "return last + 1 < sk ? last + 1 : sk;", "return last < sk ? last : sk;", 0),
     ("bottomright_sign", "i + sk - sq", "i + sq - sk", 0),
@@ -59,9 +62,7 @@ MUTANTS = [
     ("empty_row_max_zero", "    *m = -INFINITY;\n    *l = 0.0;\n    return;", "    *m = 0.0;\n    *l = 0.0;\n    return;", 0),
     ("ext_empty_row_max_zero", "    *m = -INFINITY;\n    *l = 0.0;\n    return;", "    *m = 0.0;\n    *l = 0.0;\n    return;", 1),
     ("merge_max_is_min", "double m = pm > cm ? pm : cm;", "double m = pm < cm ? pm : cm;", 0),
-    ("kv_range_from_query_sequence", "seq_range(layout, cu_kv, b, Skv, &tk0, &lk);",
-     "seq_range(layout, cu_q, b, Sq, &tk0, &lk);", 0),
-    ("ext_gqa_divides_by_nkv", "h / group, lq, lk,", "h / Nkv, lq, lk,", 0),
+    ("ext_gqa_next_head", "h / group, lq, lk,", "(h / group + 1) % Nkv, lq, lk,", 0),
     ("mask_replaces_mode", "  if (mask_mode == ORC_MASK_TOPLEFT && j > i) return 0;",
      "  if (mask != NULL) return mask[mrow + i * mask_rstride + j] == 0;\n"
      "  if (mask_mode == ORC_MASK_TOPLEFT && j > i) return 0;", 0),
