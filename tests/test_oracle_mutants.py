@@ -84,6 +84,7 @@ def _mutate(text, old, new, nth):
     return text[:pos] + new + text[pos + len(old):]
 
 
+@pytest.mark.filterwarnings("ignore::RuntimeWarning")  # a mutant's NaN or inf in the pins' arithmetic
 @pytest.mark.parametrize("name,old,new,nth", MUTANTS, ids=[m[0] for m in MUTANTS])
 def test_planted_mistake_is_caught(name, old, new, nth, tmp_path):
     src = open(SRC).read()
