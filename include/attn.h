@@ -155,9 +155,9 @@ ATTN_API int attn_fwd_accumulate(const void* q, const void* k, const void* v,
  *     [Tq, Nq, Dv]; 1 <= Dv <= Dqk. q and k have head size Dqk.
  * Other arguments, statistics, limits and errors are those of attn_fwd (D there is Dqk).
  * Supported: ATTN_F32 with Dv <= Dqk <= 256; ATTN_BF16 and ATTN_F16 with (Dqk, Dv) =
- * (64, 64), (128, 128) or (128, 64) (other pairs are ATTN_ERR_UNSUPPORTED there). On the tensor-core path a mask given with
- * atten_mask, mask_row_stride and mask_batch_stride all 16-byte aligned is read 16 bytes at a
- * time, otherwise byte by byte.
+ * (64, 64), (128, 128) or (128, 64) (other pairs are ATTN_ERR_UNSUPPORTED there). On the
+ * tensor-core path a mask given with atten_mask, mask_row_stride and mask_batch_stride all
+ * 16-byte aligned is read 16 bytes at a time, otherwise byte by byte.
  * Errors: mask_mode outside 0..3, pre_tokens + next_tokens < 0 with the band, negative
  * strides, Dv outside 1..Dqk, or a BHSD mask_row_stride < Skv give ATTN_ERR_INVALID.
  */
