@@ -655,6 +655,30 @@ def pin_merge_tnd_chunks_equal_full_varlen():
 # ---------------------------------------------------------------------------------------------
 # bf16 rounding
 # ---------------------------------------------------------------------------------------------
+def pin_bf16_inputs_read_exactly():
+    """bf16 inputs (passed to the oracle as raw 16-bit patterns) give bit-for-bit the results of
+    the same values widened to float64 by torch, for the forward, the CSR call and the merge."""
+    g = torch.Generator().manual_seed(77)
+    B, N, S, D = 2, 3, 9, 8
+    q, k, v = (torch.randn((B, N, S, D), generator=g).to(torch.bfloat16) for _ in range(3))
+    args = dict(B=B, Sq=S, Skv=S, Nq=N, Nkv=N, D=D, scale=0.3, mask_mode=W.MASK_CAUSAL_TOPLEFT,
+                layout=W.BHSD)
+    a = oracle.attn_fwd(q, k, v, **args)
+    b = oracle.attn_fwd(q.double(), k.double(), v.double(), **args)
+    assert all(np.array_equal(x, y) for x, y in zip(a, b))
+    off = np.broadcast_to(np.arange(0, 2 * S + 1, 2, dtype=np.int32), (B, N, S + 1)).copy()
+    cols = np.broadcast_to(((np.arange(2 * S) * 5) % S).astype(np.int32), (B, N, 2 * S)).copy()
+    a = oracle.sparse_csr(q, k, v, off, cols, B=B, H=N, S=S, D=D)
+    b = oracle.sparse_csr(q.double(), k.double(), v.double(), off, cols, B=B, H=N, S=S, D=D)
+    assert np.array_equal(a, b)
+    po, co = (torch.randn((S, B, N * D), generator=g).to(torch.bfloat16) for _ in range(2))
+    m1, m2 = (_rep8(torch.randn((B, N, S), generator=g).double().numpy()) for _ in range(2))
+    l1, l2 = (_rep8(1.0 + torch.rand((B, N, S), generator=g).double().numpy()) for _ in range(2))
+    a = oracle.merge(po, m1, l1, co, m2, l2, S=S, B=B, N=N, D=D)
+    b = oracle.merge(po.double(), m1, l1, co.double(), m2, l2, S=S, B=B, N=N, D=D)
+    assert all(np.array_equal(x, y) for x, y in zip(a, b))
+
+
 def pin_round_bf16_matches_torch():
     r = _rng(40)
     x = np.concatenate([

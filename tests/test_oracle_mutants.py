@@ -49,6 +49,8 @@ MUTANTS = [
     ("merge_swapped_sides", "ld(prev_out, x, et) * po + ld(cur_out, x, et) * co",
      "ld(prev_out, x, et) * co + ld(cur_out, x, et) * po", 0),
     ("merge_sum_not_rescaled", "cs_scaled[lane] = cur_sum[x] * exp(cm - m);", "cs_scaled[lane] = cur_sum[x];", 0),
+    ("bf16_decode_unshifted", "uint32_t bits = ((uint32_t)((const uint16_t *)base)[idx]) << 16;",
+     "uint32_t bits = ((uint32_t)((const uint16_t *)base)[idx]);", 0),
     ("bf16_truncates", "nearbyint(m * 256.0)", "floor(m * 256.0)", 0),
     ("band_lower_off_by_one", "(j < i - pre || j > i + next)", "(j <= i - pre || j > i + next)", 0),
     ("band_upper_sign", "(j < i - pre || j > i + next)", "(j < i - pre || j > i - next)", 0),
