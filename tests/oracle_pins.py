@@ -156,6 +156,38 @@ def pin_csr_rejects_bad_columns():
     raise AssertionError("column 2 of a 2-row slice was accepted")
 
 
+def _rejected(call) -> bool:
+    try:
+        call()
+    except ValueError:
+        return True
+    return False
+
+
+def pin_csr_rejects_bad_row_pointers():
+    """The row pointer must start at 0, never decrease and end within nnz_cap (the offset
+    argument read as a row pointer); anything else is refused, never computed."""
+    q = np.zeros((1, 1, 3, 2))
+    cols = np.zeros((1, 1, 4), np.int32)
+    for off in ([1, 2, 3, 4], [0, 3, 2, 4], [0, 1, 2, 5]):
+        o = np.array(off, np.int32).reshape(1, 1, -1)
+        assert _rejected(lambda: oracle.sparse_csr(q, q, q, o, cols, B=1, H=1, S=3, D=2)), off
+    o = np.array([0, 1, 3, 4], np.int32).reshape(1, 1, -1)
+    oracle.sparse_csr(q, q, q, o, cols, B=1, H=1, S=3, D=2)  # the same shapes, well formed
+
+
+def pin_cumulative_lengths_rejected_when_bad():
+    """Cumulative lengths (B entries, no leading zero) must not decrease and must end at the
+    token count; anything else is refused, never computed."""
+    x = np.zeros((10, 2, 4))
+    args = dict(B=3, Sq=10, Skv=10, Nq=2, Nkv=2, D=4, scale=1.0, mask_mode=W.MASK_NONE, layout=W.TND)
+    for cq, ck in (([6, 4, 10], [3, 6, 10]), ([3, 6, 10], [3, 6, 8]), ([3, 6, 9], [3, 6, 10])):
+        assert _rejected(lambda: oracle.attn_fwd(x, x, x, cu_q=np.array(cq, np.int32),
+                                                 cu_kv=np.array(ck, np.int32), **args)), (cq, ck)
+    oracle.attn_fwd(x, x, x, cu_q=np.array([3, 6, 10], np.int32), cu_kv=np.array([2, 2, 10], np.int32),
+                    **args)  # well formed, an empty key sequence included
+
+
 # ---------------------------------------------------------------------------------------------
 # Dense / varlen forward
 # ---------------------------------------------------------------------------------------------

@@ -49,6 +49,10 @@ MUTANTS = [
     ("merge_swapped_sides", "ld(prev_out, x, et) * po + ld(cur_out, x, et) * co",
      "ld(prev_out, x, et) * co + ld(cur_out, x, et) * po", 0),
     ("merge_sum_not_rescaled", "cs_scaled[lane] = cur_sum[x] * exp(cm - m);", "cs_scaled[lane] = cur_sum[x];", 0),
+    ("cu_order_unchecked", "    if (cu[b] < prev) return -2;\n", "", 0),
+    ("cu_total_unchecked", "  if (B > 0 && prev != T) return -2;\n", "", 0),
+    ("csr_rowptr_start_unchecked", "if (op[0] != 0 || op[S] > nnz_cap) return -2;", "if (op[S] > nnz_cap) return -2;", 0),
+    ("csr_rowptr_order_unchecked", "      if (op[r + 1] < op[r]) return -2;\n", "", 0),
     ("bf16_decode_unshifted", "uint32_t bits = ((uint32_t)((const uint16_t *)base)[idx]) << 16;",
      "uint32_t bits = ((uint32_t)((const uint16_t *)base)[idx]);", 0),
     ("bf16_truncates", "nearbyint(m * 256.0)", "floor(m * 256.0)", 0),
