@@ -1,7 +1,7 @@
 /*
  * attn.h -- C ABI of libattn.so: scaled-dot-product attention forward on NVIDIA B200 (sm_100a).
  *
- * Three operations, each a single asynchronous launch on the caller's CUDA stream:
+ * The operations, each an asynchronous launch on the caller's CUDA stream:
  *
  *   attn_fwd         O = softmax(scale * Q K^T + mask) V, with per-row softmax max and sum.
  *   attn_sparse_csr  the same softmax restricted to the entries of a CSR pattern (fp32).
@@ -124,6 +124,8 @@ ATTN_API int attn_fwd(const void* q, const void* k, const void* v,
  * acc_out has the element type `dtype`. first = 1 overwrites the accumulator (all 8 lanes get
  * this chunk's statistics); first = 0 folds into it (it must hold an earlier call's result).
  * Calls that fold into the same accumulator must not overlap on the device.
+ * For ATTN_BF16 and ATTN_F16, acc_out, acc_max and acc_sum must be 16-byte aligned (otherwise
+ * ATTN_ERR_INVALID): a row's 8 statistic lanes are moved as two 16-byte vectors.
  */
 ATTN_API int attn_fwd_accumulate(const void* q, const void* k, const void* v,
                                  const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_kv,
@@ -248,10 +250,14 @@ ATTN_API int attn_merge(const void* prev_out, const float* prev_max, const float
 
 /*
  * attn_get_last_error -- read and clear the calling device's status word.
- * Synchronises `stream`, then returns in *device_status the first device-side error
- * (ATTN_ERR_DATA or ATTN_ERR_TIMEOUT) recorded by any launch on the current device since the
- * previous read, or ATTN_OK. The return value is ATTN_OK, or ATTN_ERR_CUDA if the
- * synchronisation or the read failed. The word is per device, shared by all streams.
+ * Enqueues on `stream` a one-thread kernel that exchanges the word for 0 in one atomic step,
+ * copies the old value back and synchronises `stream`. *device_status is then the first
+ * device-side error (ATTN_ERR_DATA or ATTN_ERR_TIMEOUT) recorded by any launch on the current
+ * device since the previous read, or ATTN_OK. The word is per device, shared by all streams:
+ * every launch that finished before the exchange is covered, and an error that a launch still
+ * running on another stream records later is kept for the next read (none is lost). Calls on
+ * one device are serialised by a host lock. The return value is ATTN_OK, or ATTN_ERR_CUDA if
+ * the launch, the copy or the synchronisation failed.
  */
 ATTN_API int attn_get_last_error(void* stream, int* device_status);
 

@@ -61,6 +61,8 @@ def _bind(path: str):
     lib.oracle_merge.restype = I
     lib.oracle_round_bf16_array.argtypes = [P, I64, P]
     lib.oracle_round_bf16_array.restype = None
+    lib.oracle_round_f16_array.argtypes = [P, I64, P]
+    lib.oracle_round_f16_array.restype = None
     return lib
 
 
@@ -292,6 +294,15 @@ def round_bf16(x) -> np.ndarray:
     xa = np.ascontiguousarray(x, dtype=np.float64)
     out = np.zeros(xa.shape, dtype=np.uint16)
     lib.oracle_round_bf16_array(_ptr(xa), int(xa.size), _ptr(out))
+    return out
+
+
+def round_f16(x) -> np.ndarray:
+    """Round float64 values to IEEE float16 (nearest, ties to even); returns raw uint16 patterns."""
+    lib = _load()
+    xa = np.ascontiguousarray(x, dtype=np.float64)
+    out = np.zeros(xa.shape, dtype=np.uint16)
+    lib.oracle_round_f16_array(_ptr(xa), int(xa.size), _ptr(out))
     return out
 
 

@@ -527,3 +527,34 @@ void oracle_round_bf16_array(const double *x, int64_t n, uint16_t *out) {
 #pragma omp parallel for schedule(static)
   for (i = 0; i < n; ++i) out[i] = oracle_round_bf16(x[i]);
 }
+
+/*
+ * Round a double to IEEE binary16 (11 significant bits, exponents -14 .. 15, subnormal spacing
+ * 2^-24), round to nearest with ties to even, and return the 16-bit pattern. The merge page
+ * lists float16 among its output types and casts the float32 result once to the output type
+ * ("npu_ring_attention_update", 小算子等价计算逻辑: the final .to(origin_dtype)); this is that
+ * cast, done once on the double itself with nearbyint on the integer grid of the value's binade.
+ */
+uint16_t oracle_round_f16(double x) {
+  double a, r, m;
+  int e;
+  uint16_t sign = signbit(x) ? 0x8000 : 0;
+  if (isnan(x)) return 0x7E00;
+  if (isinf(x)) return (uint16_t)(sign | 0x7C00);
+  a = fabs(x);
+  if (a < 0x1p-14) {
+    r = nearbyint(a * 0x1p24); /* subnormal grid; 1024 is the smallest normal, 0x0400 */
+    return (uint16_t)(sign | (uint16_t)r);
+  }
+  m = frexp(a, &e); /* a = m * 2^e, m in [0.5, 1) */
+  r = ldexp(nearbyint(m * 2048.0), e - 11);
+  if (r >= 65536.0) return (uint16_t)(sign | 0x7C00); /* past the largest finite value */
+  m = frexp(r, &e);                                    /* r = 2^(e-1) * (2m), 2m in [1, 2) */
+  return (uint16_t)(sign | (uint16_t)((e - 1 + 15) << 10) | (uint16_t)((2.0 * m - 1.0) * 1024.0));
+}
+
+void oracle_round_f16_array(const double *x, int64_t n, uint16_t *out) {
+  int64_t i;
+#pragma omp parallel for schedule(static)
+  for (i = 0; i < n; ++i) out[i] = oracle_round_f16(x[i]);
+}

@@ -85,18 +85,52 @@ def _status_string(status: int) -> str:
         return "unknown"
 
 
-def _ptr(x) -> Optional[int]:
-    """Device data pointer of a tensor (or an int address, or None). Tensors must be on a CUDA
-    device and dense: the C ABI reads them as contiguous device arrays."""
+_ELEM = {ATTN_BF16: "bfloat16", ATTN_F32: "float32", ATTN_F16: "float16"}
+
+
+def _dtype_name(x) -> str:
+    return str(getattr(x, "dtype", "")).replace("torch.", "")
+
+
+def _ptr(x, name: str = "tensor", numel: int = 0, dtype: Optional[str] = None) -> Optional[int]:
+    """Device data pointer of a tensor argument (an int is passed through as a raw address and
+    None as a null pointer). A tensor must be a dense CUDA tensor on the current device, of
+    element type `dtype` (a torch dtype name) when given, holding at least `numel` elements:
+    the library reads exactly the sizes it is given, so a smaller or differently typed tensor,
+    or one on another GPU, would be read or written out of bounds."""
     if x is None:
         return None
     if isinstance(x, int):
         return x
     if getattr(x, "is_cuda", True) is False:
-        raise ValueError("tensor arguments must be on a CUDA device")
+        raise ValueError(f"{name} must be on a CUDA device")
     if hasattr(x, "is_contiguous") and not x.is_contiguous():
-        raise ValueError("tensor arguments must be contiguous")
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and _dtype_name(x) != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {_dtype_name(x)}")
+    if numel > 0 and x.numel() < numel:
+        raise ValueError(f"{name} holds {x.numel()} elements; the sizes given need {numel}")
+    dev = getattr(x, "device", None)
+    if dev is not None and getattr(dev, "index", None) is not None:
+        import torch
+        cur = torch.cuda.current_device()
+        if dev.index != cur:
+            raise ValueError(f"{name} is on cuda:{dev.index} but the current device is cuda:{cur}")
     return int(x.data_ptr())
+
+
+def _elem(dtype: int) -> Optional[str]:
+    return _ELEM.get(int(dtype))
+
+
+def _n(*xs) -> int:
+    """Product of sizes, 0 if any is negative (the library then rejects the sizes itself)."""
+    r = 1
+    for x in xs:
+        if int(x) < 0:
+            return 0
+        r *= int(x)
+    return r
 
 
 def _stream(stream) -> Optional[int]:
@@ -113,15 +147,31 @@ def _check(status: int, what: str) -> None:
         raise AttnError(status, what)
 
 
+def _fwd_sizes(B, Sq, Skv, Nq, Nkv, D, Dv, layout):
+    """Element counts of q, k, v, out and one statistic array in attn_fwd's layouts."""
+    if int(layout) == ATTN_TND:
+        return _n(Sq, Nq, D), _n(Skv, Nkv, D), _n(Skv, Nkv, Dv), _n(Sq, Nq, Dv), _n(Sq, Nq)
+    return (_n(B, Nq, Sq, D), _n(B, Nkv, Skv, D), _n(B, Nkv, Skv, Dv), _n(B, Nq, Sq, Dv),
+            _n(B, Nq, Sq))
+
+
+def _cu_ptr(cu, name: str, B: int):
+    return _ptr(cu, name, _n(B), "int32")
+
+
 def attn_fwd(q, k, v, *, cu_seqlens_q=None, cu_seqlens_kv=None, B: int, Sq: int, Skv: int,
              Nq: int, Nkv: int, D: int, scale: float, mask_mode: int, dtype: int, layout: int,
              out, softmax_max=None, softmax_sum=None, stream=None) -> None:
     """Fused attention forward (see ``attn_fwd`` in include/attn.h for layouts and limits)."""
     lib = load_library()
-    _check(lib.attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens_q), _ptr(cu_seqlens_kv),
+    nq, nk, nv, no, ns = _fwd_sizes(B, Sq, Skv, Nq, Nkv, D, D, layout)
+    et = _elem(dtype)
+    _check(lib.attn_fwd(_ptr(q, "q", nq, et), _ptr(k, "k", nk, et), _ptr(v, "v", nv, et),
+                        _cu_ptr(cu_seqlens_q, "cu_seqlens_q", B), _cu_ptr(cu_seqlens_kv, "cu_seqlens_kv", B),
                         int(B), int(Sq), int(Skv), int(Nq), int(Nkv), int(D), float(scale),
-                        int(mask_mode), int(dtype), int(layout), _ptr(out), _ptr(softmax_max),
-                        _ptr(softmax_sum), _stream(stream)), "attn_fwd")
+                        int(mask_mode), int(dtype), int(layout), _ptr(out, "out", no, et),
+                        _ptr(softmax_max, "softmax_max", ns, "float32"),
+                        _ptr(softmax_sum, "softmax_sum", ns, "float32"), _stream(stream)), "attn_fwd")
 
 
 def attn_fwd_accumulate(q, k, v, *, cu_seqlens_q=None, cu_seqlens_kv=None, B: int, Sq: int, Skv: int,
@@ -130,10 +180,16 @@ def attn_fwd_accumulate(q, k, v, *, cu_seqlens_q=None, cu_seqlens_kv=None, B: in
     """attn_fwd over one chunk of keys, folded into a running accumulator in attn_merge's
     layouts (see ``attn_fwd_accumulate`` in include/attn.h)."""
     lib = load_library()
-    _check(lib.attn_fwd_accumulate(_ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens_q),
-                                   _ptr(cu_seqlens_kv), int(B), int(Sq), int(Skv), int(Nq), int(Nkv),
-                                   int(D), float(scale), int(mask_mode), int(dtype), int(layout),
-                                   1 if first else 0, _ptr(acc_out), _ptr(acc_max), _ptr(acc_sum),
+    nq, nk, nv, no, ns = _fwd_sizes(B, Sq, Skv, Nq, Nkv, D, D, layout)
+    et = _elem(dtype)
+    _check(lib.attn_fwd_accumulate(_ptr(q, "q", nq, et), _ptr(k, "k", nk, et), _ptr(v, "v", nv, et),
+                                   _cu_ptr(cu_seqlens_q, "cu_seqlens_q", B),
+                                   _cu_ptr(cu_seqlens_kv, "cu_seqlens_kv", B), int(B), int(Sq),
+                                   int(Skv), int(Nq), int(Nkv), int(D), float(scale), int(mask_mode),
+                                   int(dtype), int(layout), 1 if first else 0,
+                                   _ptr(acc_out, "acc_out", no, et),
+                                   _ptr(acc_max, "acc_max", 8 * ns, "float32"),
+                                   _ptr(acc_sum, "acc_sum", 8 * ns, "float32"),
                                    _stream(stream)), "attn_fwd_accumulate")
 
 
@@ -145,20 +201,33 @@ def attn_fwd_masked(q, k, v, *, cu_seqlens_q=None, cu_seqlens_kv=None, B: int, S
     """attn_fwd with a band, an optional uint8 mask (1 = excluded) and a value head size Dv
     (see ``attn_fwd_masked`` in include/attn.h)."""
     lib = load_library()
-    _check(lib.attn_fwd_masked(_ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens_q), _ptr(cu_seqlens_kv),
+    nq, nk, nv, no, ns = _fwd_sizes(B, Sq, Skv, Nq, Nkv, Dqk, Dv, layout)
+    et = _elem(dtype)
+    nm = 0
+    if int(layout) == ATTN_BHSD and _n(B, Sq, Skv) > 0:  # the last entry the mask is read at
+        nm = max(0, (int(B) - 1) * int(mask_batch_stride) + (int(Sq) - 1) * int(mask_row_stride) + int(Skv))
+    _check(lib.attn_fwd_masked(_ptr(q, "q", nq, et), _ptr(k, "k", nk, et), _ptr(v, "v", nv, et),
+                               _cu_ptr(cu_seqlens_q, "cu_seqlens_q", B),
+                               _cu_ptr(cu_seqlens_kv, "cu_seqlens_kv", B),
                                int(B), int(Sq), int(Skv), int(Nq), int(Nkv), int(Dqk), int(Dv),
                                float(scale), int(mask_mode), int(pre_tokens), int(next_tokens),
-                               _ptr(atten_mask), int(mask_batch_stride), int(mask_row_stride),
-                               int(dtype), int(layout), _ptr(out), _ptr(softmax_max),
-                               _ptr(softmax_sum), _stream(stream)), "attn_fwd_masked")
+                               _ptr(atten_mask, "atten_mask", nm, "uint8"), int(mask_batch_stride),
+                               int(mask_row_stride), int(dtype), int(layout), _ptr(out, "out", no, et),
+                               _ptr(softmax_max, "softmax_max", ns, "float32"),
+                               _ptr(softmax_sum, "softmax_sum", ns, "float32"), _stream(stream)),
+           "attn_fwd_masked")
 
 
 def attn_sparse_csr(q, k, v, csr_offset, csr_columns, *, B: int, H: int, S: int, D: int,
                     nnz_cap: int, out, stream=None) -> None:
     """CSR-sparse attention forward in float32 (see ``attn_sparse_csr`` in include/attn.h)."""
     lib = load_library()
-    _check(lib.attn_sparse_csr(_ptr(q), _ptr(k), _ptr(v), _ptr(csr_offset), _ptr(csr_columns),
-                               int(B), int(H), int(S), int(D), int(nnz_cap), _ptr(out),
+    n = _n(B, H, S, D)
+    _check(lib.attn_sparse_csr(_ptr(q, "q", n, "float32"), _ptr(k, "k", n, "float32"),
+                               _ptr(v, "v", n, "float32"),
+                               _ptr(csr_offset, "csr_offset", _n(B, H, int(S) + 1), "int32"),
+                               _ptr(csr_columns, "csr_columns", _n(B, H, nnz_cap), "int32"),
+                               int(B), int(H), int(S), int(D), int(nnz_cap), _ptr(out, "out", n, "float32"),
                                _stream(stream)), "attn_sparse_csr")
 
 
@@ -167,9 +236,13 @@ def attn_sparse_csr_tc(q, k, v, csr_offset, csr_columns, *, B: int, H: int, S: i
     """CSR-sparse attention forward in bf16/fp16 on the tensor cores (see
     ``attn_sparse_csr_tc`` in include/attn.h)."""
     lib = load_library()
-    _check(lib.attn_sparse_csr_tc(_ptr(q), _ptr(k), _ptr(v), _ptr(csr_offset), _ptr(csr_columns),
+    n = _n(B, H, S, D)
+    et = _elem(dtype)
+    _check(lib.attn_sparse_csr_tc(_ptr(q, "q", n, et), _ptr(k, "k", n, et), _ptr(v, "v", n, et),
+                                  _ptr(csr_offset, "csr_offset", _n(B, H, int(S) + 1), "int32"),
+                                  _ptr(csr_columns, "csr_columns", _n(B, H, nnz_cap), "int32"),
                                   int(B), int(H), int(S), int(D), int(nnz_cap), int(dtype),
-                                  _ptr(out), _stream(stream)), "attn_sparse_csr_tc")
+                                  _ptr(out, "out", n, et), _stream(stream)), "attn_sparse_csr_tc")
 
 
 def attn_merge(prev_out, prev_max, prev_sum, cur_out, cur_max, cur_sum, *, S: int, B: int, N: int,
@@ -177,10 +250,19 @@ def attn_merge(prev_out, prev_max, prev_sum, cur_out, cur_max, cur_sum, *, S: in
                actual_seq_qlen=None, stream=None) -> None:
     """Merge two partial attention results (see ``attn_merge`` in include/attn.h)."""
     lib = load_library()
-    _check(lib.attn_merge(_ptr(prev_out), _ptr(prev_max), _ptr(prev_sum), _ptr(cur_out),
-                          _ptr(cur_max), _ptr(cur_sum), int(S), int(B), int(N), int(D), int(dtype),
-                          int(layout), _ptr(actual_seq_qlen), _ptr(out), _ptr(out_max),
-                          _ptr(out_sum), _stream(stream)), "attn_merge")
+    et = _elem(dtype)
+    if int(layout) == ATTN_TND:
+        no, ns = _n(S, N, D), _n(S, N, 8)
+    else:
+        no, ns = _n(S, B, N, D), _n(B, N, S, 8)
+    f = "float32"
+    _check(lib.attn_merge(_ptr(prev_out, "prev_out", no, et), _ptr(prev_max, "prev_max", ns, f),
+                          _ptr(prev_sum, "prev_sum", ns, f), _ptr(cur_out, "cur_out", no, et),
+                          _ptr(cur_max, "cur_max", ns, f), _ptr(cur_sum, "cur_sum", ns, f), int(S),
+                          int(B), int(N), int(D), int(dtype), int(layout),
+                          _ptr(actual_seq_qlen, "actual_seq_qlen", _n(B), "int64"),
+                          _ptr(out, "out", no, et), _ptr(out_max, "out_max", ns, f),
+                          _ptr(out_sum, "out_sum", ns, f), _stream(stream)), "attn_merge")
 
 
 def attn_get_last_error(stream=None) -> int:

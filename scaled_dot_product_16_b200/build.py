@@ -4,7 +4,9 @@
     python -m scaled_dot_product_16_b200.build --force    # rebuild everything
 
 Each .cu file in csrc/ is compiled to an object under _build/ (skipped when newer than its
-sources), then linked into scaled_dot_product_16_b200/libattn.so. No GPU is needed.
+sources), then linked into scaled_dot_product_16_b200/libattn.so. A second copy built with the
+test flags (STALL_FLAGS) becomes libattn_stalltest.so, which only the timeout test loads. No GPU
+is needed.
 """
 from __future__ import annotations
 
@@ -31,29 +33,44 @@ def _newest(paths):
     return max(os.path.getmtime(p) for p in paths)
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    os.makedirs(BUILD, exist_ok=True)
+# The test build: identical sources, with the attention kernel's pipeline waits bounded at 1 ms
+# and one extra wait on a barrier that nothing arrives on, so that a GPU test sees that wait run
+# out and the kernel report ATTN_ERR_TIMEOUT, drain its own work and exit (drains keep 200 ms).
+STALL_LIB = os.path.join(PKG, "libattn_stalltest.so")
+STALL_FLAGS = ["-DSDPA_TEST_STALL=1", "-DSDPA_PIPE_WAIT_NS=1000000ull"]
+
+
+def _build_lib(lib: str, objdir: str, extra, force: bool, verbose: bool) -> str:
+    os.makedirs(objdir, exist_ok=True)
     sources = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
     headers = glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(CSRC, "*.h")) + \
         glob.glob(os.path.join(INCLUDE, "*.h"))
     hdr_time = _newest(headers) if headers else 0.0
     objs = []
     for src in sources:
-        obj = os.path.join(BUILD, os.path.basename(src)[:-3] + ".o")
+        obj = os.path.join(objdir, os.path.basename(src)[:-3] + ".o")
         objs.append(obj)
         if (not force and os.path.exists(obj)
                 and os.path.getmtime(obj) >= max(os.path.getmtime(src), hdr_time)):
             continue
-        cmd = [NVCC, *ARCH, *FLAGS, "-c", src, "-o", obj]
+        cmd = [NVCC, *ARCH, *FLAGS, *extra, "-c", src, "-o", obj]
         if verbose:
             cmd.insert(1, "-Xptxas=-v")
         subprocess.run(cmd, check=True)
-    if force or not os.path.exists(LIB) or os.path.getmtime(LIB) < _newest(objs):
-        tmp = LIB + f".tmp{os.getpid()}"
+    if force or not os.path.exists(lib) or os.path.getmtime(lib) < _newest(objs):
+        tmp = lib + f".tmp{os.getpid()}"
         subprocess.run([NVCC, *ARCH, "-shared", "-o", tmp, *objs, "-lcudart_static", "-ldl",
                         "-lpthread", "-lrt"], check=True)
-        os.replace(tmp, LIB)
-    return LIB
+        os.replace(tmp, lib)
+    return lib
+
+
+def build(force: bool = False, verbose: bool = False) -> str:
+    return _build_lib(LIB, BUILD, [], force, verbose)
+
+
+def build_stall_test(force: bool = False) -> str:
+    return _build_lib(STALL_LIB, os.path.join(BUILD, "stalltest"), STALL_FLAGS, force, False)
 
 
 def main(argv=None) -> int:
@@ -62,6 +79,7 @@ def main(argv=None) -> int:
     ap.add_argument("-v", "--verbose", action="store_true", help="print ptxas resource usage")
     args = ap.parse_args(argv)
     print(build(force=args.force, verbose=args.verbose))
+    print(build_stall_test(force=args.force))
     return 0
 
 

@@ -16,32 +16,46 @@
 
 namespace {
 
-// One status word per device; kernels record the first device-side error here.
+// One status word per device; kernels record the first device-side error here. Beside it, the
+// slot attn_get_last_error reads the word into (exchanging it for 0 in one atomic step).
 __device__ int g_status_word;
+__device__ int g_status_read;
 
 constexpr int kMaxDevices = 64;
 std::mutex g_mu;
+std::mutex g_read_mu[kMaxDevices];  // one status reader at a time per device (the read slot)
 int* g_status_ptr[kMaxDevices] = {};
+int* g_read_ptr[kMaxDevices] = {};
 int g_num_sms[kMaxDevices] = {};
 
-// Device address of this device's status word and its SM count (looked up once per device).
-int device_state(int** status, int* num_sms) {
+// Device addresses of this device's status word and read slot, and its SM count (looked up
+// once per device, with that device current).
+int device_state(int** status, int* num_sms, int** read_slot = nullptr, int* device = nullptr) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return ATTN_ERR_CUDA;
   std::lock_guard<std::mutex> lk(g_mu);
   if (g_status_ptr[dev] == nullptr) {
     void* p = nullptr;
+    void* r = nullptr;
     if (cudaGetSymbolAddress(&p, g_status_word) != cudaSuccess) return ATTN_ERR_CUDA;
+    if (cudaGetSymbolAddress(&r, g_status_read) != cudaSuccess) return ATTN_ERR_CUDA;
     int sms = 0;
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
       return ATTN_ERR_CUDA;
-    g_status_ptr[dev] = static_cast<int*>(p);
+    g_read_ptr[dev] = static_cast<int*>(r);
     g_num_sms[dev] = sms;
+    g_status_ptr[dev] = static_cast<int*>(p);
   }
   *status = g_status_ptr[dev];
   *num_sms = g_num_sms[dev];
+  if (read_slot != nullptr) *read_slot = g_read_ptr[dev];
+  if (device != nullptr) *device = dev;
   return ATTN_OK;
 }
+
+// Reads the status word and clears it in one step, so an error a kernel on another stream
+// records meanwhile is kept for the next read instead of being lost between a read and a clear.
+__global__ void read_and_clear_status(int* word, int* slot) { *slot = atomicExch(word, 0); }
 
 constexpr int64_t kMaxTokens = 1 << 20;  // "1M"
 constexpr int kMaxCu = 2048;             // "2K" cumulative-length entries
@@ -172,6 +186,9 @@ int attn_fwd_accumulate(const void* q, const void* k, const void* v, const int32
                         void* acc_out, float* acc_max, float* acc_sum, void* stream) {
   if (acc_out == nullptr || acc_max == nullptr || acc_sum == nullptr) return ATTN_ERR_INVALID;
   if (first != 0 && first != 1) return ATTN_ERR_INVALID;
+  // the tensor-core epilogue moves a row's 8 statistic lanes as two 16-byte vectors
+  if ((dtype == ATTN_BF16 || dtype == ATTN_F16) && (!aligned16(acc_max) || !aligned16(acc_sum)))
+    return ATTN_ERR_INVALID;
   return fwd_impl(q, k, v, cu_seqlens_q, cu_seqlens_kv, B, Sq, Skv, Nq, Nkv, D, scale, mask_mode,
                   dtype, layout, acc_out, acc_max, acc_sum, first ? 1 : 2, stream);
 }
@@ -305,15 +322,18 @@ int attn_merge(const void* prev_out, const float* prev_max, const float* prev_su
 int attn_get_last_error(void* stream, int* device_status) {
   if (device_status == nullptr) return ATTN_ERR_INVALID;
   int* word = nullptr;
-  int sms = 0;
-  int rc = device_state(&word, &sms);
+  int* slot = nullptr;
+  int sms = 0, dev = 0;
+  int rc = device_state(&word, &sms, &slot, &dev);
   if (rc != ATTN_OK) return rc;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  std::lock_guard<std::mutex> lk(g_read_mu[dev]);
   int host = 0;
-  if (cudaStreamSynchronize(st) != cudaSuccess) return ATTN_ERR_CUDA;
-  if (cudaMemcpy(&host, word, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+  read_and_clear_status<<<1, 1, 0, st>>>(word, slot);
+  if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+  if (cudaMemcpyAsync(&host, slot, sizeof(int), cudaMemcpyDeviceToHost, st) != cudaSuccess)
     return ATTN_ERR_CUDA;
-  if (cudaMemset(word, 0, sizeof(int)) != cudaSuccess) return ATTN_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return ATTN_ERR_CUDA;
   *device_status = host;
   return ATTN_OK;
 }

@@ -48,7 +48,19 @@ constexpr int kMmaWarp = 8;
 constexpr int kTmaWarp = 9;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale when the max grows by > 2^8
-constexpr uint64_t kWaitLimitNs = 200ull * 1000ull * 1000ull;  // 200 ms per barrier wait
+// Time bounds of a barrier wait: one in the pipeline (data or a hand-off from another role),
+// and one while draining work this block already issued (its TMA loads and MMAs must land
+// before TMEM is freed and the block exits). The test build of the library shortens the first.
+#ifndef SDPA_PIPE_WAIT_NS
+#define SDPA_PIPE_WAIT_NS 200000000ull
+#endif
+constexpr uint64_t kPipeWaitNs = SDPA_PIPE_WAIT_NS;
+constexpr uint64_t kDrainWaitNs = 200ull * 1000ull * 1000ull;  // 200 ms
+// Test build only: the MMA warp first waits on a barrier that nothing arrives on, so that wait
+// runs out and the timeout path (status word, abort, drains) is exercised without any fault.
+#ifndef SDPA_TEST_STALL
+#define SDPA_TEST_STALL 0
+#endif
 #ifndef SDPA_SUSPEND_NS
 #define SDPA_SUSPEND_NS 20000
 #endif
@@ -115,21 +127,24 @@ struct Barriers {
   uint64_t p_ready[2];
   uint64_t o_done[2];
   uint64_t drain;
+  uint64_t stall;  // never arrived on (the test build waits on it)
   uint32_t tmem_base;
   int abort;
 };
 
 // Bounded wait on an mbarrier phase. Returns false (after recording a timeout, or when another
 // role of this block already gave up) instead of waiting forever.
-// With heed_abort = false (used when draining work already issued) only the time bound applies.
+// With heed_abort = false (used when draining work already issued) only the drain's time
+// bound applies.
 __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort,
                                          int* status, bool heed_abort = true) {
   if (mbar_try_wait_sleep(bar, parity, kSuspendNs)) return true;
   const uint64_t t0 = globaltimer_ns();
+  const uint64_t limit = heed_abort ? kPipeWaitNs : kDrainWaitNs;
   for (;;) {
     if (mbar_try_wait_sleep(bar, parity, kSuspendNs)) return true;
     if (heed_abort && *abort) return false;
-    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+    if (globaltimer_ns() - t0 > limit) {
       *abort = 1;
       report(status, ATTN_ERR_TIMEOUT);
       return false;
@@ -283,6 +298,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(bar_addr(&bars->q_full), 1);
     mbar_init(bar_addr(&bars->drain), 1);
+    mbar_init(bar_addr(&bars->stall), 1);
     for (int q = 0; q < 2; ++q) {
       mbar_init(bar_addr(&bars->s_full[q]), 1);
       mbar_init(bar_addr(&bars->p_ready[q]), 4);  // one arrival per softmax warp
@@ -372,7 +388,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         mma_ts_chain8(d, p_tmem, dv, C::kIdescPV, acc ? 1u : 0u);
       };
       bool ok = true;
-      if (n1 > 0) {
+      if constexpr (SDPA_TEST_STALL != 0) ok = wait_bar(bar_addr(&bars->stall), 0, abort, a.status);
+      if (ok && n1 > 0) {
         ok = wait_bar(bar_addr(&bars->q_full), 0, abort, a.status);
         if (ok) ok = full(0);
       }

@@ -60,6 +60,13 @@ def csr_flops(inp: W.CsrInputs) -> int:
     return 4 * inp.D * int(inp.offset[..., -1].astype(np.int64).sum())
 
 
+def csr_min_bytes(inp: W.CsrInputs, elem: int = 4) -> int:
+    """Compulsory HBM traffic of attn_sparse_csr: q, k, v read and out written once, plus the
+    column indices and row pointers."""
+    qkvo = 4 * inp.B * inp.H * inp.S * inp.D * elem
+    return int(qkvo + inp.columns.size * 4 + inp.offset.size * 4)
+
+
 def merge_bytes(S: int, B: int, N: int, D: int, elem: int) -> int:
     out = S * B * N * D * elem
     stats = B * N * S * 8 * 4

@@ -725,4 +725,25 @@ def pin_round_bf16_matches_torch():
     assert np.array_equal(got, want)
 
 
+def pin_round_f16_matches_numpy_and_torch():
+    """float64 -> float16 in one rounding: numpy's cast rounds a double directly (torch's goes
+    through float32, so it is compared on float32-representable values only)."""
+    r = _rng(41)
+    tie = 1 + 2 ** -11                                   # halfway between 1 and 1 + 2^-10
+    x = np.concatenate([
+        r.standard_normal(20000) * 3.0,
+        r.standard_normal(2000) * 1e-6,                  # subnormal range (below 2^-14)
+        r.standard_normal(2000) * 3e4,                   # near the largest finite value
+        np.array([tie, tie + 2 ** -40, tie - 2 ** -40, 1 + 3 * 2 ** -11, -tie, 0.0, -0.0,
+                  2 ** -25, 2 ** -25 + 2 ** -60, 3 * 2 ** -25, 2 ** -14 - 2 ** -26, 65504.0,
+                  65519.99, 65520.0, -65520.0, 1e9, np.inf, -np.inf]),
+    ])
+    with np.errstate(over="ignore"):
+        want = x.astype(np.float16).view(np.uint16)
+    assert np.array_equal(oracle.round_f16(x), want)
+    x32 = r.standard_normal(20000).astype(np.float32) * np.float32(100.0)
+    want32 = torch.from_numpy(x32).to(torch.float16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(oracle.round_f16(x32.astype(np.float64)), want32)
+
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_") and callable(v)]

@@ -181,3 +181,105 @@ def test_product_never_touches_the_oracle():
                 text = open(os.path.join(dirpath, f), encoding="utf-8").read()
                 assert not re.search(r"^\s*(import|from)\s+oracle\b", text, re.M), f
                 assert "attn_oracle" not in text, f
+
+
+class FakeCuda:
+    """Stands in for a CUDA tensor on a machine without a GPU (the binding reads only these
+    attributes before it calls the library)."""
+
+    def __init__(self, numel, dtype, index=0):
+        import torch
+        self._n, self.dtype, self.device, self.is_cuda = numel, dtype, torch.device("cuda", index), True
+
+    def numel(self):
+        return self._n
+
+    def is_contiguous(self):
+        return True
+
+    def data_ptr(self):
+        return 256
+
+
+@pytest.fixture
+def on_cuda0(monkeypatch):
+    import torch
+    monkeypatch.setattr(torch.cuda, "current_device", lambda: 0)
+    monkeypatch.setattr(sdpa, "_stream", lambda s: 0)
+
+
+def _fwd_kwargs(**kw):
+    import torch
+    bf = torch.bfloat16
+    a = dict(q=FakeCuda(2 * 4 * 64, bf), k=FakeCuda(1 * 4 * 64, bf), v=FakeCuda(1 * 4 * 64, bf),
+             B=1, Sq=4, Skv=4, Nq=2, Nkv=1, D=64, scale=0.125, mask_mode=0, dtype=sdpa.ATTN_BF16,
+             layout=sdpa.ATTN_BHSD, out=FakeCuda(2 * 4 * 64, bf), softmax_max=FakeCuda(8, torch.float32),
+             softmax_sum=FakeCuda(8, torch.float32))
+    a.update(kw)
+    return a
+
+
+def test_binding_refuses_undersized_mistyped_and_foreign_tensors(lib, on_cuda0):
+    """Each refusal comes from the binding, before the library is called: a tensor smaller than
+    the sizes given, a tensor whose element type is not the declared one, integer arrays of the
+    wrong width, and a tensor on another device than the current one."""
+    import torch
+    bf, f32 = torch.bfloat16, torch.float32
+    refused = [
+        (dict(q=FakeCuda(2 * 4 * 64 - 1, bf)), "holds"),                 # q one element short
+        (dict(out=FakeCuda(100, bf)), "holds"),                            # out too small
+        (dict(softmax_max=FakeCuda(7, f32)), "holds"),                     # statistics too small
+        (dict(q=FakeCuda(2 * 4 * 64, torch.float16)), "bfloat16"),         # fp16 data, bf16 declared
+        (dict(q=FakeCuda(2 * 4 * 64, f32), k=FakeCuda(256, f32), v=FakeCuda(256, f32),
+              out=FakeCuda(512, f32), dtype=sdpa.ATTN_BF16), "bfloat16"),  # fp32 data, bf16 declared
+        (dict(softmax_sum=FakeCuda(8, bf)), "float32"),                    # statistics must be fp32
+        (dict(k=FakeCuda(256, bf, index=1)), "current device"),            # k on another GPU
+    ]
+    for kw, msg in refused:
+        with pytest.raises(ValueError, match=msg):
+            sdpa.attn_fwd(**_fwd_kwargs(**kw))
+    # TND: cumulative lengths must be int32 with B entries
+    tnd = dict(layout=sdpa.ATTN_TND, B=2, Sq=4, Skv=4, q=FakeCuda(4 * 2 * 64, bf), k=FakeCuda(4 * 64, bf),
+               v=FakeCuda(4 * 64, bf), out=FakeCuda(4 * 2 * 64, bf))
+    with pytest.raises(ValueError, match="int32"):
+        sdpa.attn_fwd(**_fwd_kwargs(**tnd, cu_seqlens_q=FakeCuda(2, torch.int64), cu_seqlens_kv=FakeCuda(2, torch.int32)))
+    with pytest.raises(ValueError, match="holds"):
+        sdpa.attn_fwd(**_fwd_kwargs(**tnd, cu_seqlens_q=FakeCuda(1, torch.int32), cu_seqlens_kv=FakeCuda(2, torch.int32)))
+    # CSR: fp32 tensors, int32 row pointers and columns of the stated sizes
+    n = 1 * 2 * 8 * 64
+    csr = dict(B=1, H=2, S=8, D=64, nnz_cap=10)
+    good = [FakeCuda(n, f32) for _ in range(3)] + [FakeCuda(2 * 9, torch.int32), FakeCuda(20, torch.int32)]
+    with pytest.raises(ValueError, match="csr_columns"):
+        sdpa.attn_sparse_csr(*good[:4], FakeCuda(19, torch.int32), out=FakeCuda(n, f32), **csr)
+    with pytest.raises(ValueError, match="csr_offset"):
+        sdpa.attn_sparse_csr(*good[:3], FakeCuda(2 * 9, torch.int64), good[4], out=FakeCuda(n, f32), **csr)
+    with pytest.raises(ValueError, match="float32"):
+        sdpa.attn_sparse_csr(FakeCuda(n, bf), *good[1:], out=FakeCuda(n, f32), **csr)
+    # merge: TND lengths are int64; statistics fp32 with 8 lanes per row
+    S, N, D = 16, 2, 64
+    po = FakeCuda(S * N * D, bf)
+    st = FakeCuda(S * N * 8, f32)
+    with pytest.raises(ValueError, match="int64"):
+        sdpa.attn_merge(po, st, st, po, st, st, S=S, B=2, N=N, D=D, dtype=sdpa.ATTN_BF16, out=po,
+                        out_max=st, out_sum=st, layout=sdpa.ATTN_TND,
+                        actual_seq_qlen=FakeCuda(2, torch.int32))
+    with pytest.raises(ValueError, match="holds"):
+        sdpa.attn_merge(po, FakeCuda(S * N, f32), st, po, st, st, S=S, B=2, N=N, D=D,
+                        dtype=sdpa.ATTN_BF16, out=po, out_max=st, out_sum=st, layout=sdpa.ATTN_TND)
+    # accumulator statistics carry 8 lanes per row
+    with pytest.raises(ValueError, match="acc_max"):
+        a = _fwd_kwargs()
+        sdpa.attn_fwd_accumulate(a["q"], a["k"], a["v"], B=1, Sq=4, Skv=4, Nq=2, Nkv=1, D=64, scale=0.125,
+                                 mask_mode=0, dtype=sdpa.ATTN_BF16, layout=sdpa.ATTN_BHSD, first=True,
+                                 acc_out=FakeCuda(512, bf), acc_max=FakeCuda(8, f32), acc_sum=FakeCuda(64, f32))
+
+
+def test_accumulate_refuses_unaligned_statistics(lib):
+    """The tensor-core epilogue moves a row's 8 statistic lanes as 16-byte vectors, so for 16-bit
+    types a 4-byte-aligned accumulator (a sliced view, say) is refused on the host."""
+    def call(am, al, dtype):
+        return lib.attn_fwd_accumulate(16, 16, 16, None, None, 1, 8, 8, 2, 1, 64, 0.125, 0, dtype,
+                                       sdpa.ATTN_BHSD, 1, 16, am, al, None)
+    assert call(20, 16, sdpa.ATTN_BF16) == sdpa.ATTN_ERR_INVALID
+    assert call(16, 36, sdpa.ATTN_F16) == sdpa.ATTN_ERR_INVALID
+    assert call(24, 40, sdpa.ATTN_BF16) == sdpa.ATTN_ERR_INVALID

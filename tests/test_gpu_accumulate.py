@@ -21,15 +21,18 @@ def _chunks_bhsd(inp, n):
 def _accumulate_bhsd(inp, n_chunks):
     B, N, S, D = inp.B, inp.Nq, inp.Sq, inp.D
     q = inp.q.cuda()
-    acc = torch.empty((S, B, N * D), dtype=inp.q.dtype, device="cuda")
-    am = torch.empty((B, N, S, 8), device="cuda")
-    al = torch.empty_like(am)
+    acc = G.Guarded((S, B, N * D), inp.q.dtype)
+    am = G.Guarded((B, N, S, 8), torch.float32)
+    al = G.Guarded((B, N, S, 8), torch.float32)
     for idx, (k, v, c) in enumerate(_chunks_bhsd(inp, n_chunks)):
         sdpa.attn_fwd_accumulate(q, k.cuda(), v.cuda(), B=B, Sq=S, Skv=c, Nq=N, Nkv=inp.Nkv, D=D,
                                  scale=inp.scale, mask_mode=W.MASK_NONE, dtype=inp.dtype,
-                                 layout=W.BHSD, first=idx == 0, acc_out=acc, acc_max=am, acc_sum=al)
+                                 layout=W.BHSD, first=idx == 0, acc_out=acc.t, acc_max=am.t,
+                                 acc_sum=al.t)
     assert sdpa.attn_get_last_error() == 0
-    return acc.cpu(), am.cpu(), al.cpu()
+    for g in (acc, am, al):
+        g.check("accumulator")
+    return acc.t.cpu(), am.t.cpu(), al.t.cpu()
 
 
 @pytest.mark.parametrize("tdt", [torch.bfloat16, torch.float16, torch.float32], ids=["bf16", "f16", "f32"])
@@ -39,7 +42,7 @@ def test_bhsd_chunks_equal_full(tdt, D):
     acc, am, al = _accumulate_bhsd(inp, 4)
     ref, rm, rl = G.oracle_fwd(inp)
     out = acc.reshape(inp.Sq, inp.B, inp.Nq, D).permute(1, 2, 0, 3)
-    G.check_out(G.f64(out), ref, inp.dtype, "accumulated out")
+    G.check_out(G.f64(out), ref, inp.dtype, "accumulated out", abs_ref=lambda: G.oracle_abs_fwd(inp))
     for lane in (0, 7):
         G.check_stats(am[..., lane].numpy(), al[..., lane].numpy(), rm, rl, "accumulated stats")
 
@@ -79,9 +82,10 @@ def test_tnd_chunks_equal_full(tdt):
     T, N, D = inp.Sq, inp.Nq, inp.D
     q = inp.q.cuda()
     cq = torch.from_numpy(inp.cu_q).cuda()
-    acc = torch.empty((T, N * D), dtype=tdt, device="cuda")
-    am = torch.empty((T, N, 8), device="cuda")
-    al = torch.empty_like(am)
+    acc_g = G.Guarded((T, N * D), tdt)
+    am_g = G.Guarded((T, N, 8), torch.float32)
+    al_g = G.Guarded((T, N, 8), torch.float32)
+    acc, am, al = acc_g.t, am_g.t, al_g.t
     for part in range(3):  # every sequence's keys split in three, some chunks empty
         idx, lk = [], []
         for s0, L in zip(starts, lens):
@@ -95,8 +99,11 @@ def test_tnd_chunks_equal_full(tdt):
                                  mask_mode=W.MASK_NONE, dtype=inp.dtype, layout=W.TND, first=part == 0,
                                  acc_out=acc, acc_max=am, acc_sum=al)
     assert sdpa.attn_get_last_error() == 0
+    for g in (acc_g, am_g, al_g):
+        g.check("TND accumulator")
     ref, rm, rl = G.oracle_fwd(inp)
-    G.check_out(G.f64(acc.cpu().reshape(T, N, D)), ref, inp.dtype, "accumulated TND out")
+    G.check_out(G.f64(acc.cpu().reshape(T, N, D)), ref, inp.dtype, "accumulated TND out",
+                abs_ref=lambda: G.oracle_abs_fwd(inp))
     G.check_stats(am[..., 0].cpu().numpy(), al[..., 0].cpu().numpy(), rm, rl, "accumulated TND stats")
 
 
@@ -106,8 +113,8 @@ def test_ring_cfg5_full_size_sampled():
     inp = W.dense_bhsd(4, 32, 8192, 128, causal=False, dtype=torch.bfloat16, seed=0, cfg=5)
     acc, am, al = _accumulate_bhsd(inp, 4)
     out = acc.reshape(8192, 4, 32, 128).permute(1, 2, 0, 3)
-    rows_h, rows_t = G.sample_rows(inp, 5, n_random=128, edge=16)
+    rows_h, rows_t = G.sample_rows(inp, 5, n_random=512, edge=8)
     og, mg, lg = G.gather_rows(out, am[..., 0], al[..., 0], inp, rows_h, rows_t)
     ref, rm, rl = G.oracle_rows(inp, rows_h, rows_t)
-    G.check_out(og, ref, W.BF16, "ring out")
+    G.check_out(og, ref, W.BF16, "ring out", abs_ref=lambda: G.oracle_abs_rows(inp, rows_h, rows_t))
     G.check_stats(mg, lg, rm, rl, "ring stats")

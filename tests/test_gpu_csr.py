@@ -16,9 +16,11 @@ def _run(q, k, v, off, cols, B, H, S, D):
     dq, dk, dv = (torch.as_tensor(x).float().cuda().contiguous() for x in (q, k, v))
     doff = torch.from_numpy(np.ascontiguousarray(off, np.int32)).cuda()
     dcol = torch.from_numpy(np.ascontiguousarray(cols, np.int32)).cuda()
-    out = torch.full_like(dq, float("nan"))
-    sdpa.attn_sparse_csr(dq, dk, dv, doff, dcol, B=B, H=H, S=S, D=D, nnz_cap=cols.shape[-1], out=out)
-    return out.cpu(), sdpa.attn_get_last_error()
+    out = G.guarded_like(dq)  # NaN-filled: every element must be written
+    sdpa.attn_sparse_csr(dq, dk, dv, doff, dcol, B=B, H=H, S=S, D=D, nnz_cap=cols.shape[-1], out=out.t)
+    st = sdpa.attn_get_last_error()
+    out.check("csr out")
+    return out.t.cpu(), st
 
 
 def test_paddle_worked_example():
@@ -214,11 +216,12 @@ def test_row_per_warp_path_on_misaligned_tensors():
     dq = buf[1:].view(B, H, S, D)
     dq.copy_(q.cuda())
     dk, dv = k.cuda(), v.cuda()
-    out = torch.full_like(dk, float("nan"))
+    out = G.guarded_like(dk)
     sdpa.attn_sparse_csr(dq, dk, dv, torch.from_numpy(off).cuda(), torch.from_numpy(cols).cuda(),
-                         B=B, H=H, S=S, D=D, nnz_cap=cols.shape[-1], out=out)
+                         B=B, H=H, S=S, D=D, nnz_cap=cols.shape[-1], out=out.t)
     assert sdpa.attn_get_last_error() == 0
-    G.check_out(out.cpu().numpy(), ref, W.F32, "row-per-warp path")
+    out.check("row-per-warp out")
+    G.check_out(out.t.cpu().numpy(), ref, W.F32, "row-per-warp path")
     out2, st = _run(q, k, v, off, cols, B, H, S, D)
     assert st == 0
     G.check_out(out2.numpy(), ref, W.F32, "tiled path")

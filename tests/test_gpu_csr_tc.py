@@ -20,10 +20,12 @@ def _run(q, k, v, off, cols, B, H, S, D):
     dq, dk, dv = (torch.as_tensor(x).cuda().contiguous() for x in (q, k, v))
     doff = torch.from_numpy(np.ascontiguousarray(off, np.int32)).cuda()
     dcol = torch.from_numpy(np.ascontiguousarray(cols, np.int32)).cuda()
-    out = torch.full_like(dq, float("nan"))
+    out = G.guarded_like(dq)  # NaN-filled: every element must be written
     sdpa.attn_sparse_csr_tc(dq, dk, dv, doff, dcol, B=B, H=H, S=S, D=D, nnz_cap=cols.shape[-1],
-                            dtype=W.dtype_code(dq.dtype), out=out)
-    return out.cpu(), sdpa.attn_get_last_error()
+                            dtype=W.dtype_code(dq.dtype), out=out.t)
+    st = sdpa.attn_get_last_error()
+    out.check("csr_tc out")
+    return out.t.cpu(), st
 
 
 def _inputs(B, H, S, D, dtype, seed):
@@ -47,11 +49,17 @@ def _distinct_pattern(rng, B, H, S, max_per_row, empty_every=0):
     return offs.reshape(B, H, S + 1), cols.reshape(B, H, cap)
 
 
+def _abs_ref(q, k, v, off, cols, B, H, S, D):
+    """A = sum_j w_j |v_j| per output element (the oracle on |V|), for the rule where |exact| >= 4."""
+    return lambda: oracle.sparse_csr(q, k, v.abs(), off, cols, B=B, H=H, S=S, D=D)
+
+
 def _check(q, k, v, off, cols, B, H, S, D):
     out, st = _run(q, k, v, off, cols, B, H, S, D)
     assert st == 0
     ref = oracle.sparse_csr(q, k, v, off, cols, B=B, H=H, S=S, D=D)
-    G.check_out(G.f64(out), ref, W.dtype_code(q.dtype), "csr_tc out")
+    G.check_out(G.f64(out), ref, W.dtype_code(q.dtype), "csr_tc out",
+                abs_ref=_abs_ref(q, k, v, off, cols, B, H, S, D))
 
 
 @pytest.mark.parametrize("dtype", [BF, F16], ids=["bf16", "f16"])
@@ -106,11 +114,13 @@ def test_narrow_union_marked_in_one_pass(D, aligned):
     buf = torch.zeros(cols.size + 1, dtype=torch.int32, device="cuda")
     dcol = (buf[:-1] if aligned else buf[1:]).view(cols.shape)
     dcol.copy_(torch.from_numpy(cols))
-    out = torch.full_like(dq, float("nan"))
+    out = G.guarded_like(dq)
     sdpa.attn_sparse_csr_tc(dq, dk, dv, doff, dcol, B=B, H=H, S=S, D=D, nnz_cap=cols.shape[-1],
-                            dtype=sdpa.ATTN_BF16, out=out)
+                            dtype=sdpa.ATTN_BF16, out=out.t)
     assert sdpa.attn_get_last_error() == 0
-    G.check_out(G.f64(out.cpu()), ref, W.BF16, "one-pass marks")
+    out.check("csr_tc out")
+    G.check_out(G.f64(out.t.cpu()), ref, W.BF16, "one-pass marks",
+                abs_ref=_abs_ref(q, k, v, off, cols, B, H, S, D))
 
 
 @pytest.mark.parametrize("S,D", [(32768, 64), (32767, 128)])
@@ -162,7 +172,8 @@ def test_data_errors_zero_only_the_bad_rows():
     assert torch.all(out[0, 0, 20] == 0) and torch.all(out[0, 0, 150] == 0)
     keep = np.ones(S, bool)
     keep[[20, 150]] = False
-    G.check_out(G.f64(out)[0, 0, keep], ref[0, 0, keep], W.BF16, "other rows")
+    absr = oracle.sparse_csr(q, k, v.abs(), off, cols, B=B, H=H, S=S, D=D)
+    G.check_out(G.f64(out)[0, 0, keep], ref[0, 0, keep], W.BF16, "other rows", abs_ref=absr[0, 0, keep])
 
 
 def test_validation():
@@ -172,6 +183,9 @@ def test_validation():
     with pytest.raises(sdpa.AttnError) as e:
         sdpa.attn_sparse_csr_tc(q, q, q, off, cols, B=1, H=1, S=8, D=96, nnz_cap=1, dtype=W.BF16, out=q)
     assert e.value.status == sdpa.ATTN_ERR_UNSUPPORTED
-    with pytest.raises(sdpa.AttnError) as e:
+    with pytest.raises(ValueError, match="float32"):  # bf16 tensors declared fp32: the binding refuses
         sdpa.attn_sparse_csr_tc(q, q, q, off, cols, B=1, H=1, S=8, D=96, nnz_cap=1, dtype=W.F32, out=q)
+    with pytest.raises(sdpa.AttnError) as e:  # fp32 tensors: the library runs 16-bit types only
+        qf = q.float()
+        sdpa.attn_sparse_csr_tc(qf, qf, qf, off, cols, B=1, H=1, S=8, D=96, nnz_cap=1, dtype=W.F32, out=qf)
     assert e.value.status == sdpa.ATTN_ERR_INVALID

@@ -15,7 +15,7 @@ BF, F32 = torch.bfloat16, torch.float32
 def _full_check(inp, stats=True):
     out, m, l = G.run_fwd(inp, stats=stats)
     ref, rm, rl = G.oracle_fwd(inp)
-    info = G.check_out(G.f64(out), ref, inp.dtype)
+    info = G.check_out(G.f64(out), ref, inp.dtype, abs_ref=lambda: G.oracle_abs_fwd(inp))
     if stats:
         G.check_stats(m.numpy(), l.numpy(), rm, rl)
     return info
@@ -83,7 +83,7 @@ def test_no_stats_pointer():
     inp = W.dense_bhsd(1, 2, 300, 128, causal=True, dtype=BF, seed=3, cfg=16)
     out, _, _ = G.run_fwd(inp, stats=False)
     ref, _, _ = G.oracle_fwd(inp)
-    G.check_out(G.f64(out), ref, inp.dtype)
+    G.check_out(G.f64(out), ref, inp.dtype, abs_ref=lambda: G.oracle_abs_fwd(inp))
 
 
 # ---- full-size configurations: sampled rows ----------------------------------------------------
@@ -92,7 +92,7 @@ def _sampled_check(inp, seed):
     rows_h, rows_t = G.sample_rows(inp, seed)
     og, mg, lg = G.gather_rows(out, m, l, inp, rows_h, rows_t)
     ref, rm, rl = G.oracle_rows(inp, rows_h, rows_t)
-    G.check_out(og, ref, inp.dtype)
+    G.check_out(og, ref, inp.dtype, abs_ref=lambda: G.oracle_abs_rows(inp, rows_h, rows_t))
     G.check_stats(mg, lg, rm, rl)
     # every output is finite (no NaN from masked or padded rows)
     assert torch.isfinite(out.float()).all()
@@ -133,6 +133,47 @@ def test_varlen_equals_dense_per_sequence():
         start += L
 
 
+@pytest.mark.parametrize("masked", [False, True], ids=["attn_fwd", "attn_fwd_masked"])
+def test_tnd_rows_past_each_sequence_untouched(masked):
+    """Each sequence of a packed batch run as a batch of its own, on views that start at its
+    first token: the last row block of a sequence covers rows past its end (the next sequence's
+    tokens, pre-filled with the NaN pattern), and none of them may be stored. Afterwards the
+    assembled outputs equal the packed call's bit for bit."""
+    lens = [300, 129, 1, 513, 0, 256, 77]
+    inp = W.varlen_tnd(lens, 4, 2, 128, causal=True, dtype=BF, seed=21, cfg=24)
+    q, k, v, _, _ = G.to_dev(inp)
+    out = G.Guarded(tuple(q.shape), q.dtype)
+    m = G.Guarded((inp.Sq, inp.Nq), torch.float32)
+    l = G.Guarded((inp.Sq, inp.Nq), torch.float32)
+    starts = np.concatenate([[0], np.cumsum(lens)[:-1]]).tolist()
+    for s0, L in zip(starts, lens):
+        if L == 0:
+            continue
+        before = [g.buf.view(torch.int16).clone() for g in (out, m, l)]
+        cu = torch.tensor([L], dtype=torch.int32, device="cuda")
+        kw = dict(cu_seqlens_q=cu, cu_seqlens_kv=cu, B=1, Sq=L, Skv=L, Nq=4, Nkv=2, scale=inp.scale,
+                  dtype=W.BF16, layout=W.TND, out=out.t[s0:s0 + L], softmax_max=m.t[s0:s0 + L],
+                  softmax_sum=l.t[s0:s0 + L])
+        sl = slice(s0, s0 + L)
+        if masked:
+            sdpa.attn_fwd_masked(q[sl], k[sl], v[sl], Dqk=128, Dv=128, mask_mode=W.MASK_CAUSAL_TOPLEFT, **kw)
+        else:
+            sdpa.attn_fwd(q[sl], k[sl], v[sl], D=128, mask_mode=W.MASK_CAUSAL_TOPLEFT, **kw)
+        assert sdpa.attn_get_last_error() == 0
+        for g, b, per_row in ((out, before[0], inp.Nq * 128), (m, before[1], inp.Nq * 2),
+                              (l, before[2], inp.Nq * 2)):
+            now = g.buf.view(torch.int16)
+            a = g.g * g.buf.element_size() // 2 + s0 * per_row  # first int16 of this sequence's rows
+            e = a + L * per_row
+            assert torch.equal(now[:a], b[:a]) and torch.equal(now[e:], b[e:]), \
+                f"sequence at {s0} (length {L}) stored outside its rows"
+        for g in (out, m, l):
+            g.check()
+    whole = G.run_fwd(inp)
+    assert torch.equal(out.t.cpu(), whole[0])
+    assert torch.equal(m.t.cpu(), whole[1]) and torch.equal(l.t.cpu(), whole[2])
+
+
 # ---- boundary errors ------------------------------------------------------------------------------
 def test_bad_cu_seqlens_reports_data_error():
     inp = W.varlen_tnd([100, 200], 2, 2, 128, causal=True, dtype=BF, seed=1, cfg=18)
@@ -151,9 +192,11 @@ def test_host_validation():
     out = torch.empty_like(q)
     kw = dict(B=1, Sq=64, Skv=64, Nq=2, Nkv=2, D=128, scale=0.1, mask_mode=0, dtype=W.BF16,
               layout=W.BHSD, out=out)
-    with pytest.raises(sdpa.AttnError) as e:
-        sdpa.attn_fwd(q, k, v, **{**kw, "Nkv": 3})
+    with pytest.raises(sdpa.AttnError) as e:  # Nq not a multiple of Nkv (tensors large enough)
+        sdpa.attn_fwd(q, k, v, **{**kw, "Nq": 3, "Nkv": 2, "Sq": 32, "Skv": 32})
     assert e.value.status == sdpa.ATTN_ERR_INVALID
+    with pytest.raises(ValueError, match="holds"):  # k too small for Nkv = 3: refused by the binding
+        sdpa.attn_fwd(q, k, v, **{**kw, "Nkv": 3})
     with pytest.raises(sdpa.AttnError) as e:
         sdpa.attn_fwd(q, k, v, **{**kw, "D": 96})
     assert e.value.status == sdpa.ATTN_ERR_UNSUPPORTED

@@ -24,17 +24,21 @@ def _run(inp, *, mode, pre=0, nxt=0, mask=None, bs=0, rs=0, Dv=None, stats=True)
     Dv = inp.D if Dv is None else Dv
     shape_o = (inp.B, inp.Nq, inp.Sq, Dv) if inp.layout == W.BHSD else (inp.Sq, inp.Nq, Dv)
     shape_s = (inp.B, inp.Nq, inp.Sq) if inp.layout == W.BHSD else (inp.Sq, inp.Nq)
-    out = torch.full(shape_o, 7.0, dtype=q.dtype, device="cuda")  # every element must be written
-    m = torch.empty(shape_s, device="cuda") if stats else None
-    l = torch.empty(shape_s, device="cuda") if stats else None
+    out = G.Guarded(shape_o, q.dtype)  # NaN-filled: every element must be written
+    m = G.Guarded(shape_s, torch.float32) if stats else None
+    l = G.Guarded(shape_s, torch.float32) if stats else None
     md = None if mask is None else torch.from_numpy(mask).cuda()
     sdpa.attn_fwd_masked(q, k, v, cu_seqlens_q=cq, cu_seqlens_kv=ck, B=inp.B, Sq=inp.Sq,
                          Skv=inp.Skv, Nq=inp.Nq, Nkv=inp.Nkv, Dqk=inp.D, Dv=Dv, scale=inp.scale,
                          mask_mode=mode, pre_tokens=pre, next_tokens=nxt, atten_mask=md,
                          mask_batch_stride=bs, mask_row_stride=rs, dtype=inp.dtype,
-                         layout=inp.layout, out=out, softmax_max=m, softmax_sum=l)
+                         layout=inp.layout, out=out.t, softmax_max=m.t if stats else None,
+                         softmax_sum=l.t if stats else None)
     assert sdpa.attn_get_last_error() == 0
-    return out.cpu(), (m.cpu() if stats else None), (l.cpu() if stats else None)
+    for g in (out, m, l):
+        if g is not None:
+            g.check()
+    return out.t.cpu(), (m.t.cpu() if stats else None), (l.t.cpu() if stats else None)
 
 
 def _oracle(inp, *, mode, pre=0, nxt=0, mask=None, bs=0, rs=0, Dv=None):
@@ -48,7 +52,7 @@ def _oracle(inp, *, mode, pre=0, nxt=0, mask=None, bs=0, rs=0, Dv=None):
 def _check(inp, **kw):
     out, m, l = _run(inp, **kw)
     ref, rm, rl = _oracle(inp, **kw)
-    G.check_out(G.f64(out), ref, inp.dtype)
+    G.check_out(G.f64(out), ref, inp.dtype, abs_ref=lambda: _oracle(G.abs_v(inp), **kw)[0])
     G.check_stats(m.numpy(), l.numpy(), rm, rl)
     return out, m, l
 
@@ -161,7 +165,12 @@ def test_band_full_size_sampled():
                                            Nq=inp.Nq, Nkv=inp.Nkv, Dqk=inp.D, Dv=inp.D,
                                            scale=inp.scale, mask_mode=BAND, pre_tokens=1023,
                                            next_tokens=0, layout=inp.layout)
-    G.check_out(og, ref, inp.dtype)
+    absr = lambda: oracle.attn_fwd_ext_rows(inp.q, inp.k, inp.v.abs(), rows_h, rows_t, cu_q=inp.cu_q,  # noqa: E731
+                                            cu_kv=inp.cu_kv, B=inp.B, Sq=inp.Sq, Skv=inp.Skv,
+                                            Nq=inp.Nq, Nkv=inp.Nkv, Dqk=inp.D, Dv=inp.D,
+                                            scale=inp.scale, mask_mode=BAND, pre_tokens=1023,
+                                            next_tokens=0, layout=inp.layout)[0]
+    G.check_out(og, ref, inp.dtype, abs_ref=absr)
     G.check_stats(mg, lg, rm, rl)
     assert torch.isfinite(out.float()).all()
 
@@ -219,5 +228,5 @@ def test_causal_attention_from_band_masked_key_chunks():
         assert sdpa.attn_get_last_error() == 0
     got = acc[0].cpu().reshape(S, B, N, D).permute(1, 2, 0, 3)
     ref, rm, rl = G.oracle_fwd(full)
-    G.check_out(G.f64(got), ref, W.BF16, "causal from chunks")
+    G.check_out(G.f64(got), ref, W.BF16, "causal from chunks", abs_ref=lambda: G.oracle_abs_fwd(full))
     G.check_stats(acc[1][..., 0].cpu().numpy(), acc[2][..., 0].cpu().numpy(), rm, rl, "causal stats")

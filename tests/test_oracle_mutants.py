@@ -56,6 +56,9 @@ MUTANTS = [
     ("bf16_decode_unshifted", "uint32_t bits = ((uint32_t)((const uint16_t *)base)[idx]) << 16;",
      "uint32_t bits = ((uint32_t)((const uint16_t *)base)[idx]);", 0),
     ("bf16_truncates", "nearbyint(m * 256.0)", "floor(m * 256.0)", 0),
+    ("f16_truncates", "nearbyint(m * 2048.0)", "floor(m * 2048.0)", 0),
+    ("f16_subnormal_grid_off", "nearbyint(a * 0x1p24)", "nearbyint(a * 0x1p23) * 2.0", 0),
+    ("f16_exponent_bias_off", "(e - 1 + 15) << 10", "(e + 15) << 10", 0),
     ("band_lower_off_by_one", "(j < i - pre || j > i + next)", "(j <= i - pre || j > i + next)", 0),
     ("band_upper_sign", "(j < i - pre || j > i + next)", "(j < i - pre || j > i - next)", 0),
     ("mask_polarity", "mask[mrow + i * mask_rstride + j] != 0", "mask[mrow + i * mask_rstride + j] == 0", 0),
