@@ -312,7 +312,26 @@ def next_rows(fwd: "FwdCase", csr: "CsrCase", rank: int, stream, peaks: dict) ->
                                  "ms": ms, "tflops": c.flops / (ms / 1e3) / 1e12,
                                  "frac_of_bf16_peak": c.flops / (ms / 1e3) / 1e12 / tensor,
                                  "fp32_kernel_ms": ms32, "speedup_vs_fp32": ms32 / ms}
-    del qb, kb, vb, outb
+    # the same call from a plan of the pattern: the plan is built once (timed on its own) and
+    # each call then only gathers the union's key/value rows and multiplies
+    nb = sdpa.attn_csr_plan_size(B=ci.B, H=ci.H, S=ci.S, nnz_cap=ci.nnz_cap)
+    plan = torch.empty(nb, dtype=torch.uint8, device="cuda")
+
+    def mkplan():
+        sdpa.attn_csr_plan(c.off, c.col, B=ci.B, H=ci.H, S=ci.S, nnz_cap=ci.nnz_cap, plan=plan)
+
+    def planned():
+        sdpa.attn_sparse_csr_tc_planned(qb, kb, vb, plan, B=ci.B, H=ci.H, S=ci.S, D=ci.D,
+                                        nnz_cap=ci.nnz_cap, dtype=W.BF16, out=outb)
+
+    ms_plan = _device_ms(mkplan, 20, stream)
+    ms_exec = _device_ms(planned, 20, stream)
+    res["attn_sparse_csr_tc_planned"] = {
+        "workload": "2x8x4096x64 bf16, window 256 + every 64th column, from a plan",
+        "ms": ms_exec, "tflops": c.flops / (ms_exec / 1e3) / 1e12, "plan_ms": ms_plan,
+        "plan_bytes": nb, "speedup_vs_per_call_union": ms / ms_exec,
+        "plan_plus_call_ms": ms_plan + ms_exec}
+    del qb, kb, vb, outb, plan
     # merge in the TND layout (ring-attention update of a packed batch): T = 65,536 tokens,
     # N = 32, D = 128, bf16 outputs, [T, N, 8] statistics, with actual_seq_qlen checked
     T, N, D = 65536, 32, 128

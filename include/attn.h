@@ -9,6 +9,8 @@
  *   attn_fwd_accumulate  attn_fwd over one chunk of keys folded into a running merge result.
  *   attn_fwd_masked  attn_fwd with band limits, an explicit mask and a value head size Dv.
  *   attn_sparse_csr_tc  attn_sparse_csr in bf16 / fp16 on the tensor cores.
+ *   attn_csr_plan    the pattern bookkeeping of attn_sparse_csr_tc, once per pattern, into a
+ *                    caller-owned buffer that attn_sparse_csr_tc_planned then reads.
  *
  * Conventions shared by every call
  *   - All tensor pointers are DEVICE pointers owned by the caller. The library allocates no
@@ -216,6 +218,42 @@ ATTN_API int attn_sparse_csr_tc(const void* q, const void* k, const void* v,
                                 const int32_t* csr_offset, const int32_t* csr_columns,
                                 int B, int H, int S, int D, int64_t nnz_cap, int dtype,
                                 void* out, void* stream);
+
+/*
+ * CSR pattern plans -- the pattern bookkeeping of attn_sparse_csr_tc, done once per pattern.
+ *
+ * Defined by: "paddle.nn.functional.sparse_attention" (Paddle 2.3 API doc), 参数: the pattern is
+ * offset [B, H, S+1] (a row pointer per (b, h)) and columns [B, H, nnz_cap]. The two-phase form
+ * (size the caller-owned buffer, then run) follows "aclnnFlashAttentionVarLenScore" (CANN 8.5
+ * API doc), 函数原型 (GetWorkspaceSize, then the call that takes the workspace).
+ *
+ * A plan holds, for every block of 128 query rows of every (b, h): the sorted union of the
+ * columns the block's rows store, a bit per (row, union column) saying which of them the row
+ * stores, and which rows are bad. It depends on the pattern only, so a model with a fixed
+ * sparsity pattern builds it once and reuses it for every call.
+ *
+ * attn_csr_plan_size: *bytes = the plan's size for this shape, computed on the host from the
+ *   arguments alone: B * H * ceil(S/128) * (64 + 20 * ucap) with ucap = min(S, nnz_cap) rounded
+ *   up to 128. S <= 32768 (larger is ATTN_ERR_UNSUPPORTED); negative sizes or a null `bytes`
+ *   are ATTN_ERR_INVALID. Launches nothing.
+ * attn_csr_plan: fills `plan` (device memory owned by the caller, 16-byte aligned, at least
+ *   attn_csr_plan_size bytes, else ATTN_ERR_INVALID) from csr_offset / csr_columns (as for
+ *   attn_sparse_csr). Asynchronous on `stream`; the plan may be used by later launches on the
+ *   same stream. Data errors are recorded in the status word and in the plan: a row pointer that
+ *   starts above 0, decreases or passes nnz_cap, a column outside [0, S), or a column stored
+ *   twice in one row make that row bad (its output zeros, ATTN_ERR_DATA).
+ * attn_sparse_csr_tc_planned: attn_sparse_csr_tc (same definition, types, shapes and limits)
+ *   computed from a plan of the pattern instead of the pattern itself. plan / plan_bytes must
+ *   satisfy the rules above for the same B, H, S and nnz_cap; a plan record that was not built
+ *   for this S and nnz_cap (or not built at all) is not used: its rows are written as zeros and
+ *   ATTN_ERR_DATA is recorded. Each plan must not be rewritten while a call that reads it runs.
+ */
+ATTN_API int attn_csr_plan_size(int B, int H, int S, int64_t nnz_cap, int64_t* bytes);
+ATTN_API int attn_csr_plan(const int32_t* csr_offset, const int32_t* csr_columns, int B, int H,
+                           int S, int64_t nnz_cap, void* plan, int64_t plan_bytes, void* stream);
+ATTN_API int attn_sparse_csr_tc_planned(const void* q, const void* k, const void* v,
+                                        const void* plan, int64_t plan_bytes, int B, int H, int S,
+                                        int D, int64_t nnz_cap, int dtype, void* out, void* stream);
 
 /*
  * attn_merge -- merge two partial attention results (the ring-attention update).

@@ -1,7 +1,8 @@
 """Python binding of libattn.so: scaled-dot-product attention forward on B200 (sm_100a).
 
 The operations (attn_fwd, attn_fwd_masked, attn_fwd_accumulate, attn_sparse_csr,
-attn_sparse_csr_tc, attn_merge, attn_get_last_error) are the C-ABI calls declared in
+attn_sparse_csr_tc, attn_csr_plan_size, attn_csr_plan, attn_sparse_csr_tc_planned, attn_merge,
+attn_get_last_error) are the C-ABI calls declared in
 ``include/attn.h``; the functions here carry the same names and only marshal arguments (tensor
 data pointers, sizes, the current CUDA stream) into them. Every step of the computation runs in the library's CUDA kernels.
 There is no CPU path: if ``libattn.so`` is missing the first call raises.
@@ -20,7 +21,8 @@ __all__ = [
     "attn_fwd", "attn_fwd_accumulate", "attn_sparse_csr", "attn_merge", "attn_get_last_error", "AttnError",
     "ATTN_BF16", "ATTN_F32", "ATTN_F16", "ATTN_BHSD", "ATTN_TND", "ATTN_MASK_NONE",
     "ATTN_MASK_CAUSAL_TOPLEFT", "ATTN_MASK_CAUSAL_BOTTOMRIGHT", "ATTN_MASK_BAND", "lib_path",
-    "load_library", "attn_fwd_masked", "attn_sparse_csr_tc",
+    "load_library", "attn_fwd_masked", "attn_sparse_csr_tc", "attn_csr_plan_size", "attn_csr_plan",
+    "attn_sparse_csr_tc_planned",
 ]
 
 ATTN_OK, ATTN_ERR_INVALID, ATTN_ERR_UNSUPPORTED, ATTN_ERR_CUDA, ATTN_ERR_DATA, ATTN_ERR_TIMEOUT = range(6)
@@ -66,6 +68,12 @@ def load_library():
         lib.attn_sparse_csr_tc.argtypes = [P, P, P, P, P, I, I, I, I, I64, I, P, P]
         lib.attn_sparse_csr_tc.restype = I
         lib.attn_sparse_csr.restype = I
+        lib.attn_csr_plan_size.argtypes = [I, I, I, I64, ctypes.POINTER(I64)]
+        lib.attn_csr_plan_size.restype = I
+        lib.attn_csr_plan.argtypes = [P, P, I, I, I, I64, P, I64, P]
+        lib.attn_csr_plan.restype = I
+        lib.attn_sparse_csr_tc_planned.argtypes = [P, P, P, P, I64, I, I, I, I, I64, I, P, P]
+        lib.attn_sparse_csr_tc_planned.restype = I
         lib.attn_merge.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, P, P, P, P, P]
         lib.attn_merge.restype = I
         lib.attn_get_last_error.argtypes = [P, ctypes.POINTER(I)]
@@ -243,6 +251,45 @@ def attn_sparse_csr_tc(q, k, v, csr_offset, csr_columns, *, B: int, H: int, S: i
                                   _ptr(csr_columns, "csr_columns", _n(B, H, nnz_cap), "int32"),
                                   int(B), int(H), int(S), int(D), int(nnz_cap), int(dtype),
                                   _ptr(out, "out", n, et), _stream(stream)), "attn_sparse_csr_tc")
+
+
+def attn_csr_plan_size(*, B: int, H: int, S: int, nnz_cap: int) -> int:
+    """Bytes of the plan of a CSR pattern of this shape (``attn_csr_plan_size`` in
+    include/attn.h); allocate that many bytes (uint8, on the device) for attn_csr_plan."""
+    lib = load_library()
+    n = ctypes.c_int64(0)
+    _check(lib.attn_csr_plan_size(int(B), int(H), int(S), int(nnz_cap), ctypes.byref(n)),
+           "attn_csr_plan_size")
+    return int(n.value)
+
+
+def attn_csr_plan(csr_offset, csr_columns, *, B: int, H: int, S: int, nnz_cap: int, plan,
+                  stream=None) -> None:
+    """Build the plan of a CSR pattern into `plan` (a uint8 device tensor of at least
+    attn_csr_plan_size bytes); see ``attn_csr_plan`` in include/attn.h."""
+    lib = load_library()
+    nb = attn_csr_plan_size(B=B, H=H, S=S, nnz_cap=nnz_cap)
+    _check(lib.attn_csr_plan(_ptr(csr_offset, "csr_offset", _n(B, H, int(S) + 1), "int32"),
+                             _ptr(csr_columns, "csr_columns", _n(B, H, nnz_cap), "int32"), int(B),
+                             int(H), int(S), int(nnz_cap), _ptr(plan, "plan", nb, "uint8"),
+                             int(plan.numel()) if plan is not None and not isinstance(plan, int) else nb,
+                             _stream(stream)), "attn_csr_plan")
+
+
+def attn_sparse_csr_tc_planned(q, k, v, plan, *, B: int, H: int, S: int, D: int, nnz_cap: int,
+                               dtype: int, out, stream=None) -> None:
+    """attn_sparse_csr_tc from a plan of the pattern (see ``attn_sparse_csr_tc_planned`` in
+    include/attn.h)."""
+    lib = load_library()
+    n = _n(B, H, S, D)
+    et = _elem(dtype)
+    nb = attn_csr_plan_size(B=B, H=H, S=S, nnz_cap=nnz_cap)
+    _check(lib.attn_sparse_csr_tc_planned(_ptr(q, "q", n, et), _ptr(k, "k", n, et), _ptr(v, "v", n, et),
+                                          _ptr(plan, "plan", nb, "uint8"),
+                                          int(plan.numel()) if plan is not None and not isinstance(plan, int) else nb,
+                                          int(B), int(H), int(S), int(D), int(nnz_cap), int(dtype),
+                                          _ptr(out, "out", n, et), _stream(stream)),
+           "attn_sparse_csr_tc_planned")
 
 
 def attn_merge(prev_out, prev_max, prev_sum, cur_out, cur_max, cur_sum, *, S: int, B: int, N: int,

@@ -12,6 +12,7 @@
 #include <mutex>
 
 #include "attn.h"
+#include "csr_plan.cuh"
 #include "launch.h"
 
 namespace {
@@ -66,7 +67,7 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 extern "C" {
 
-int attn_abi_version(void) { return (1 << 16) | 2; }  // 1.2: attn_fwd_masked, attn_sparse_csr_tc
+int attn_abi_version(void) { return (1 << 16) | 3; }  // 1.3: CSR plans (attn_csr_plan, ..._planned)
 
 const char* attn_status_string(int s) {
   switch (s) {
@@ -271,6 +272,73 @@ int attn_sparse_csr_tc(const void* q, const void* k, const void* v, const int32_
   a.dtype = dtype;
   a.nnz_cap = nnz_cap;
   a.cols_vec = csr_columns != nullptr && aligned16(csr_columns) && nnz_cap % 4 == 0;
+  a.out = out;
+  int sms = 0;
+  int rc = device_state(&a.status, &sms);
+  if (rc != ATTN_OK) return rc;
+  const cudaError_t e = sdpa::launch_sparse_csr_tc(a, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+int attn_csr_plan_size(int B, int H, int S, int64_t nnz_cap, int64_t* bytes) {
+  if (bytes == nullptr || B < 0 || H < 0 || S < 0 || nnz_cap < 0) return ATTN_ERR_INVALID;
+  if (S > 32768) return ATTN_ERR_UNSUPPORTED;
+  const int64_t n = sdpa::plan_bytes(B, H, S, nnz_cap);
+  if (n < 0) return ATTN_ERR_UNSUPPORTED;
+  *bytes = n;
+  return ATTN_OK;
+}
+
+int attn_csr_plan(const int32_t* csr_offset, const int32_t* csr_columns, int B, int H, int S,
+                  int64_t nnz_cap, void* plan, int64_t plan_bytes, void* stream) {
+  int64_t need = 0;
+  const int rc0 = attn_csr_plan_size(B, H, S, nnz_cap, &need);
+  if (rc0 != ATTN_OK) return rc0;
+  if ((int64_t)B * H * S == 0) return ATTN_OK;
+  if (csr_offset == nullptr || plan == nullptr) return ATTN_ERR_INVALID;
+  if (nnz_cap > 0 && csr_columns == nullptr) return ATTN_ERR_INVALID;
+  if (plan_bytes < need || !aligned16(plan)) return ATTN_ERR_INVALID;
+  sdpa::CsrPlanArgs a{};
+  a.offset = csr_offset;
+  a.columns = csr_columns;
+  a.B = B;
+  a.H = H;
+  a.S = S;
+  a.nnz_cap = nnz_cap;
+  a.cols_vec = csr_columns != nullptr && aligned16(csr_columns) && nnz_cap % 4 == 0;
+  a.plan = static_cast<uint8_t*>(plan);
+  int sms = 0;
+  int rc = device_state(&a.status, &sms);
+  if (rc != ATTN_OK) return rc;
+  const cudaError_t e = sdpa::launch_csr_plan(a, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+int attn_sparse_csr_tc_planned(const void* q, const void* k, const void* v, const void* plan,
+                               int64_t plan_bytes, int B, int H, int S, int D, int64_t nnz_cap,
+                               int dtype, void* out, void* stream) {
+  if (dtype != ATTN_BF16 && dtype != ATTN_F16) return ATTN_ERR_INVALID;
+  int64_t need = 0;
+  const int rc0 = attn_csr_plan_size(B, H, S, nnz_cap, &need);
+  if (rc0 != ATTN_OK) return rc0;
+  if (D < 1) return ATTN_ERR_INVALID;
+  if ((int64_t)B * H * S == 0) return ATTN_OK;
+  if (q == nullptr || k == nullptr || v == nullptr || out == nullptr || plan == nullptr)
+    return ATTN_ERR_INVALID;
+  if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
+  if (plan_bytes < need || !aligned16(plan)) return ATTN_ERR_INVALID;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return ATTN_ERR_INVALID;
+  sdpa::CsrTcArgs a{};
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.plan = static_cast<const uint8_t*>(plan);
+  a.B = B;
+  a.H = H;
+  a.S = S;
+  a.D = D;
+  a.dtype = dtype;
+  a.nnz_cap = nnz_cap;
   a.out = out;
   int sms = 0;
   int rc = device_state(&a.status, &sms);

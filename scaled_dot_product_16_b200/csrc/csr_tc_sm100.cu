@@ -29,6 +29,7 @@
 #include <math.h>
 
 #include "common.cuh"
+#include "csr_plan.cuh"
 #include "csr_union.cuh"
 #include "launch.h"
 #include "sm100.cuh"
@@ -129,7 +130,9 @@ __device__ __forceinline__ void gather_tile(uint32_t dst, RowFn src_row, const u
   }
 }
 
-template <int HD, bool F16>
+// PLANNED: the union list, the rows' marks and the bad rows come from a plan of the pattern
+// (csr_plan.cuh) instead of being built here; the block then only gathers and multiplies.
+template <int HD, bool F16, bool PLANNED>
 __global__ void __launch_bounds__(kThreads, 1) csr_tc_kernel(CsrTcArgs a, float scale_log2) {
   using C = CsrCfg<HD, F16>;
   extern __shared__ uint8_t smem_raw[];
@@ -149,8 +152,8 @@ __global__ void __launch_bounds__(kThreads, 1) csr_tc_kernel(CsrTcArgs a, float 
   const int tiles_q = (S + kRows - 1) / kRows;
   const int64_t bh = blockIdx.x / tiles_q;
   const int r0 = (int)(blockIdx.x - bh * tiles_q) * kRows;
-  const int32_t* off = a.offset + bh * (int64_t)(S + 1);
-  const int32_t* cols = a.columns + bh * a.nnz_cap;
+  const int32_t* off = PLANNED ? nullptr : a.offset + bh * (int64_t)(S + 1);
+  const int32_t* cols = PLANNED ? nullptr : a.columns + bh * a.nnz_cap;
   const uint16_t* Qb = static_cast<const uint16_t*>(a.q) + bh * (int64_t)S * HD;
   const uint16_t* Kb = static_cast<const uint16_t*>(a.k) + bh * (int64_t)S * HD;
   const uint16_t* Vb = static_cast<const uint16_t*>(a.v) + bh * (int64_t)S * HD;
@@ -176,7 +179,8 @@ __global__ void __launch_bounds__(kThreads, 1) csr_tc_kernel(CsrTcArgs a, float 
     tmem_alloc(smem_u32(&bars->tmem_base), kTmemCols);
     tmem_relinquish();
   }
-  for (int w = threadIdx.x; w < nw * 8; w += kThreads) reinterpret_cast<uint32_t*>(bytes)[w] = 0u;
+  if constexpr (!PLANNED)
+    for (int w = threadIdx.x; w < nw * 8; w += kThreads) reinterpret_cast<uint32_t*>(bytes)[w] = 0u;
   for (int x = threadIdx.x; x < kRows; x += kThreads) row_bad[x] = 0;
   tc_fence_before();
   __syncthreads();
@@ -184,11 +188,35 @@ __global__ void __launch_bounds__(kThreads, 1) csr_tc_kernel(CsrTcArgs a, float 
   const uint32_t tmem = bars->tmem_base;
   volatile int* abort = &bars->abort;
 
-  // ---- the union of the block's rows' columns (csr_union.cuh) ---------------------------------
+  // ---- the union of the block's rows' columns (csr_union.cuh), or the plan's ------------------
   const int r = warp * 32 + lane;
   const int i = r0 + r;
-  const CsrUnion un{bitmap, wpre, bytes, row_c0, row_c1, row_bad, misc};
-  const int U = csr_block_union<kThreads, kRows>(un, off, cols, S, r0, a.nnz_cap, a.cols_vec, a.status);
+  const int32_t* plan_cols = nullptr;  // PLANNED: the block's union list
+  const uint4* plan_marks = nullptr;   // PLANNED: [tile][row] marks
+  int U;
+  if constexpr (PLANNED) {
+    const int64_t ucap = plan_ucap(S, a.nnz_cap);
+    const uint8_t* rec = a.plan + (int64_t)blockIdx.x * plan_block_bytes(S, a.nnz_cap);
+    plan_cols = reinterpret_cast<const int32_t*>(rec + kPlanHeader);
+    plan_marks = reinterpret_cast<const uint4*>(rec + kPlanHeader + 4 * ucap);
+    if (threadIdx.x < kRows) {
+      const PlanHeader* h = reinterpret_cast<const PlanHeader*>(rec);
+      // a record that is not a plan of this shape gives zeros and ATTN_ERR_DATA, and nothing
+      // it holds is used as an index
+      const bool valid = h->magic == kPlanMagic && h->S == S && h->ucap == (int32_t)ucap &&
+                         h->U >= 0 && h->U <= ucap;
+      row_bad[threadIdx.x] = !valid || ((h->bad[threadIdx.x >> 5] >> (threadIdx.x & 31)) & 1u);
+      if (threadIdx.x == 0) {
+        misc[0] = valid ? h->U : 0;
+        if (!valid) report(a.status, ATTN_ERR_DATA);
+      }
+    }
+    __syncthreads();
+    U = misc[0];
+  } else {
+    const CsrUnion un{bitmap, wpre, bytes, row_c0, row_c1, row_bad, misc};
+    U = csr_block_union<kThreads, kRows>(un, off, cols, S, r0, a.nnz_cap, a.cols_vec, a.status);
+  }
   const int T = (U + kKeys - 1) / kKeys;  // gathered key tiles
 
   const uint32_t sQ = smem_u32(smem + C::kQOff);
@@ -215,7 +243,16 @@ __global__ void __launch_bounds__(kThreads, 1) csr_tc_kernel(CsrTcArgs a, float 
 #pragma unroll
       for (int m = 0; m < kKeys / 32; ++m) {
         const int u = t * kKeys + m * 32 + lane;
-        kc[m * 32 + lane] = u < U ? union_col(u) : -1;
+        if constexpr (PLANNED) {
+          int c = u < U ? __ldg(plan_cols + u) : -1;
+          if (c >= S) {  // not a column of this pattern: the plan was built for another one
+            report(a.status, ATTN_ERR_DATA);
+            c = -1;
+          }
+          kc[m * 32 + lane] = c;
+        } else {
+          kc[m * 32 + lane] = u < U ? union_col(u) : -1;
+        }
       }
       __syncwarp();
       gather_tile<HD>(sK(s), [&](int k) { return kc[k] >= 0 ? Kb + (int64_t)kc[k] * HD : nullptr; }, Kb, lane);
@@ -278,7 +315,9 @@ __global__ void __launch_bounds__(kThreads, 1) csr_tc_kernel(CsrTcArgs a, float 
     float m = -INFINITY, l = 0.f;
     bool ok = true;
     for (int t = 0; t < T; ++t) {
-      if ((t * kKeys) % C::kWin == 0) {
+      uint4 pmark = make_uint4(0u, 0u, 0u, 0u);
+      if constexpr (PLANNED) pmark = __ldg(plan_marks + (int64_t)t * kRows + r);  // before the waits
+      if (!PLANNED && (t * kKeys) % C::kWin == 0) {
         // this row's bytes for union columns [t*128, t*128 + kWin): the thread reads its own
         // row's columns (16 at a time) and marks its own bytes, so no other thread is involved
         const int base = t * kKeys;
@@ -326,7 +365,15 @@ __global__ void __launch_bounds__(kThreads, 1) csr_tc_kernel(CsrTcArgs a, float 
 #pragma unroll
       for (int c = 0; c < 4; ++c) tmem_ld32f(Sa + c * 32, s[c]);
       tmem_wait_ld();
-      {
+      if constexpr (PLANNED) {
+        // this row's marks for the tile's 128 union columns: bit c of word x = column 32x + c
+        const uint32_t wd[4] = {pmark.x, pmark.y, pmark.z, pmark.w};
+#pragma unroll
+        for (int x = 0; x < 4; ++x)
+#pragma unroll
+          for (int c = 0; c < 32; ++c)
+            if (((wd[x] >> c) & 1u) == 0u) s[x][c] = -INFINITY;
+      } else {
         // this row's bytes for the tile's 128 union columns
         const uint4* mb = reinterpret_cast<const uint4*>(bytes + r * C::kWinStride + (t * kKeys) % C::kWin);
 #pragma unroll
@@ -432,26 +479,31 @@ __global__ void __launch_bounds__(kThreads, 1) csr_tc_kernel(CsrTcArgs a, float 
   }
 }
 
-template <int HD, bool F16>
+template <int HD, bool F16, bool PLANNED>
 cudaError_t launch_hd(const CsrTcArgs& a, cudaStream_t st) {
   using C = CsrCfg<HD, F16>;
-  cudaError_t e = cudaFuncSetAttribute(csr_tc_kernel<HD, F16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       C::kSmemBytes);
+  auto kernel = csr_tc_kernel<HD, F16, PLANNED>;
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return e;
   const int64_t blocks = (int64_t)a.B * a.H * ((a.S + kRows - 1) / kRows);
   if (blocks <= 0) return cudaSuccess;
   if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
   const float scale_log2 = (1.0f / sqrtf((float)HD)) * 1.4426950408889634f;
-  csr_tc_kernel<HD, F16><<<(unsigned)blocks, kThreads, C::kSmemBytes, st>>>(a, scale_log2);
+  kernel<<<(unsigned)blocks, kThreads, C::kSmemBytes, st>>>(a, scale_log2);
   return cudaGetLastError();
+}
+
+template <bool PLANNED>
+cudaError_t launch_tc(const CsrTcArgs& a, cudaStream_t st) {
+  const bool f16 = a.dtype == ATTN_F16;
+  if (a.D == 128) return f16 ? launch_hd<128, true, PLANNED>(a, st) : launch_hd<128, false, PLANNED>(a, st);
+  return f16 ? launch_hd<64, true, PLANNED>(a, st) : launch_hd<64, false, PLANNED>(a, st);
 }
 
 }  // namespace
 
 cudaError_t launch_sparse_csr_tc(const CsrTcArgs& a, cudaStream_t st) {
-  const bool f16 = a.dtype == ATTN_F16;
-  if (a.D == 128) return f16 ? launch_hd<128, true>(a, st) : launch_hd<128, false>(a, st);
-  return f16 ? launch_hd<64, true>(a, st) : launch_hd<64, false>(a, st);
+  return a.plan != nullptr ? launch_tc<true>(a, st) : launch_tc<false>(a, st);
 }
 
 }  // namespace sdpa

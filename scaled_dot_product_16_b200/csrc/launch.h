@@ -45,12 +45,23 @@ struct CsrTcArgs {  // attn_sparse_csr_tc: 16-bit q, k, v, out [B, H, S, D]
   const void* q;
   const void* k;
   const void* v;
-  const int32_t* offset;
-  const int32_t* columns;
+  const int32_t* offset;   // unused with a plan
+  const int32_t* columns;  // unused with a plan
+  const uint8_t* plan;     // a plan of the pattern (csr_plan.cuh), or null: build per block
   int B, H, S, D, dtype;
   int64_t nnz_cap;
   bool cols_vec;  // columns 16-byte aligned and nnz_cap % 4 == 0: read 4 indices at a time
   void* out;
+  int* status;
+};
+
+struct CsrPlanArgs {  // attn_csr_plan: the pattern of a CSR call and the plan buffer to fill
+  const int32_t* offset;
+  const int32_t* columns;
+  int B, H, S;
+  int64_t nnz_cap;
+  bool cols_vec;
+  uint8_t* plan;
   int* status;
 };
 
@@ -76,5 +87,6 @@ cudaError_t launch_sparse_csr(const CsrArgs& a, cudaStream_t st);
 bool sparse_csr_tiled_supported(const CsrArgs& a);
 cudaError_t launch_sparse_csr_tiled(const CsrArgs& a, cudaStream_t st);
 cudaError_t launch_sparse_csr_tc(const CsrTcArgs& a, cudaStream_t st);
+cudaError_t launch_csr_plan(const CsrPlanArgs& a, cudaStream_t st);
 
 }  // namespace sdpa

@@ -44,8 +44,8 @@ def pytest_terminal_summary(terminalreporter, exitstatus, config):
     for f, a in sorted(by_file.items()):
         tr.write_line(f"{f}: {a['checks']} checks, {a['n']} elements; 16-bit max |err| "
                       f"{a['max_abs_bf16_f16']:.3g} ({a['max_abs_below_4']:.3g} where |exact| < 4), "
-                      f"{a['n_over_1e-2']} above 1e-2 (all need |exact| >= 4: "
-                      f"{a['n_at_or_above_4']} such elements); fp32 max |err| {a['max_abs_f32']:.3g}")
+                      f"{a['n_over_1e-2']} above 1e-2, each within its bound; {a['n_at_or_above_4']} elements with "
+                      f"|exact| >= 4; fp32 max |err| {a['max_abs_f32']:.3g}")
     for r in rep:
         if any(k in r["test"] for k in ("cfg1", "cfg2", "cfg3", "cfg4", "cfg5", "ring_cfg5")):
             tr.write_line(f"  {r['test']} [{r['what']}, {r['dtype']}]: n={r['n']} max|err|={r['max_abs']:.3g} "

@@ -2,14 +2,17 @@
 float64 oracle under the stated tolerances, with guard regions around every output.
 
 Tolerances (written here, used by every parity test):
-  * bf16 and fp16 outputs: |gpu - exact| <= 1e-2 wherever |exact| < 4. Only where |exact| >= 4,
-    where the output's own rounding can already exceed 1e-2 (bf16 spacing is 2^-5 on [4, 8)),
-    the bound is max(1e-2, ulp(exact) / 2 + c * A) with A = sum_j w_j |v_j| (the softmax-
-    weighted mean of |v| in that element's column, which the oracle gives when it is handed |V|)
-    and c = u_P + 2^-13 + 2^-12: u_P (2^-8 for bf16, 2^-11 for fp16) bounds the rounding of the
-    probabilities P the kernel feeds to the P.V product, 2^-13 its exp2 (the polynomial's relative
-    error is 7.5e-5), and 2^-12 the fp32 accumulation over at most 65,536 keys (a rounding of
-    2^-24 per 16-key product step). Each of the three bounds |sum_j w_j e_j v_j| <= e * A.
+  * bf16 and fp16 outputs: |gpu - exact| <= max(1e-2, ulp(exact) / 2 + c * A), where ulp(exact)/2
+    is the output's own rounding and c * A bounds what the kernel's arithmetic adds before it:
+    A = sum_j w_j |v_j| (the softmax-weighted mean of |v| in that element's column, which the
+    oracle gives when it is handed |V|) and c = u_P + 2^-13 + 2^-12, with u_P (2^-8 for bf16,
+    2^-11 for fp16) the relative rounding of the probabilities P the tensor cores multiply with V
+    (a 16-bit operand), 2^-13 the relative error of the kernel's exp2 (its polynomial's is
+    7.5e-5), and 2^-12 the fp32 accumulation over at most 65,536 keys (a rounding of 2^-24 per
+    16-key product step); each bounds |sum_j w_j e_j v_j| <= e * A. The bound exceeds 1e-2 only
+    in rows dominated by a few large |v| (few visible keys, or |exact| >= 4 where bf16's own
+    spacing is 2^-5); A is computed only for elements whose error is above 1e-2, and every such
+    element is counted in the report.
   * fp32 outputs: |gpu - exact| <= 1e-5.
   * softmax max: |gpu - exact| <= 1e-3 * max(1, |exact|); softmax sum: relative 1e-3. Rows that
     see no key must give max = -inf and sum = 0 on both sides.
@@ -40,7 +43,7 @@ from scaled_dot_product_16_b200 import workloads as W
 BF16_ABS = 1e-2
 F32_ABS = 1e-5
 STAT_REL = 1e-3
-BIG = 4.0                                   # |exact| from which rounding alone can pass 1e-2
+BIG = 4.0                                   # |exact| from which bf16's own rounding can pass 1e-2
 UNIT_P = {W.BF16: 2.0 ** -8, W.F16: 2.0 ** -11}
 EXP2_REL = 2.0 ** -13
 ACC_REL = 2.0 ** -12
@@ -83,14 +86,15 @@ def check_out(gpu: np.ndarray, ref: np.ndarray, dtype: int, what: str = "out", a
     extra = {}
     if dtype in (W.BF16, W.F16):
         tol = np.full(ref.shape, BF16_ABS)
-        big = np.abs(ref) >= BIG
-        if big.any():
+        over = err > BF16_ABS
+        if over.any():
             A = abs_ref() if callable(abs_ref) else abs_ref
-            assert A is not None, f"{what}: elements with |exact| >= {BIG} need the oracle's A"
+            assert A is not None, f"{what}: {int(over.sum())} elements above 1e-2 and no A to bound them"
             A = np.asarray(A, np.float64)
-            half = (bf16_ulp(ref[big]) if dtype == W.BF16 else f16_ulp(ref[big])) / 2
-            tol[big] = np.maximum(BF16_ABS, half + (UNIT_P[dtype] + EXP2_REL + ACC_REL) * A[big])
-            extra["max_err_over_half_ulp_at_or_above_4"] = float(np.max(err[big] / half))
+            half = (bf16_ulp(ref[over]) if dtype == W.BF16 else f16_ulp(ref[over])) / 2
+            bound = half + (UNIT_P[dtype] + EXP2_REL + ACC_REL) * A[over]
+            tol[over] = np.maximum(BF16_ABS, bound)
+            extra["max_err_over_bound_above_1e-2"] = float(np.max(err[over] / bound))
     else:
         tol = np.full(ref.shape, F32_ABS)
     bad = ~(err <= tol)
@@ -101,21 +105,26 @@ def check_out(gpu: np.ndarray, ref: np.ndarray, dtype: int, what: str = "out", a
 
 
 def check_rne(gpu: torch.Tensor, ref: np.ndarray, dtype: int, eps: np.ndarray, what: str = "out") -> dict:
-    """A 16-bit result computed in fp32 and rounded once: its bits must be the oracle's rounding
-    of the exact value, or (where a rounding midpoint lies within eps of the exact value, eps
-    bounding the fp32 arithmetic's error) the rounding of exact +- eps."""
+    """A 16-bit result computed in fp32 and rounded once: its value must be the rounding of a
+    value within eps of the exact one (eps bounding the fp32 arithmetic's error), that is, lie
+    between the roundings of exact - eps and exact + eps. Where no rounding boundary falls in
+    that window the two are the same value and the result must be bit for bit the rounding of
+    the exact value."""
     rnd = oracle.round_bf16 if dtype == W.BF16 else oracle.round_f16
+    tdt = torch.bfloat16 if dtype == W.BF16 else torch.float16
     ref = np.asarray(ref, np.float64)
-    got = gpu.contiguous().view(torch.int16).numpy().view(np.uint16)
+
+    def value(bits):
+        return torch.from_numpy(bits.view(np.int16)).view(tdt).to(torch.float64).numpy()
+
+    got_bits = gpu.contiguous().view(torch.int16).numpy().view(np.uint16)
     want, lo, hi = rnd(ref), rnd(ref - eps), rnd(ref + eps)
-    ok = (got == want) | (got == lo) | (got == hi)
-    widened = (W.BF16, W.F16)
-    g64 = gpu.to(torch.float64).numpy()
-    info = _record(what, dtype, np.abs(g64 - ref), ref, {
-        "n_not_bit_equal_to_rne": int((got != want).sum()),
-        "n_near_midpoint": int((lo != hi).sum())})
-    assert dtype in widened
-    assert ok.all(), f"{what}: {int((~ok).sum())} elements are not the rounding of the exact value"
+    got, lo_v, hi_v = value(got_bits), value(lo), value(hi)
+    ok = (got_bits == want) | ((got >= lo_v) & (got <= hi_v))
+    info = _record(what, dtype, np.abs(got - ref), ref, {
+        "n_not_bit_equal_to_rne": int((got_bits != want).sum()),
+        "n_window_holds_a_boundary": int((lo != hi).sum())})
+    assert ok.all(), f"{what}: {int((~ok).sum())} elements are not the rounding of a value within eps"
     return info
 
 

@@ -283,3 +283,28 @@ def test_accumulate_refuses_unaligned_statistics(lib):
     assert call(20, 16, sdpa.ATTN_BF16) == sdpa.ATTN_ERR_INVALID
     assert call(16, 36, sdpa.ATTN_F16) == sdpa.ATTN_ERR_INVALID
     assert call(24, 40, sdpa.ATTN_BF16) == sdpa.ATTN_ERR_INVALID
+
+
+def test_plan_size_and_validation_without_gpu(lib):
+    import ctypes
+    n = ctypes.c_int64(0)
+    assert lib.attn_csr_plan_size(2, 8, 4096, 1278208, ctypes.byref(n)) == sdpa.ATTN_OK
+    # 2*8 slices x 32 row blocks x (64 + 20 * 4096) bytes
+    assert n.value == 2 * 8 * 32 * (64 + 20 * 4096)
+    assert lib.attn_csr_plan_size(1, 1, 300, 10, ctypes.byref(n)) == sdpa.ATTN_OK
+    assert n.value == 3 * (64 + 20 * 128)             # ucap = 10 rounded up to 128
+    assert lib.attn_csr_plan_size(1, 1, 32769, 10, ctypes.byref(n)) == sdpa.ATTN_ERR_UNSUPPORTED
+    assert lib.attn_csr_plan_size(-1, 1, 8, 10, ctypes.byref(n)) == sdpa.ATTN_ERR_INVALID
+    assert lib.attn_csr_plan_size(1, 1, 8, 10, None) == sdpa.ATTN_ERR_INVALID
+    need = 64 + 20 * 128
+    P = 16
+    assert lib.attn_csr_plan(P, P, 1, 1, 8, 10, P, need - 1, None) == sdpa.ATTN_ERR_INVALID  # too small
+    assert lib.attn_csr_plan(P, P, 1, 1, 8, 10, 24, need, None) == sdpa.ATTN_ERR_INVALID     # unaligned
+    assert lib.attn_csr_plan(None, P, 1, 1, 8, 10, P, need, None) == sdpa.ATTN_ERR_INVALID
+    assert lib.attn_csr_plan(P, P, 0, 1, 8, 10, P, 0, None) == sdpa.ATTN_OK                  # empty
+    tcp = lib.attn_sparse_csr_tc_planned
+    assert tcp(P, P, P, P, need, 1, 1, 8, 64, 10, sdpa.ATTN_F32, P, None) == sdpa.ATTN_ERR_INVALID
+    assert tcp(P, P, P, P, need, 1, 1, 8, 96, 10, sdpa.ATTN_BF16, P, None) == sdpa.ATTN_ERR_UNSUPPORTED
+    assert tcp(P, P, P, P, need - 16, 1, 1, 8, 64, 10, sdpa.ATTN_BF16, P, None) == sdpa.ATTN_ERR_INVALID
+    assert tcp(P, P, P, None, need, 1, 1, 8, 64, 10, sdpa.ATTN_BF16, P, None) == sdpa.ATTN_ERR_INVALID
+    assert tcp(P, P, P, P, need, 0, 1, 8, 64, 10, sdpa.ATTN_BF16, P, None) == sdpa.ATTN_OK

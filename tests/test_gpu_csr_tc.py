@@ -189,3 +189,126 @@ def test_validation():
         qf = q.float()
         sdpa.attn_sparse_csr_tc(qf, qf, qf, off, cols, B=1, H=1, S=8, D=96, nnz_cap=1, dtype=W.F32, out=qf)
     assert e.value.status == sdpa.ATTN_ERR_INVALID
+
+
+# ---- plans: the pattern's bookkeeping once, then calls that only gather and multiply ---------
+def _plan(off, cols, B, H, S):
+    """Build the plan of a pattern on the device (inside a guarded buffer). Returns (plan
+    tensor, guard, device status of the plan call)."""
+    nbytes = sdpa.attn_csr_plan_size(B=B, H=H, S=S, nnz_cap=cols.shape[-1])
+    g = G.Guarded((nbytes,), torch.uint8, fill=False)
+    sdpa.attn_csr_plan(torch.from_numpy(np.ascontiguousarray(off, np.int32)).cuda(),
+                       torch.from_numpy(np.ascontiguousarray(cols, np.int32)).cuda(),
+                       B=B, H=H, S=S, nnz_cap=cols.shape[-1], plan=g.t)
+    st = sdpa.attn_get_last_error()
+    g.check("plan")
+    return g.t, st
+
+
+def _run_planned(q, k, v, plan, B, H, S, D, nnz_cap):
+    dq, dk, dv = (torch.as_tensor(x).cuda().contiguous() for x in (q, k, v))
+    out = G.guarded_like(dq)
+    sdpa.attn_sparse_csr_tc_planned(dq, dk, dv, plan, B=B, H=H, S=S, D=D, nnz_cap=nnz_cap,
+                                    dtype=W.dtype_code(dq.dtype), out=out.t)
+    st = sdpa.attn_get_last_error()
+    out.check("planned out")
+    return out.t.cpu(), st
+
+
+@pytest.mark.parametrize("dtype", [BF, F16], ids=["bf16", "f16"])
+@pytest.mark.parametrize("D", [64, 128])
+def test_planned_equals_per_call_union(dtype, D):
+    """The planned call gives bit for bit the result of the call that builds the union itself
+    (same union order, same marks), and both agree with the oracle; the plan is built once and
+    serves two different sets of inputs."""
+    rng = np.random.default_rng(70 + D)
+    B, H, S = 2, 3, 333
+    off, cols = _distinct_pattern(rng, B, H, S, 60, empty_every=7)
+    plan, st = _plan(off, cols, B, H, S)
+    assert st == 0
+    for seed in (D, D + 1):
+        q, k, v = _inputs(B, H, S, D, dtype, seed)
+        got, st = _run_planned(q, k, v, plan, B, H, S, D, cols.shape[-1])
+        assert st == 0
+        want, st = _run(q, k, v, off, cols, B, H, S, D)
+        assert st == 0
+        assert torch.equal(got, want)
+        ref = oracle.sparse_csr(q, k, v, off, cols, B=B, H=H, S=S, D=D)
+        G.check_out(G.f64(got), ref, W.dtype_code(dtype), "planned out",
+                    abs_ref=_abs_ref(q, k, v, off, cols, B, H, S, D))
+
+
+@pytest.mark.parametrize("D", [64, 128])
+def test_planned_union_wider_than_one_window(D):
+    """Rows of up to 150 random columns over 2,560 keys: unions of about 2,000 columns, so the
+    plan's marks are built over two windows of 2,048 union columns."""
+    rng = np.random.default_rng(5 + D)
+    B, H, S = 1, 2, 2560
+    off, cols = _distinct_pattern(rng, B, H, S, 150)
+    plan, st = _plan(off, cols, B, H, S)
+    assert st == 0
+    q, k, v = _inputs(B, H, S, D, BF, 5)
+    got, st = _run_planned(q, k, v, plan, B, H, S, D, cols.shape[-1])
+    assert st == 0
+    ref = oracle.sparse_csr(q, k, v, off, cols, B=B, H=H, S=S, D=D)
+    G.check_out(G.f64(got), ref, W.BF16, "planned wide union", abs_ref=_abs_ref(q, k, v, off, cols, B, H, S, D))
+
+
+def test_planned_cfg4_full_size_bf16():
+    """Configuration 4's shape and pattern (B=2, H=8, S=4096, D=64, window 256 + every 64th
+    column) in bf16 from a plan: every row against the oracle."""
+    inp = W.cfg4_csr(seed=0)
+    q, k, v = (x.to(BF) for x in (inp.q, inp.k, inp.v))
+    plan, st = _plan(inp.offset, inp.columns, inp.B, inp.H, inp.S)
+    assert st == 0
+    got, st = _run_planned(q, k, v, plan, inp.B, inp.H, inp.S, inp.D, inp.nnz_cap)
+    assert st == 0
+    ref = oracle.sparse_csr(q, k, v, inp.offset, inp.columns, B=inp.B, H=inp.H, S=inp.S, D=inp.D)
+    G.check_out(G.f64(got), ref, W.BF16, "planned cfg4",
+                abs_ref=_abs_ref(q, k, v, inp.offset, inp.columns, inp.B, inp.H, inp.S, inp.D))
+
+
+def test_planned_data_errors_zero_only_the_bad_rows():
+    B, H, S, D = 1, 1, 300, 64
+    q, k, v = _inputs(B, H, S, D, BF, 12)
+    offs, c = W.window_stride_pattern(S, half_window=8, stride=100)
+    off = offs.reshape(1, 1, -1).copy()
+    cols = c.reshape(1, 1, -1).copy()
+    ref = oracle.sparse_csr(q, k, v, off, cols, B=B, H=H, S=S, D=D)
+    bad = cols.copy()
+    bad[0, 0, off[0, 0, 20]] = S                       # row 20: a column out of range
+    bad[0, 0, off[0, 0, 150] + 1] = bad[0, 0, off[0, 0, 150]]  # row 150: a column stored twice
+    plan, st = _plan(off, bad, B, H, S)
+    assert st == sdpa.ATTN_ERR_DATA
+    out, st = _run_planned(q, k, v, plan, B, H, S, D, cols.shape[-1])
+    assert st == 0
+    assert torch.all(out[0, 0, 20] == 0) and torch.all(out[0, 0, 150] == 0)
+    keep = np.ones(S, bool)
+    keep[[20, 150]] = False
+    absr = oracle.sparse_csr(q, k, v.abs(), off, cols, B=B, H=H, S=S, D=D)
+    G.check_out(G.f64(out)[0, 0, keep], ref[0, 0, keep], W.BF16, "other rows", abs_ref=absr[0, 0, keep])
+
+
+def test_buffer_that_is_not_a_plan_is_refused_on_the_device():
+    """A buffer of the right size that no attn_csr_plan call filled (all zeros), or a plan built
+    for another key count, is not used: every row is written as zeros and ATTN_ERR_DATA is set."""
+    B, H, S, D = 1, 2, 300, 64
+    offs, c = W.window_stride_pattern(S)
+    off = np.broadcast_to(offs, (B, H, S + 1)).copy()
+    cols = np.broadcast_to(c, (B, H, c.shape[0])).copy()
+    q, k, v = _inputs(B, H, S, D, BF, 13)
+    nbytes = sdpa.attn_csr_plan_size(B=B, H=H, S=S, nnz_cap=cols.shape[-1])
+    zero = torch.zeros(nbytes, dtype=torch.uint8, device="cuda")
+    out, st = _run_planned(q, k, v, zero, B, H, S, D, cols.shape[-1])
+    assert st == sdpa.ATTN_ERR_DATA and torch.all(out == 0)
+    # a plan of the same pattern cut to 290 keys has another S in every record
+    S2 = 290
+    offs2, c2 = W.window_stride_pattern(S2)
+    off2 = np.broadcast_to(offs2, (B, H, S2 + 1)).copy()
+    cols2 = np.broadcast_to(c2, (B, H, c2.shape[0])).copy()
+    plan2, st = _plan(off2, cols2, B, H, S2)
+    assert st == 0
+    big = torch.zeros(max(nbytes, plan2.numel()), dtype=torch.uint8, device="cuda")
+    big[:plan2.numel()].copy_(plan2)
+    out, st = _run_planned(q, k, v, big, B, H, S, D, cols.shape[-1])
+    assert st == sdpa.ATTN_ERR_DATA and torch.all(out == 0)
