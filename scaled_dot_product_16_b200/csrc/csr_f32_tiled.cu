@@ -46,7 +46,7 @@ constexpr int kPStride = kKeys + 2;          // padded row of P: a warp's 4 rows
 template <int D>
 struct F32Cfg {
   static constexpr int kKStride = D + 4;  // floats per staged key row (16-byte groups: key k -> k mod 8)
-  static constexpr int kQsOff = 0;                                    // float Qs[kRows][D], scaled
+  static constexpr int kQsOff = 0;                                    // float Qt[D][kRows], scaled
   static constexpr int kKsOff = kQsOff + kRows * D * 4;               // float Ks[2][kKeys][kKStride]
   static constexpr int kVsOff = kKsOff + 2 * kKeys * kKStride * 4;    // float Vs[2][kKeys][D]
   static constexpr int kPsOff = kVsOff + 2 * kKeys * D * 4;           // float Ps[kRows][kPStride]
@@ -157,7 +157,7 @@ template <int D>
 __global__ void __launch_bounds__(kThreads, D == 64 ? 2 : 1) csr_f32_tiled_kernel(CsrArgs a) {
   using C = F32Cfg<D>;
   extern __shared__ __align__(16) uint8_t smem[];
-  float* Qs = reinterpret_cast<float*>(smem + C::kQsOff);
+  float* Qt = reinterpret_cast<float*>(smem + C::kQsOff);
   float* Ks = reinterpret_cast<float*>(smem + C::kKsOff);
   float* Vs = reinterpret_cast<float*>(smem + C::kVsOff);
   float* Ps = reinterpret_cast<float*>(smem + C::kPsOff);
@@ -195,12 +195,17 @@ __global__ void __launch_bounds__(kThreads, D == 64 ? 2 : 1) csr_f32_tiled_kerne
   const int U = csr_block_union<kThreads, kRows>(un, off, cols, S, r0, a.nnz_cap, a.cols_vec, a.status);
   const int T = (U + kKeys - 1) / kKeys;
 
-  // Q, scaled: Qs[r][d] = q[r0 + r][d] / sqrt(D); rows past S are zero
+  // Q, scaled and transposed: Qt[d][r] = q[r0 + r][d] / sqrt(D); rows past S are zero. With d
+  // outermost, the 4 rows a thread multiplies are one 16-byte read, and the 16 rows a warp reads
+  // at one d are 64 contiguous bytes (one wavefront; row-major, they were 4 bank-conflicting ones)
   for (int x = tid; x < kRows * (D / 4); x += kThreads) {
-    const int rr = x / (D / 4), c4 = x % (D / 4);
+    const int rr = x % kRows, c4 = x / kRows;  // consecutive threads: consecutive rows (no conflict)
     float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
     if (r0 + rr < S) v = __ldg(reinterpret_cast<const float4*>(Qb + (int64_t)(r0 + rr) * D) + c4);
-    reinterpret_cast<float4*>(Qs + rr * D)[c4] = make_float4(v.x * scale, v.y * scale, v.z * scale, v.w * scale);
+    Qt[(4 * c4 + 0) * kRows + rr] = v.x * scale;
+    Qt[(4 * c4 + 1) * kRows + rr] = v.y * scale;
+    Qt[(4 * c4 + 2) * kRows + rr] = v.z * scale;
+    Qt[(4 * c4 + 3) * kRows + rr] = v.w * scale;
   }
 
   const int rg = tid >> 3;  // rows 4rg .. 4rg+3
@@ -235,6 +240,10 @@ __global__ void __launch_bounds__(kThreads, D == 64 ? 2 : 1) csr_f32_tiled_kerne
                     min(kKeys, U - (t + 1) * kKeys), Kb, Vb);
     const float* Kt = Ks + b * (kKeys * C::kKStride);
     const float* Vt = Vs + b * (kKeys * D);
+    // A warp whose 16 rows store none of this tile's 32 union columns has nothing to add: it
+    // skips the tile's products (its softmax state and output stay as they are).
+    const uint32_t wmark = marks[(16 * warp + (lane & 15)) * kMaskStride + t % kWinTiles];
+    if (!__any_sync(0xffffffffu, wmark != 0u)) continue;
 
     // scores of rows 4rg.. against keys kg + 8j
     float sc[4][4];
@@ -242,21 +251,32 @@ __global__ void __launch_bounds__(kThreads, D == 64 ? 2 : 1) csr_f32_tiled_kerne
     for (int i = 0; i < 4; ++i)
 #pragma unroll
       for (int j = 0; j < 4; ++j) sc[i][j] = 0.f;
-#pragma unroll 4
+#pragma unroll 2
     for (int d = 0; d < D; d += 4) {
       float4 kk[4];
 #pragma unroll
       for (int j = 0; j < 4; ++j) kk[j] = *reinterpret_cast<const float4*>(Kt + (kg + 8 * j) * C::kKStride + d);
+      float4 qq[4];  // qq[dd] = rows 4rg .. 4rg+3 at d + dd
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float4 qq = *reinterpret_cast<const float4*>(Qs + (4 * rg + i) * D + d);
+      for (int dd = 0; dd < 4; ++dd) qq[dd] = *reinterpret_cast<const float4*>(Qt + (d + dd) * kRows + 4 * rg);
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          sc[i][j] = fmaf(qq.x, kk[j].x, sc[i][j]);
-          sc[i][j] = fmaf(qq.y, kk[j].y, sc[i][j]);
-          sc[i][j] = fmaf(qq.z, kk[j].z, sc[i][j]);
-          sc[i][j] = fmaf(qq.w, kk[j].w, sc[i][j]);
-        }
+      for (int j = 0; j < 4; ++j) {
+        sc[0][j] = fmaf(qq[0].x, kk[j].x, sc[0][j]);
+        sc[1][j] = fmaf(qq[0].y, kk[j].x, sc[1][j]);
+        sc[2][j] = fmaf(qq[0].z, kk[j].x, sc[2][j]);
+        sc[3][j] = fmaf(qq[0].w, kk[j].x, sc[3][j]);
+        sc[0][j] = fmaf(qq[1].x, kk[j].y, sc[0][j]);
+        sc[1][j] = fmaf(qq[1].y, kk[j].y, sc[1][j]);
+        sc[2][j] = fmaf(qq[1].z, kk[j].y, sc[2][j]);
+        sc[3][j] = fmaf(qq[1].w, kk[j].y, sc[3][j]);
+        sc[0][j] = fmaf(qq[2].x, kk[j].z, sc[0][j]);
+        sc[1][j] = fmaf(qq[2].y, kk[j].z, sc[1][j]);
+        sc[2][j] = fmaf(qq[2].z, kk[j].z, sc[2][j]);
+        sc[3][j] = fmaf(qq[2].w, kk[j].z, sc[3][j]);
+        sc[0][j] = fmaf(qq[3].x, kk[j].w, sc[0][j]);
+        sc[1][j] = fmaf(qq[3].y, kk[j].w, sc[1][j]);
+        sc[2][j] = fmaf(qq[3].z, kk[j].w, sc[2][j]);
+        sc[3][j] = fmaf(qq[3].w, kk[j].w, sc[3][j]);
       }
     }
     // online softmax per row over the 8 threads that share it
