@@ -256,6 +256,33 @@ ATTN_API int attn_sparse_csr_tc_planned(const void* q, const void* k, const void
                                         int D, int64_t nnz_cap, int dtype, void* out, void* stream);
 
 /*
+ * attn_sparse_csr_tc_noalloc -- attn_sparse_csr_tc for callers that cannot allocate device memory.
+ *
+ * The pages have no counterpart of this call; it exists for this library's users. The planned
+ * form above is the fastest, but it needs a plan buffer the caller allocates. A caller that runs
+ * inside a host application owning all GPU memory through its own pool (a plugin that is given
+ * no workspace), or on a path where cudaMalloc's possible device synchronisation or failure is
+ * not acceptable, cannot provide one. This call keeps a fixed scratch array of 48 MiB inside the
+ * library (a static device variable, held on every GPU where the library's code is loaded until
+ * the process exits), builds the plan there and runs the planned kernel. It allocates nothing
+ * and frees nothing.
+ *
+ * Arguments, layouts, limits, results and data errors are those of attn_sparse_csr_tc (the result
+ * is that of attn_sparse_csr_tc_planned on the same pattern). A pattern whose plan
+ * (attn_csr_plan_size) exceeds 48 MiB is refused with ATTN_ERR_UNSUPPORTED before any launch;
+ * workload 4's shape (B=2, H=8, S=4096, nnz_cap=1,278,208) needs 41,975,808 bytes.
+ * The first call on each device looks up the scratch array's device address with that device
+ * current; make that first call before any stream capture. Every call shares the one array:
+ * calls whose kernels can overlap on the GPU (other streams, other host threads) race on it and
+ * must be ordered by the caller. The array keeps the last call's plan; nothing in it needs to
+ * start at zero, since each call's plan kernel writes every byte its planned kernel reads.
+ */
+ATTN_API int attn_sparse_csr_tc_noalloc(const void* q, const void* k, const void* v,
+                                        const int32_t* csr_offset, const int32_t* csr_columns,
+                                        int B, int H, int S, int D, int64_t nnz_cap, int dtype,
+                                        void* out, void* stream);
+
+/*
  * attn_merge -- merge two partial attention results (the ring-attention update).
  *
  * Defined by: "npu_ring_attention_update" (MindSpeed op doc), 小算子等价计算逻辑 (equivalent

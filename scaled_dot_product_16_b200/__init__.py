@@ -22,7 +22,7 @@ __all__ = [
     "ATTN_BF16", "ATTN_F32", "ATTN_F16", "ATTN_BHSD", "ATTN_TND", "ATTN_MASK_NONE",
     "ATTN_MASK_CAUSAL_TOPLEFT", "ATTN_MASK_CAUSAL_BOTTOMRIGHT", "ATTN_MASK_BAND", "lib_path",
     "load_library", "attn_fwd_masked", "attn_sparse_csr_tc", "attn_csr_plan_size", "attn_csr_plan",
-    "attn_sparse_csr_tc_planned",
+    "attn_sparse_csr_tc_planned", "attn_sparse_csr_tc_noalloc",
 ]
 
 ATTN_OK, ATTN_ERR_INVALID, ATTN_ERR_UNSUPPORTED, ATTN_ERR_CUDA, ATTN_ERR_DATA, ATTN_ERR_TIMEOUT = range(6)
@@ -74,6 +74,8 @@ def load_library():
         lib.attn_csr_plan.restype = I
         lib.attn_sparse_csr_tc_planned.argtypes = [P, P, P, P, I64, I, I, I, I, I64, I, P, P]
         lib.attn_sparse_csr_tc_planned.restype = I
+        lib.attn_sparse_csr_tc_noalloc.argtypes = [P, P, P, P, P, I, I, I, I, I64, I, P, P]
+        lib.attn_sparse_csr_tc_noalloc.restype = I
         lib.attn_merge.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, P, P, P, P, P]
         lib.attn_merge.restype = I
         lib.attn_get_last_error.argtypes = [P, ctypes.POINTER(I)]
@@ -290,6 +292,22 @@ def attn_sparse_csr_tc_planned(q, k, v, plan, *, B: int, H: int, S: int, D: int,
                                           int(B), int(H), int(S), int(D), int(nnz_cap), int(dtype),
                                           _ptr(out, "out", n, et), _stream(stream)),
            "attn_sparse_csr_tc_planned")
+
+
+def attn_sparse_csr_tc_noalloc(q, k, v, csr_offset, csr_columns, *, B: int, H: int, S: int, D: int,
+                               nnz_cap: int, dtype: int, out, stream=None) -> None:
+    """attn_sparse_csr_tc for callers that cannot allocate device memory: the library plans the
+    pattern into its own fixed 48 MiB scratch array and runs the planned kernel (see
+    ``attn_sparse_csr_tc_noalloc`` in include/attn.h; calls that overlap on the GPU race)."""
+    lib = load_library()
+    n = _n(B, H, S, D)
+    et = _elem(dtype)
+    _check(lib.attn_sparse_csr_tc_noalloc(_ptr(q, "q", n, et), _ptr(k, "k", n, et), _ptr(v, "v", n, et),
+                                          _ptr(csr_offset, "csr_offset", _n(B, H, int(S) + 1), "int32"),
+                                          _ptr(csr_columns, "csr_columns", _n(B, H, nnz_cap), "int32"),
+                                          int(B), int(H), int(S), int(D), int(nnz_cap), int(dtype),
+                                          _ptr(out, "out", n, et), _stream(stream)),
+           "attn_sparse_csr_tc_noalloc")
 
 
 def attn_merge(prev_out, prev_max, prev_sum, cur_out, cur_max, cur_sum, *, S: int, B: int, N: int,
