@@ -279,12 +279,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int rows1 = min(kBM, w.sq - w.row0 - kBM);  // <= 0: no second tile
   const bool has1 = rows1 > 0;
   // Key tiles run from jlo (the band's first tile for the block's first row; 0 otherwise) to
-  // the tile holding each Q tile's last visible key; n0 and n1 count tiles from jlo.
+  // the tile holding each Q tile's last visible key; n0 and n1 count tiles from jlo. With the
+  // band, Q1 starts at its own first tile: s1 tiles after jlo (its first row is 128 later).
   const int jlo = EXT >= 1 ? visible_begin(a.mask_mode, w.row0, a.pre) / kBN : 0;
   const int kv_end0 = visible_end(a.mask_mode, w.row0 + rows0 - 1, w.sq, w.sk, a.next);
   const int kv_end1 = has1 ? visible_end(a.mask_mode, w.row0 + kBM + rows1 - 1, w.sq, w.sk, a.next) : 0;
   const int n0 = max((kv_end0 + kBN - 1) / kBN, jlo) - jlo;
   const int n1 = has1 ? max((kv_end1 + kBN - 1) / kBN, jlo) - jlo : n0;  // tiles loaded (n1 >= n0)
+  const int s1 = EXT >= 1 && has1 ? visible_begin(a.mask_mode, w.row0 + kBM, a.pre) / kBN - jlo : 0;
 
   const uint32_t bar_base = smem_u32(bars);
   auto bar_addr = [&](const uint64_t* p) { return smem_u32(p); };
@@ -393,13 +395,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         ok = wait_bar(bar_addr(&bars->q_full), 0, abort, a.status);
         if (ok) ok = full(0);
       }
+      // Q1 works on key tiles s1 .. n1-1 (s1 = 0 except with the band)
+      auto act1 = [&](int j) { return has1 && j >= s1; };
       if (ok && n1 > 0) {
         tc_fence_after();
         if (n0 > 0) {
           issue_qk(S0, dq0, 0);
           mma_commit(bar_addr(&bars->s_full[0]));
         }
-        if (has1) {
+        if (act1(0)) {
           issue_qk(S1, dq1, 0);
           mma_commit(bar_addr(&bars->s_full[1]));
         }
@@ -424,15 +428,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             mma_commit(bar_addr(&bars->s_full[0]));
           }
         }
-        if (has1) {
-          if (!(ok = wait_bar(bar_addr(&bars->p_ready[1]), j & 1, abort, a.status))) break;
+        if (act1(j)) {
+          if (!(ok = wait_bar(bar_addr(&bars->p_ready[1]), (j - s1) & 1, abort, a.status))) break;
           tc_fence_after();
-          issue_pv(O1, S1, iv, j > 0);
+          issue_pv(O1, S1, iv, j > s1);
           if (j == n1 - 1) mma_commit(bar_addr(&bars->o_done[1]));
         }
         release(iv);
         if (next) {
-          if (has1) {
+          if (act1(j + 1)) {
             issue_qk(S1, dq1, ik);
             mma_commit(bar_addr(&bars->s_full[1]));
           }
@@ -449,6 +453,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int q = warp >> 2;                       // Q tile of this warpgroup
     const int quarter = warp & 3;                  // TMEM lane quarter of this warp
     const int r = quarter * 32 + lane;             // row within the Q tile = TMEM lane
+    const int j0 = q == 0 ? 0 : s1;                // this Q tile's key tiles: j0 .. n-1
     const int n = q == 0 ? n0 : (has1 ? n1 : 0);
     const int rows = q == 0 ? rows0 : rows1;
     const int i = w.row0 + q * kBM + r;            // row within the sequence
@@ -467,8 +472,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     float l = 0.f;
     bool ok = true;
     if (q == 0 || has1) {
-      for (int j = 0; j < n; ++j) {
-        ok = __all_sync(0xffffffffu, wait_bar(bar_addr(&bars->s_full[q]), j & 1, abort, a.status));
+      for (int j = j0; j < n; ++j) {
+        ok = __all_sync(0xffffffffu, wait_bar(bar_addr(&bars->s_full[q]), (j - j0) & 1, abort, a.status));
         if (!ok) break;
         tc_fence_after();
         const int kbase = (jlo + j) * kBN;
@@ -569,8 +574,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         l += ((rs[0].x + rs[0].y) + (rs[1].x + rs[1].y)) + ((rs[2].x + rs[2].y) + (rs[3].x + rs[3].y));
         // rescale O (complete up to tile j-1: the S_j commit covers every earlier MMA)
-        if (__any_sync(0xffffffffu, bump && j > 0)) {
-          const float f = (bump && j > 0) ? corr : 1.f;
+        if (__any_sync(0xffffffffu, bump && j > j0)) {
+          const float f = (bump && j > j0) ? corr : 1.f;
 #pragma unroll
           for (int c = 0; c < HDV / 32; ++c) {
             uint32_t o[32];
@@ -590,7 +595,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     // ---- epilogue: O / l -> bf16, statistics ------------------------------------------------
-    const bool have_o = ok && n > 0 && (q == 0 || has1);
+    const bool have_o = ok && n > j0 && (q == 0 || has1);
     if (have_o) ok = __all_sync(0xffffffffu, wait_bar(bar_addr(&bars->o_done[q]), 0, abort, a.status));
     tc_fence_after();
     if (q == 0 || has1) {
