@@ -46,7 +46,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # default varlen batch (75,336 tokens), from a one-pass ncu capture of that launch. It is
 # reported only for that workload and while the kernel source still has the hash it was
 # measured on.
-TRAFFIC = {"kernel_sha": "3612f886071302b1", "tokens": 75_336, "bytes_per_launch": 937_927_936 + 600_918_272}
+TRAFFIC = {"kernel_sha": "2912c639f4479bce", "tokens": 75_336, "bytes_per_launch": 936_911_616 + 602_196_480}
 
 
 KERNEL_SOURCES = ("fwd_bf16_sm100.cu", "sm100.cuh", "common.cuh", "launch.h")
@@ -609,6 +609,39 @@ def run_ours(args, rank: int, world: int, local: int):
         print(json.dumps(line), flush=True)
 
 
+def run_op(args):
+    """One operation alone, `--warmup` + `--steps` times, for profiling it (no timing printed)."""
+    sdpa.load_library()
+    if args.op == "band":
+        fwd = FwdCase(W.cfg3_varlen_gqa(seed=0, max_len=args.max_len))
+        i = fwd.inp
+
+        def fn():
+            sdpa.attn_fwd_masked(fwd.q, fwd.k, fwd.v, cu_seqlens_q=fwd.cq, cu_seqlens_kv=fwd.ck, B=i.B,
+                                 Sq=i.Sq, Skv=i.Skv, Nq=i.Nq, Nkv=i.Nkv, Dqk=i.D, Dv=i.D, scale=i.scale,
+                                 mask_mode=sdpa.ATTN_MASK_BAND, pre_tokens=1023, next_tokens=0,
+                                 dtype=i.dtype, layout=i.layout, out=fwd.out, softmax_max=fwd.m,
+                                 softmax_sum=fwd.l)
+    else:  # the tensor-core CSR from a plan: each step builds the plan and runs the call
+        c = CsrCase(W.cfg4_csr(seed=0))
+        ci = c.inp
+        qb, kb, vb = (t.to(torch.bfloat16) for t in (c.q, c.k, c.v))
+        outb = torch.empty_like(qb)
+        plan = torch.empty(sdpa.attn_csr_plan_size(B=ci.B, H=ci.H, S=ci.S, nnz_cap=ci.nnz_cap),
+                           dtype=torch.uint8, device="cuda")
+
+        def fn():
+            sdpa.attn_csr_plan(c.off, c.col, B=ci.B, H=ci.H, S=ci.S, nnz_cap=ci.nnz_cap, plan=plan)
+            sdpa.attn_sparse_csr_tc_planned(qb, kb, vb, plan, B=ci.B, H=ci.H, S=ci.S, D=ci.D,
+                                            nnz_cap=ci.nnz_cap, dtype=W.BF16, out=outb)
+    for _ in range(args.warmup + args.steps):
+        fn()
+    torch.cuda.synchronize()
+    if sdpa.attn_get_last_error() != 0:
+        raise RuntimeError("device status set")
+    print(json.dumps({"op": args.op, "launches": args.warmup + args.steps}), flush=True)
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -623,9 +656,15 @@ def main(argv=None):
                     help="skip timing the ring fold, the band and the tensor-core CSR")
     ap.add_argument("--cpu-budget", type=float, default=20.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--ref-rows", type=int, default=2048, help="oracle rows per reference step")
+    ap.add_argument("--op", choices=["band", "csr_tc_planned"], default=None,
+                    help="run only this operation (for profiling it), no timing line")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
+    if args.op is not None:
+        torch.cuda.set_device(0)
+        run_op(args)
+        return
     rank, world, local = dist_setup(use_gpu=args.impl != "reference")
     try:
         if args.impl == "reference":
