@@ -88,8 +88,7 @@ __device__ __forceinline__ void stage_tile(uint32_t ks, uint32_t vs, const int* 
 }
 
 // Marks for rows of the block: bit u - W0 of row x's words is set when row x stores union column
-// u (W0 <= u < W0 + kWin). A warp per row reads the row's columns (coalesced, 32 at a time) and
-// ORs each one's bit into shared memory (atomically: lanes can hit the same word). A row that
+// u (W0 <= u < W0 + kWin), built a warp per row (csr_mark_row in csr_union.cuh). A row that
 // stores some column twice sets fewer bits than it has entries in the window: it is marked heavy.
 // Every thread of the block calls this; it ends with the marks complete.
 __device__ __forceinline__ void build_marks(uint32_t* marks, const CsrUnion& un, int* row_heavy,
@@ -98,29 +97,8 @@ __device__ __forceinline__ void build_marks(uint32_t* marks, const CsrUnion& un,
   for (int x = threadIdx.x; x < kRows * kMaskStride; x += kThreads) marks[x] = 0u;
   __syncthreads();
   for (int rr = warp; rr < kRows; rr += kThreads / 32) {
-    const int c1 = un.row_c1[rr];
-    int n = 0;
-    for (int base = un.row_c0[rr]; base < c1; base += 32) {
-      const int e = base + lane;
-      int w = -1;  // the mark word this lane sets a bit in, if any
-      uint32_t bit = 0u;
-      if (e < c1) {
-        const int j = __ldg(cols + e);
-        if (j >= 0 && j < S) {  // bad columns are already flagged; the row is zeroed
-          const int u = csr_union_index(un.bitmap, un.wpre, j) - W0;
-          if (u >= 0 && u < kWin) {
-            w = u >> 5;
-            bit = 1u << (u & 31);
-            ++n;
-          }
-        }
-      }
-      // (lanes that share a word serialise on it; grouping them first with __match_any_sync
-      // measured slower here: 0.415 against 0.372 ms on workload 4)
-      if (w >= 0) atomicOr(&marks[rr * kMaskStride + w], bit);
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) n += __shfl_xor_sync(0xffffffffu, n, o);
+    const int n = csr_mark_row(marks + rr * kMaskStride, un.bitmap, un.wpre, cols, un.row_c0[rr], un.row_c1[rr],
+                               S, W0, kWin);
     if (lane == 0) row_cnt[rr] = n;
   }
   __syncthreads();
@@ -256,24 +234,20 @@ __global__ void __launch_bounds__(kThreads, D == 64 ? 2 : 1) csr_f32_tiled_kerne
       float4 qq[4];  // qq[dd] = rows 4rg .. 4rg+3 at d + dd
 #pragma unroll
       for (int dd = 0; dd < 4; ++dd) qq[dd] = *reinterpret_cast<const float4*>(Qt + (d + dd) * kRows + 4 * rg);
+      // rows (4rg, 4rg+1) and (4rg+2, 4rg+3) as fp32 pairs: one packed FMA for two scores
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        sc[0][j] = fmaf(qq[0].x, kk[j].x, sc[0][j]);
-        sc[1][j] = fmaf(qq[0].y, kk[j].x, sc[1][j]);
-        sc[2][j] = fmaf(qq[0].z, kk[j].x, sc[2][j]);
-        sc[3][j] = fmaf(qq[0].w, kk[j].x, sc[3][j]);
-        sc[0][j] = fmaf(qq[1].x, kk[j].y, sc[0][j]);
-        sc[1][j] = fmaf(qq[1].y, kk[j].y, sc[1][j]);
-        sc[2][j] = fmaf(qq[1].z, kk[j].y, sc[2][j]);
-        sc[3][j] = fmaf(qq[1].w, kk[j].y, sc[3][j]);
-        sc[0][j] = fmaf(qq[2].x, kk[j].z, sc[0][j]);
-        sc[1][j] = fmaf(qq[2].y, kk[j].z, sc[1][j]);
-        sc[2][j] = fmaf(qq[2].z, kk[j].z, sc[2][j]);
-        sc[3][j] = fmaf(qq[2].w, kk[j].z, sc[3][j]);
-        sc[0][j] = fmaf(qq[3].x, kk[j].w, sc[0][j]);
-        sc[1][j] = fmaf(qq[3].y, kk[j].w, sc[1][j]);
-        sc[2][j] = fmaf(qq[3].z, kk[j].w, sc[2][j]);
-        sc[3][j] = fmaf(qq[3].w, kk[j].w, sc[3][j]);
+        const float kd[4] = {kk[j].x, kk[j].y, kk[j].z, kk[j].w};
+#pragma unroll
+        for (int dd = 0; dd < 4; ++dd) {
+          const float2 k2 = make_float2(kd[dd], kd[dd]);
+          float2 lo = __ffma2_rn(make_float2(qq[dd].x, qq[dd].y), k2, make_float2(sc[0][j], sc[1][j]));
+          float2 hi = __ffma2_rn(make_float2(qq[dd].z, qq[dd].w), k2, make_float2(sc[2][j], sc[3][j]));
+          sc[0][j] = lo.x;
+          sc[1][j] = lo.y;
+          sc[2][j] = hi.x;
+          sc[3][j] = hi.y;
+        }
       }
     }
     // online softmax per row over the 8 threads that share it
@@ -326,12 +300,16 @@ __global__ void __launch_bounds__(kThreads, D == 64 ? 2 : 1) csr_f32_tiled_kerne
 #pragma unroll
       for (int c = 0; c < kV4; ++c) {
         const float4 vv = *reinterpret_cast<const float4*>(Vt + k * D + 4 * kg + 32 * c);
+        // output columns (4kg + 32c, +1) and (+2, +3) as fp32 pairs
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          o[i][4 * c + 0] = fmaf(pk[i], vv.x, o[i][4 * c + 0]);
-          o[i][4 * c + 1] = fmaf(pk[i], vv.y, o[i][4 * c + 1]);
-          o[i][4 * c + 2] = fmaf(pk[i], vv.z, o[i][4 * c + 2]);
-          o[i][4 * c + 3] = fmaf(pk[i], vv.w, o[i][4 * c + 3]);
+          const float2 p2 = make_float2(pk[i], pk[i]);
+          const float2 lo = __ffma2_rn(p2, make_float2(vv.x, vv.y), make_float2(o[i][4 * c + 0], o[i][4 * c + 1]));
+          const float2 hi = __ffma2_rn(p2, make_float2(vv.z, vv.w), make_float2(o[i][4 * c + 2], o[i][4 * c + 3]));
+          o[i][4 * c + 0] = lo.x;
+          o[i][4 * c + 1] = lo.y;
+          o[i][4 * c + 2] = hi.x;
+          o[i][4 * c + 3] = hi.y;
         }
       }
     }

@@ -10,10 +10,9 @@
 //   1. the union of the rows' columns (csr_union.cuh): a byte per column from one streamed
 //      pass over the block's column indices, packed into a bitmap with a popcount prefix;
 //   2. the union list: a thread per bitmap word writes the columns of its set bits in order;
-//   3. the marks, 2,048 union columns at a time: a warp per row reads the row's columns
-//      (coalesced) and sets the bit of each one's union index in shared memory (lanes that hit
-//      the same word OR their bits together first, then one atomic OR per word: a row's columns
-//      are mostly consecutive); the window is then written out as a uint4 per
+//   3. the marks, 2,048 union columns at a time: a warp per row, each lane a contiguous run of
+//      the row's columns, ORs the bits of their union indices into register words and those
+//      into shared memory (csr_mark_row in csr_union.cuh); the window is then written out as a uint4 per
 //      (tile, row), and a row whose set bits number fewer than its entries stored a column
 //      twice, which marks cannot hold: it is flagged bad (ATTN_ERR_DATA);
 //   4. the header: magic, S, ucap, U and the bad-row bits.
@@ -86,30 +85,7 @@ __global__ void __launch_bounds__(kThreads) csr_plan_kernel(CsrPlanArgs a) {
     for (int x = tid; x < kPlanRows * kMarkStride; x += kThreads) marks[x] = 0u;
     __syncthreads();
     for (int rr = warp; rr < kPlanRows; rr += kWarps) {
-      const int c1 = row_c1[rr];
-      int n = 0;
-      for (int base = row_c0[rr]; base < c1; base += 32) {
-        const int e = base + lane;
-        int w = -1;  // the mark word this lane sets a bit in, if any
-        uint32_t bit = 0u;
-        if (e < c1) {
-          const int j = __ldg(cols + e);
-          if (j >= 0 && j < S) {  // a bad column has flagged its row already
-            const int u = csr_union_index(bitmap, wpre, j) - W0;
-            if (u >= 0 && u < kWin) {
-              w = u >> 5;
-              bit = 1u << (u & 31);
-              ++n;
-            }
-          }
-        }
-        // lanes that set bits in the same word OR them together; one atomic per word
-        const unsigned grp = __match_any_sync(0xffffffffu, w);
-        const uint32_t bits = __reduce_or_sync(grp, bit);
-        if (w >= 0 && lane == __ffs(grp) - 1) atomicOr(&marks[rr * kMarkStride + w], bits);
-      }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) n += __shfl_xor_sync(0xffffffffu, n, o);
+      const int n = csr_mark_row(marks + rr * kMarkStride, bitmap, wpre, cols, row_c0[rr], row_c1[rr], S, W0, kWin);
       if (lane == 0) row_cnt[rr] = n;
     }
     __syncthreads();
