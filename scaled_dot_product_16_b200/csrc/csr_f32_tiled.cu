@@ -21,7 +21,9 @@
 //    different bank groups); an unmarked score is left out of the online softmax.
 //  * P goes through shared memory to the P.V product (4 rows x D/8 columns per thread, columns
 //    4kg + 32c, so 8 neighbouring threads read 128 contiguous bytes of a value row).
-// All arithmetic is fp32 FMA with expf, as the row-per-warp kernel does. A row that stores some
+// All arithmetic is fp32 FMA. The softmax works in log2 units (Q is staged pre-scaled by
+// log2(e) / sqrt(D)), so each probability is one subtraction and one ex2.approx (relative error
+// about 2^-22, far inside the fp32 tolerance) instead of an expf. A row that stores some
 // column more than once (each copy weighs once, which a bit cannot hold) is recomputed exactly
 // by a row-per-warp pass at the end.
 #include <math.h>
@@ -62,6 +64,12 @@ struct F32Cfg {
   static_assert(kSmemBytes <= 232448, "227 KB of shared memory per block");
   static_assert(D != 64 || kSmemBytes <= 112 * 1024, "two blocks per SM at D = 64");
 };
+
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -159,6 +167,7 @@ __global__ void __launch_bounds__(kThreads, D == 64 ? 2 : 1) csr_f32_tiled_kerne
   const float* Vb = a.v + bh * (int64_t)S * D;
   const int nw = (S + 31) >> 5;
   const float scale = 1.0f / sqrtf((float)D);
+  const float scale2 = scale * 1.4426950408889634f;  // scores in log2 units for the tiles
 
   for (int w = tid; w < nw * 8; w += kThreads) reinterpret_cast<uint32_t*>(bytes)[w] = 0u;
   for (int x = tid; x < kRows; x += kThreads) {
@@ -170,17 +179,17 @@ __global__ void __launch_bounds__(kThreads, D == 64 ? 2 : 1) csr_f32_tiled_kerne
   const int U = csr_block_union<kThreads, kRows>(un, off, cols, S, r0, a.nnz_cap, a.cols_vec, a.status);
   const int T = (U + kKeys - 1) / kKeys;
 
-  // Q, scaled and transposed: Qt[d][r] = q[r0 + r][d] / sqrt(D); rows past S are zero. With d
+  // Q, scaled and transposed: Qt[d][r] = q[r0 + r][d] * log2(e) / sqrt(D); rows past S are zero. With d
   // outermost, the 4 rows a thread multiplies are one 16-byte read, and the 16 rows a warp reads
   // at one d are 64 contiguous bytes (one wavefront; row-major, they were 4 bank-conflicting ones)
   for (int x = tid; x < kRows * (D / 4); x += kThreads) {
     const int rr = x % kRows, c4 = x / kRows;  // consecutive threads: consecutive rows (no conflict)
     float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
     if (r0 + rr < S) v = __ldg(reinterpret_cast<const float4*>(Qb + (int64_t)(r0 + rr) * D) + c4);
-    Qt[(4 * c4 + 0) * kRows + rr] = v.x * scale;
-    Qt[(4 * c4 + 1) * kRows + rr] = v.y * scale;
-    Qt[(4 * c4 + 2) * kRows + rr] = v.z * scale;
-    Qt[(4 * c4 + 3) * kRows + rr] = v.w * scale;
+    Qt[(4 * c4 + 0) * kRows + rr] = v.x * scale2;
+    Qt[(4 * c4 + 1) * kRows + rr] = v.y * scale2;
+    Qt[(4 * c4 + 2) * kRows + rr] = v.z * scale2;
+    Qt[(4 * c4 + 3) * kRows + rr] = v.w * scale2;
   }
 
   const int rg = tid >> 3;  // rows 4rg .. 4rg+3
@@ -270,10 +279,10 @@ __global__ void __launch_bounds__(kThreads, D == 64 ? 2 : 1) csr_f32_tiled_kerne
 #pragma unroll
       for (int j = 0; j < 4; ++j) p[i][j] = 0.f;
       if (mnew != -INFINITY) {
-        corr[i] = m[i] == -INFINITY ? 0.f : expf(m[i] - mnew);
+        corr[i] = m[i] == -INFINITY ? 0.f : ex2_approx(m[i] - mnew);
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          p[i][j] = has[j] ? expf(sc[i][j] - mnew) : 0.f;
+          p[i][j] = has[j] ? ex2_approx(sc[i][j] - mnew) : 0.f;
           rs += p[i][j];
         }
       }

@@ -312,3 +312,23 @@ def test_buffer_that_is_not_a_plan_is_refused_on_the_device():
     big[:plan2.numel()].copy_(plan2)
     out, st = _run_planned(q, k, v, big, B, H, S, D, cols.shape[-1])
     assert st == sdpa.ATTN_ERR_DATA and torch.all(out == 0)
+
+
+def test_plan_is_deterministic_and_reusable():
+    """A plan depends on the pattern only: two builds of the same pattern give the same bytes
+    (the marks' atomic ORs land in any order but OR is order-free), and one plan serves any
+    number of calls with bit-identical results."""
+    rng = np.random.default_rng(91)
+    B, H, S, D = 1, 2, 700, 64
+    off, cols = _distinct_pattern(rng, B, H, S, 80)
+    p1, st1 = _plan(off, cols, B, H, S)
+    p2, st2 = _plan(off, cols, B, H, S)
+    assert st1 == 0 and st2 == 0
+    # both buffers start zeroed, so the whole plans compare, unused tails included
+    assert torch.equal(p1, p2)
+    q, k, v = _inputs(B, H, S, D, BF, 91)
+    a, sa = _run_planned(q, k, v, p1, B, H, S, D, cols.shape[-1])
+    b, sb = _run_planned(q, k, v, p1, B, H, S, D, cols.shape[-1])
+    c, sc = _run_planned(q, k, v, p2, B, H, S, D, cols.shape[-1])
+    assert sa == sb == sc == 0
+    assert torch.equal(a, b) and torch.equal(a, c)
