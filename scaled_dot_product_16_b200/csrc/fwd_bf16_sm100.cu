@@ -21,15 +21,18 @@
 //     diagonal and ragged tiles are masked element by element, rows past a sequence's end are
 //     never stored, and zero-length sequences produce no work.
 //
-// Roles (320 threads): warps 0-3 softmax Q0, warps 4-7 softmax Q1, warp 8 MMA issue,
-// warp 9 TMA producer. TMEM: S0 [0,128) S1 [128,256) O0 [256,256+D) O1 [256+D,256+2D).
+// Roles (384 threads): warps 0-3 softmax Q0, warps 4-7 softmax Q1, warp 8 MMA issue,
+// warp 9 TMA producer (warps 10-11 idle). TMEM: S0 [0,128) S1 [128,256) O0 [256,256+D) O1 [256+D,256+2D).
 //
 // Every mbarrier wait is bounded in time: if a wait runs out the block records
 // ATTN_ERR_TIMEOUT, stops issuing work, drains what it started and frees its TMEM.
 #include <cuda.h>
 #include <math.h>
 
+#include <atomic>
+#include <map>
 #include <mutex>
+#include <utility>
 
 #include "common.cuh"
 #include "launch.h"
@@ -43,9 +46,16 @@ using namespace sm100;
 constexpr int kBM = 128;          // rows per Q tile (= TMEM lanes)
 constexpr int kBN = 128;          // keys per K/V tile
 constexpr int kRowsPerBlock = 2 * kBM;
-constexpr int kThreads = 320;
+constexpr int kThreads = 384;
 constexpr int kMmaWarp = 8;
-constexpr int kTmaWarp = 9;
+constexpr int kTmaWarp = 9;       // warps 10 and 11 only complete the producer warpgroup
+// Register split: the block is launched with kRegsLaunch a thread (the limit for 384 threads,
+// which the host checks before each launch); the softmax warpgroups raise theirs to
+// kRegsSoftmax, the producer warpgroup lowers its own to kRegsProducer.
+constexpr int kRegsLaunch = 168;
+constexpr int kRegsSoftmax = 216;
+constexpr int kRegsProducer = 72;
+static_assert(256 * kRegsSoftmax + 128 * kRegsProducer <= kThreads * kRegsLaunch, "register split");
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale when the max grows by > 2^8
 // Time bounds of a barrier wait: one in the pipeline (data or a hand-off from another role),
@@ -110,7 +120,7 @@ struct Cfg {
   static constexpr int kQOff = 0;
   static constexpr int kKVOff = 2 * kTileBytes;
   static constexpr int kBarOff = kKVOff + kStages * kTileBytes;
-  static constexpr int kSmemBytes = kBarOff + 256 + 1024;  // barriers + 1 KB for alignment
+  static constexpr int kSmemBytes = kBarOff + 512 + 1024;  // barriers + 1 KB for alignment
   static_assert(kStages >= 2 && kStages <= 8, "barrier arrays hold 8 stages");
   static_assert(kSmemBytes <= 232448, "227 KB of shared memory per block");
   static constexpr uint32_t kFmt = F16 ? 0u : 1u;  // instruction-descriptor operand format
@@ -119,18 +129,46 @@ struct Cfg {
   static_assert(HDV <= HD && HDV % 64 == 0, "value head size");
 };
 
+// Work counters of the persistent grid, a pair per slot: the next item to hand out (counted
+// past the first gridDim.x items, which block x takes without asking) and the blocks finished.
+// A launch draws its items from one slot with atomicAdd; its last block to finish puts both back
+// to 0, so the next launch that uses the slot starts from 0. The host gives every stream its own
+// slot (launches on one stream run one after another), and launches that cannot be given one
+// divide the items statically instead.
+constexpr int kSchedSlots = 256;
+__device__ int g_sched[kSchedSlots * 2];
+
+// One work item decoded: 256 query rows (two 128-row tiles) of query head h of sequence b.
+struct Unit {
+  int b, h;          // sequence and query head; b < 0 marks the end of the block's work
+  int q0, sq, sk;    // first query token and query length of the sequence; its key length
+  int row0;          // first row (within the sequence) of the 256 rows
+  int rows0, rows1;  // rows of Q0 and Q1 (rows1 <= 0: no second tile)
+  int jlo;           // first key tile (the band's first tile for row0; 0 otherwise)
+  int n0, n1;        // key tiles from jlo up to Q0's / Q1's last visible key (n1 >= n0)
+  int s1;            // Q1's first key tile, counted from jlo (0 except with the band)
+};
+
+constexpr int kUnitSlots = 4;    // decoded items the TMA warp may run ahead
+constexpr int kUnitReaders = 9;  // the MMA warp and the eight softmax warps read each item
+
 struct Barriers {
   uint64_t kv_full[8];
   uint64_t kv_empty[8];
   uint64_t q_full;
+  uint64_t q_empty;  // the last S MMAs of an item have run: Q may be overwritten
   uint64_t s_full[2];
   uint64_t p_ready[2];
   uint64_t o_done[2];
   uint64_t drain;
   uint64_t stall;  // never arrived on (the test build waits on it)
+  uint64_t unit_full[kUnitSlots];   // an item (or the end mark) is in the slot
+  uint64_t unit_empty[kUnitSlots];  // every reader has taken the slot's item
+  Unit units[kUnitSlots];
   uint32_t tmem_base;
   int abort;
 };
+static_assert(sizeof(Barriers) <= 512, "the barrier area of the shared-memory layout");
 
 // Bounded wait on an mbarrier phase. Returns false (after recording a timeout, or when another
 // role of this block already gave up) instead of waiting forever.
@@ -199,112 +237,109 @@ __device__ __forceinline__ void merge_into_stats(const FwdArgs& a, int64_t so, f
   *f_o *= cs0 * inv;
 }
 
-struct Work {
-  int b, h, g;      // sequence, query head, key/value head
-  int q0, sq;       // first query token and query length of the sequence
-  int k0, sk;       // same for keys
-  int row0;         // first row (within the sequence) of this block's 256 rows
-};
+// Decodes item x. Items run query-head fastest; for BHSD the 256-row blocks go by level (the
+// last row block of every sequence first), for TND sequence by sequence with each sequence's last
+// row block first, so that the heaviest items of a sequence come first. Run by one full warp;
+// every lane gets the result. Returns false for an item past the last row block (an item there
+// with h == 0 checks the key-side cumulative lengths) and for a sequence whose keys lie outside
+// [0, Skv), recording ATTN_ERR_DATA for bad lengths.
+template <int EXT>
+__device__ __forceinline__ bool decode_unit(const FwdArgs& a, int units_per_seq, int x, Unit& U, int& k0) {
+  const int lane = threadIdx.x & 31;
+  const int h = x % a.Nq;
+  const int y = x / a.Nq;
+  int b = 0, u = 0;
+  bool ok = true;
+  if (a.layout == ATTN_BHSD) {
+    const int level = y / a.B;  // 0 = last row block of every sequence
+    b = y - level * a.B;
+    u = units_per_seq - 1 - level;
+    ok = u >= 0;
+  } else {
+    bool bad;
+    int t;
+    ok = warp_find_tile(a.cu_q, a.B, a.Sq, kRowsPerBlock, y, &b, &t, a.status, &bad);
+    if (ok) {
+      int qs, ql;
+      seq_span(a.cu_q, b, &qs, &ql);
+      u = (ql + kRowsPerBlock - 1) / kRowsPerBlock - 1 - t;
+    } else if (!bad && h == 0) {
+      int sb, st;
+      bool bad2;
+      warp_find_tile(a.cu_kv, a.B, a.Skv, 1 << 30, 1 << 30, &sb, &st, a.status, &bad2);
+    }
+  }
+  if (!ok) return false;
+  U.b = b;
+  U.h = h;
+  U.row0 = u * kRowsPerBlock;
+  if (a.layout == ATTN_BHSD) {
+    U.q0 = 0;
+    U.sq = a.Sq;
+    k0 = 0;
+    U.sk = a.Skv;
+  } else {
+    seq_span(a.cu_q, b, &U.q0, &U.sq);
+    seq_span(a.cu_kv, b, &k0, &U.sk);
+    if (k0 < 0 || U.sk < 0 || k0 + U.sk > a.Skv) {
+      if (lane == 0) report(a.status, ATTN_ERR_DATA);
+      return false;
+    }
+  }
+  U.rows0 = min(kBM, U.sq - U.row0);
+  U.rows1 = min(kBM, U.sq - U.row0 - kBM);
+  const bool has1 = U.rows1 > 0;
+  // Key tiles run from jlo to the tile holding each Q tile's last visible key; n0 and n1 count
+  // tiles from jlo. With the band, Q1 starts at its own first tile: s1 tiles after jlo.
+  U.jlo = EXT >= 1 ? visible_begin(a.mask_mode, U.row0, a.pre) / kBN : 0;
+  const int kv_end0 = visible_end(a.mask_mode, U.row0 + U.rows0 - 1, U.sq, U.sk, a.next);
+  const int kv_end1 = has1 ? visible_end(a.mask_mode, U.row0 + kBM + U.rows1 - 1, U.sq, U.sk, a.next) : 0;
+  U.n0 = max((kv_end0 + kBN - 1) / kBN, U.jlo) - U.jlo;
+  U.n1 = has1 ? max((kv_end1 + kBN - 1) / kBN, U.jlo) - U.jlo : U.n0;
+  U.s1 = EXT >= 1 && has1 ? visible_begin(a.mask_mode, U.row0 + kBM, a.pre) / kBN - U.jlo : 0;
+  return true;
+}
 
 // EXT: the masked-call features. 0: plain calls, whose softmax loop carries none of their code;
 // 1: the band's lower edge; 2: the band and an explicit mask (its bytes take registers that the
 // band alone does not need).
+//
+// Persistent: each block (one per SM) takes items one after another, from the scheduler slot
+// `sched` when there is one, else x = blockIdx.x + k * gridDim.x. The TMA warp decodes each item
+// and hands it to the MMA warp and the softmax warps through a ring of kUnitSlots shared-memory
+// slots; its loads of item u+1 (the first K/V tiles, then Q once the last S of item u has run)
+// overlap the last softmax, P.V and epilogue of item u, and the block's setup is paid once.
 template <int HD, int HDV, bool F16, int EXT>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, FwdArgs a, int units_per_seq,
-                    float scale_log2) {
+                    float scale_log2, int n_items, int* sched) {
   using C = Cfg<HD, HDV, F16>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   Barriers* bars = reinterpret_cast<Barriers*>(smem + C::kBarOff);
-  __shared__ int s_work[4];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-
-  // ---- work unit: (sequence b, 256-row block) of query head h -----------------------------
-  // Block ids run head-fastest; within a head the heaviest (last) row blocks come first.
-  const int h = (int)(blockIdx.x % (unsigned)a.Nq);
-  const int y = (int)(blockIdx.x / (unsigned)a.Nq);
-  if (warp == 0) {
-    int b = 0, u = 0, ok = 1;
-    if (a.layout == ATTN_BHSD) {
-      const int level = y / a.B;  // 0 = last row block of every sequence
-      b = y - level * a.B;
-      u = units_per_seq - 1 - level;
-      ok = u >= 0;
-    } else {
-      bool bad;
-      int t;
-      ok = warp_find_tile(a.cu_q, a.B, a.Sq, kRowsPerBlock, y, &b, &t, a.status, &bad);
-      if (ok) {
-        int qs, ql;
-        seq_span(a.cu_q, b, &qs, &ql);
-        u = (ql + kRowsPerBlock - 1) / kRowsPerBlock - 1 - t;
-      } else if (!bad && h == 0) {
-        int sb, st;
-        bool bad2;  // a block past the last unit validates the key-side lengths
-        warp_find_tile(a.cu_kv, a.B, a.Skv, 1 << 30, 1 << 30, &sb, &st, a.status, &bad2);
-      }
-    }
-    if (lane == 0) {
-      s_work[0] = ok;
-      s_work[1] = b;
-      s_work[2] = u;
-    }
-  }
-  __syncthreads();
-  if (!s_work[0]) return;
-
-  Work w;
-  w.b = s_work[1];
-  w.h = h;
-  w.g = h / (a.Nq / a.Nkv);
-  w.row0 = s_work[2] * kRowsPerBlock;
-  if (a.layout == ATTN_BHSD) {
-    w.q0 = 0;
-    w.sq = a.Sq;
-    w.k0 = 0;
-    w.sk = a.Skv;
-  } else {
-    seq_span(a.cu_q, w.b, &w.q0, &w.sq);
-    seq_span(a.cu_kv, w.b, &w.k0, &w.sk);
-    if (w.k0 < 0 || w.sk < 0 || w.k0 + w.sk > a.Skv) {
-      if (threadIdx.x == 0) report(a.status, ATTN_ERR_DATA);
-      return;
-    }
-  }
-  // rows and key tiles of each Q tile
-  const int rows0 = min(kBM, w.sq - w.row0);
-  const int rows1 = min(kBM, w.sq - w.row0 - kBM);  // <= 0: no second tile
-  const bool has1 = rows1 > 0;
-  // Key tiles run from jlo (the band's first tile for the block's first row; 0 otherwise) to
-  // the tile holding each Q tile's last visible key; n0 and n1 count tiles from jlo. With the
-  // band, Q1 starts at its own first tile: s1 tiles after jlo (its first row is 128 later).
-  const int jlo = EXT >= 1 ? visible_begin(a.mask_mode, w.row0, a.pre) / kBN : 0;
-  const int kv_end0 = visible_end(a.mask_mode, w.row0 + rows0 - 1, w.sq, w.sk, a.next);
-  const int kv_end1 = has1 ? visible_end(a.mask_mode, w.row0 + kBM + rows1 - 1, w.sq, w.sk, a.next) : 0;
-  const int n0 = max((kv_end0 + kBN - 1) / kBN, jlo) - jlo;
-  const int n1 = has1 ? max((kv_end1 + kBN - 1) / kBN, jlo) - jlo : n0;  // tiles loaded (n1 >= n0)
-  const int s1 = EXT >= 1 && has1 ? visible_begin(a.mask_mode, w.row0 + kBM, a.pre) / kBN - jlo : 0;
-
-  const uint32_t bar_base = smem_u32(bars);
   auto bar_addr = [&](const uint64_t* p) { return smem_u32(p); };
-  (void)bar_base;
 
-  // ---- setup: barriers, TMEM -------------------------------------------------------------
+  // ---- setup (once per block): barriers, TMEM ----------------------------------------------
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kStages; ++s) {
       mbar_init(bar_addr(&bars->kv_full[s]), 1);
       mbar_init(bar_addr(&bars->kv_empty[s]), 1);
     }
     mbar_init(bar_addr(&bars->q_full), 1);
+    mbar_init(bar_addr(&bars->q_empty), 1);
     mbar_init(bar_addr(&bars->drain), 1);
     mbar_init(bar_addr(&bars->stall), 1);
     for (int q = 0; q < 2; ++q) {
       mbar_init(bar_addr(&bars->s_full[q]), 1);
       mbar_init(bar_addr(&bars->p_ready[q]), 4);  // one arrival per softmax warp
       mbar_init(bar_addr(&bars->o_done[q]), 1);
+    }
+    for (int s = 0; s < kUnitSlots; ++s) {
+      mbar_init(bar_addr(&bars->unit_full[s]), 1);
+      mbar_init(bar_addr(&bars->unit_empty[s]), kUnitReaders);
     }
     bars->abort = 0;
     fence_mbar_init();
@@ -322,45 +357,92 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t sQ = smem_u32(smem + C::kQOff);
   const uint32_t sKV = smem_u32(smem + C::kKVOff);
 
+  if (warp >= 8) {
+  // the producer warpgroup gives registers to the softmax warpgroups (each branch sets its own
+  // count first, so that the code after it is compiled for that count)
+  setmaxnreg_dec<kRegsProducer>();
   if (warp == kTmaWarp) {
-    // =============================== TMA producer =======================================
+    // =============================== TMA producer (and item decoder) ===========================
+    const bool bhsd = a.layout == ATTN_BHSD;
     if (lane == 0) {
-      const bool bhsd = a.layout == ATTN_BHSD;
-      const int qhead = bhsd ? w.b * a.Nq + w.h : w.h;
-      const int khead = bhsd ? w.b * a.Nkv + w.g : w.g;
-      auto load_tile = [&](const CUtensorMap* map, uint32_t dst, uint32_t bar, int tok, int head,
-                           int boxes) {
-        for (int x = 0; x < boxes; ++x) {
-          if (bhsd)
-            tma_load_3d(dst + x * (kBM * 128), map, bar, x * 64, tok, head);
-          else
-            tma_load_3d(dst + x * (kBM * 128), map, bar, x * 64, head, tok);
-        }
-      };
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
-      const uint32_t qbar = bar_addr(&bars->q_full);
-      mbar_arrive_expect_tx(qbar, (has1 ? 2 : 1) * C::kTileBytes);
-      load_tile(&tm_q, sQ, qbar, w.q0 + w.row0, qhead, C::kBoxes);
-      if (has1) load_tile(&tm_q, sQ + C::kTileBytes, qbar, w.q0 + w.row0 + kBM, qhead, C::kBoxes);
-      // K0, V0, K1, V1, ... through the ring
-      int issued = 0;
-      for (int i = 0; i < 2 * n1; ++i, ++issued) {
-        const int s = i % C::kStages, r = i / C::kStages;
-        if (r > 0 && !wait_bar(bar_addr(&bars->kv_empty[s]), (r - 1) & 1, abort, a.status)) break;
-        const uint32_t fb = bar_addr(&bars->kv_full[s]);
-        mbar_arrive_expect_tx(fb, (i & 1) ? C::kTileBytesV : C::kTileBytes);
-        const int j = i >> 1;
-        load_tile((i & 1) ? &tm_v : &tm_k, sKV + s * C::kTileBytes, fb, w.k0 + (jlo + j) * kBN, khead,
-                  (i & 1) ? C::kBoxesV : C::kBoxes);
+    }
+    auto load_tile = [&](const CUtensorMap* map, uint32_t dst, uint32_t bar, int tok, int head, int boxes) {
+      for (int x = 0; x < boxes; ++x) {
+        if (bhsd)
+          tma_load_3d(dst + x * (kBM * 128), map, bar, x * 64, tok, head);
+        else
+          tma_load_3d(dst + x * (kBM * 128), map, bar, x * 64, head, tok);
       }
-      // drain: every stage this thread filled must have landed before the block exits
-      for (int i = max(0, issued - C::kStages); i < issued; ++i) {
-        const int s = i % C::kStages, r = i / C::kStages;
-        wait_bar(bar_addr(&bars->kv_full[s]), r & 1, abort, a.status, false);
+    };
+    uint32_t it = 0;  // K/V tiles issued by this block: position in the ring
+    int qn = 0;       // Q loads issued
+    int k = 0;        // items handed out
+    bool ok = true;
+    int64_t x = blockIdx.x;
+    for (;;) {
+      Unit U;
+      int k0 = 0;
+      const bool end = x >= n_items;
+      const bool live = !end && decode_unit<EXT>(a, units_per_seq, (int)x, U, k0);
+      if (end || live) {
+        // hand the item (or the end mark) to the other roles through slot k % kUnitSlots
+        if (lane == 0) {
+          const int slot = k % kUnitSlots;
+          if (k >= kUnitSlots)
+            ok = wait_bar(bar_addr(&bars->unit_empty[slot]), ((k / kUnitSlots) - 1) & 1, abort, a.status);
+          if (ok) {
+            if (end) bars->units[slot].b = -1;
+            else bars->units[slot] = U;
+            mbar_arrive(bar_addr(&bars->unit_full[slot]));  // releases the slot's contents
+          }
+        }
+        ok = __shfl_sync(0xffffffffu, ok, 0) != 0;
+        ++k;
+        if (!ok || end) break;
+        if (lane == 0 && U.n1 > 0) {
+          const int g = U.h / (a.Nq / a.Nkv);
+          const int qhead = bhsd ? U.b * a.Nq + U.h : U.h;
+          const int khead = bhsd ? U.b * a.Nkv + g : g;
+          const int nl = 2 * U.n1;
+          // K0, V0, K1, V1, ... through the ring; Q once the previous item's last S has run
+          auto load_kv = [&](int i) {
+            const uint32_t s = it % C::kStages, r = it / C::kStages;
+            if (r > 0 && !wait_bar(bar_addr(&bars->kv_empty[s]), (r - 1) & 1, abort, a.status)) return false;
+            const uint32_t fb = bar_addr(&bars->kv_full[s]);
+            mbar_arrive_expect_tx(fb, (i & 1) ? C::kTileBytesV : C::kTileBytes);
+            load_tile((i & 1) ? &tm_v : &tm_k, sKV + s * C::kTileBytes, fb, k0 + (U.jlo + (i >> 1)) * kBN, khead,
+                      (i & 1) ? C::kBoxesV : C::kBoxes);
+            ++it;
+            return true;
+          };
+          const int first = min(2, nl);
+          for (int i = 0; ok && i < first; ++i) ok = load_kv(i);
+          if (ok && qn > 0) ok = wait_bar(bar_addr(&bars->q_empty), (qn - 1) & 1, abort, a.status);
+          if (ok) {
+            const bool has1 = U.rows1 > 0;
+            const uint32_t qbar = bar_addr(&bars->q_full);
+            mbar_arrive_expect_tx(qbar, (has1 ? 2 : 1) * C::kTileBytes);
+            load_tile(&tm_q, sQ, qbar, U.q0 + U.row0, qhead, C::kBoxes);
+            if (has1) load_tile(&tm_q, sQ + C::kTileBytes, qbar, U.q0 + U.row0 + kBM, qhead, C::kBoxes);
+            ++qn;
+          }
+          for (int i = first; ok && i < nl; ++i) ok = load_kv(i);
+        }
+        ok = __shfl_sync(0xffffffffu, ok, 0) != 0;
+        if (!ok) break;
       }
-      wait_bar(bar_addr(&bars->q_full), 0, abort, a.status, false);
+      int64_t nx = 0;
+      if (lane == 0) nx = sched != nullptr ? (int64_t)gridDim.x + atomicAdd(sched, 1) : x + gridDim.x;
+      x = __shfl_sync(0xffffffffu, nx, 0);
+    }
+    if (lane == 0) {
+      // drain: every load this thread issued must have landed before the block exits
+      for (uint32_t i = it > (uint32_t)C::kStages ? it - C::kStages : 0u; i < it; ++i)
+        wait_bar(bar_addr(&bars->kv_full[i % C::kStages]), (i / C::kStages) & 1, abort, a.status, false);
+      if (qn > 0) wait_bar(bar_addr(&bars->q_full), (qn - 1) & 1, abort, a.status, false);
     }
   } else if (warp == kMmaWarp) {
     // =============================== MMA issue ==========================================
@@ -374,299 +456,346 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t dk0 = smem_desc_sw128(sKV, 16, 1024);
       const uint64_t dv0 = smem_desc_sw128(sKV, kBN * 128, 1024);
       const uint32_t kvfull0 = bar_addr(&bars->kv_full[0]), kvempty0 = bar_addr(&bars->kv_empty[0]);
-      auto full = [&](int i) {
+      auto full = [&](uint32_t i) {
         return wait_bar(kvfull0 + 8 * (i % C::kStages), (i / C::kStages) & 1, abort, a.status);
       };
-      auto release = [&](int i) { mma_commit(kvempty0 + 8 * (i % C::kStages)); };
-      auto issue_qk = [&](uint32_t d, uint64_t dq, int i) {
+      auto release = [&](uint32_t i) { mma_commit(kvempty0 + 8 * (i % C::kStages)); };
+      auto issue_qk = [&](uint32_t d, uint64_t dq, uint32_t i) {
         const uint64_t dk = dk0 + (uint64_t)(((i % C::kStages) * C::kTileBytes) >> 4);
         if constexpr (HD == 128)
           mma_ss_chain8(d, dq, dk, C::kIdescQK, 0u);
         else
           mma_ss_chain4(d, dq, dk, C::kIdescQK, 0u);
       };
-      auto issue_pv = [&](uint32_t d, uint32_t p_tmem, int i, bool acc) {
+      auto issue_pv = [&](uint32_t d, uint32_t p_tmem, uint32_t i, bool acc) {
         const uint64_t dv = dv0 + (uint64_t)(((i % C::kStages) * C::kTileBytes) >> 4);
         mma_ts_chain8(d, p_tmem, dv, C::kIdescPV, acc ? 1u : 0u);
       };
       bool ok = true;
       if constexpr (SDPA_TEST_STALL != 0) ok = wait_bar(bar_addr(&bars->stall), 0, abort, a.status);
-      if (ok && n1 > 0) {
-        ok = wait_bar(bar_addr(&bars->q_full), 0, abort, a.status);
-        if (ok) ok = full(0);
-      }
-      // Q1 works on key tiles s1 .. n1-1 (s1 = 0 except with the band)
-      auto act1 = [&](int j) { return has1 && j >= s1; };
-      if (ok && n1 > 0) {
+      uint32_t it = 0;        // K/V tiles consumed (the same sequence the TMA warp issues)
+      int qn = 0;             // Q loads consumed
+      uint32_t pc0 = 0, pc1 = 0;  // P hand-offs taken from each softmax warpgroup
+      for (int k = 0; ok; ++k) {
+        const int slot = k % kUnitSlots;
+        if (!(ok = wait_bar(bar_addr(&bars->unit_full[slot]), (k / kUnitSlots) & 1, abort, a.status))) break;
+        const Unit* us = &bars->units[slot];
+        const int ub = us->b, n0 = us->n0, n1 = us->n1, s1 = us->s1;
+        const bool has1 = us->rows1 > 0;
+        mbar_arrive(bar_addr(&bars->unit_empty[slot]));
+        if (ub < 0) break;
+        if (n1 <= 0) continue;
+        // Q1 works on key tiles s1 .. n1-1 (s1 = 0 except with the band)
+        auto act1 = [&](int j) { return has1 && j >= s1; };
+        // after the S MMAs of the item's last key tile: Q may be overwritten once they have run
+        auto after_s = [&](int t) {
+          if (t == n1 - 1) mma_commit(bar_addr(&bars->q_empty));
+        };
+        ok = wait_bar(bar_addr(&bars->q_full), qn & 1, abort, a.status);
+        ++qn;
+        if (ok) ok = full(it);
+        if (!ok) break;
         tc_fence_after();
         if (n0 > 0) {
-          issue_qk(S0, dq0, 0);
+          issue_qk(S0, dq0, it);
           mma_commit(bar_addr(&bars->s_full[0]));
         }
         if (act1(0)) {
-          issue_qk(S1, dq1, 0);
+          issue_qk(S1, dq1, it);
           mma_commit(bar_addr(&bars->s_full[1]));
         }
-        release(0);
-      }
-      for (int j = 0; ok && j < n1; ++j) {
-        const int iv = 2 * j + 1, ik = 2 * j + 2;
-        if (!(ok = full(iv))) break;
-        tc_fence_after();
-        if (j < n0) {
-          if (!(ok = wait_bar(bar_addr(&bars->p_ready[0]), j & 1, abort, a.status))) break;
+        after_s(0);
+        release(it);
+        for (int j = 0; ok && j < n1; ++j) {
+          const uint32_t iv = it + 2 * j + 1, ik = it + 2 * j + 2;
+          if (!(ok = full(iv))) break;
           tc_fence_after();
-          issue_pv(O0, S0, iv, j > 0);
-          if (j == n0 - 1) mma_commit(bar_addr(&bars->o_done[0]));
-        }
-        const bool next = j + 1 < n1;
-        if (next) {
-          if (!(ok = full(ik))) break;
-          tc_fence_after();
-          if (j + 1 < n0) {
-            issue_qk(S0, dq0, ik);
-            mma_commit(bar_addr(&bars->s_full[0]));
+          if (j < n0) {
+            if (!(ok = wait_bar(bar_addr(&bars->p_ready[0]), pc0 & 1, abort, a.status))) break;
+            ++pc0;
+            tc_fence_after();
+            issue_pv(O0, S0, iv, j > 0);
+            if (j == n0 - 1) mma_commit(bar_addr(&bars->o_done[0]));
+          }
+          const bool next = j + 1 < n1;
+          if (next) {
+            if (!(ok = full(ik))) break;
+            tc_fence_after();
+            if (j + 1 < n0) {
+              issue_qk(S0, dq0, ik);
+              mma_commit(bar_addr(&bars->s_full[0]));
+            }
+          }
+          if (act1(j)) {
+            if (!(ok = wait_bar(bar_addr(&bars->p_ready[1]), pc1 & 1, abort, a.status))) break;
+            ++pc1;
+            tc_fence_after();
+            issue_pv(O1, S1, iv, j > s1);
+            if (j == n1 - 1) mma_commit(bar_addr(&bars->o_done[1]));
+          }
+          release(iv);
+          if (next) {
+            if (act1(j + 1)) {
+              issue_qk(S1, dq1, ik);
+              mma_commit(bar_addr(&bars->s_full[1]));
+            }
+            after_s(j + 1);
+            release(ik);
           }
         }
-        if (act1(j)) {
-          if (!(ok = wait_bar(bar_addr(&bars->p_ready[1]), (j - s1) & 1, abort, a.status))) break;
-          tc_fence_after();
-          issue_pv(O1, S1, iv, j > s1);
-          if (j == n1 - 1) mma_commit(bar_addr(&bars->o_done[1]));
-        }
-        release(iv);
-        if (next) {
-          if (act1(j + 1)) {
-            issue_qk(S1, dq1, ik);
-            mma_commit(bar_addr(&bars->s_full[1]));
-          }
-          release(ik);
-        }
+        it += 2 * n1;
       }
       if (!ok) *abort = 1;
       // every MMA and commit issued above must have completed before TMEM is freed
       mma_commit(bar_addr(&bars->drain));
       wait_bar(bar_addr(&bars->drain), 0, abort, a.status, false);
     }
+  }
   } else {
+    setmaxnreg_inc<kRegsSoftmax>();
     // =============================== softmax + epilogue ================================
     const int q = warp >> 2;                       // Q tile of this warpgroup
     const int quarter = warp & 3;                  // TMEM lane quarter of this warp
     const int r = quarter * 32 + lane;             // row within the Q tile = TMEM lane
-    const int j0 = q == 0 ? 0 : s1;                // this Q tile's key tiles: j0 .. n-1
-    const int n = q == 0 ? n0 : (has1 ? n1 : 0);
-    const int rows = q == 0 ? rows0 : rows1;
-    const int i = w.row0 + q * kBM + r;            // row within the sequence
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     const uint32_t S = tmem + lane_off + q * 128;
     const uint32_t O = tmem + lane_off + 256 + q * HDV;
-    const int lim = i < w.sq ? visible_end(a.mask_mode, i, w.sq, w.sk, a.next) : w.sk;
-    const int lo = EXT >= 1 && i < w.sq ? visible_begin(a.mask_mode, i, a.pre) : 0;
-    // explicit mask row of this query (rows past the sequence read none)
-    const uint8_t* mrow = nullptr;
-    if constexpr (EXT == 2)
-      if (i < w.sq && a.mask != nullptr) mrow = a.mask + (int64_t)w.b * a.mask_bs + (int64_t)i * a.mask_rs;
+    uint32_t sfc = 0;  // S hand-offs taken, over all of the block's items
+    uint32_t odc = 0;  // final-O hand-offs taken
+    for (int k = 0;; ++k) {
+      const int slot = k % kUnitSlots;
+      if (!__all_sync(0xffffffffu, wait_bar(bar_addr(&bars->unit_full[slot]), (k / kUnitSlots) & 1, abort, a.status)))
+        break;
+      // the item stays in its slot until this warp is done with it (fields are read as needed)
+      const Unit& w = bars->units[slot];
+      if (w.b < 0) break;
+      const bool has1 = w.rows1 > 0;
+      const int jlo = w.jlo;
+      const int j0 = q == 0 ? 0 : w.s1;              // this Q tile's key tiles: j0 .. n-1
+      const int n = q == 0 ? w.n0 : (has1 ? w.n1 : 0);
+      const int i = w.row0 + q * kBM + r;            // row within the sequence
+      const int lim = i < w.sq ? visible_end(a.mask_mode, i, w.sq, w.sk, a.next) : w.sk;
+      const int lo = EXT >= 1 && i < w.sq ? visible_begin(a.mask_mode, i, a.pre) : 0;
+      // explicit mask row of this query (rows past the sequence read none)
+      const uint8_t* mrow = nullptr;
+      if constexpr (EXT == 2)
+        if (i < w.sq && a.mask != nullptr) mrow = a.mask + (int64_t)w.b * a.mask_bs + (int64_t)i * a.mask_rs;
 
-    float m = -INFINITY;        // running max used for P (log2 units, lazily updated)
-    float mraw = -INFINITY;     // true max of the raw scores q.k
-    float l = 0.f;
-    bool ok = true;
-    if (q == 0 || has1) {
-      for (int j = j0; j < n; ++j) {
-        ok = __all_sync(0xffffffffu, wait_bar(bar_addr(&bars->s_full[q]), (j - j0) & 1, abort, a.status));
-        if (!ok) break;
-        tc_fence_after();
-        const int kbase = (jlo + j) * kBN;
-        uint4 mk[EXT == 2 ? 8 : 1];
-        if constexpr (EXT == 2) {
-          // the mask bytes of this row's 128 keys (16 at a time when aligned and whole);
-          // issued before the TMEM loads so the two latencies overlap
-          if (mrow == nullptr) {
-            // band only, or a row past the sequence: nothing to read
-          } else if (a.mask_vec && kbase + kBN <= w.sk) {
-            const uint4* src = reinterpret_cast<const uint4*>(mrow + kbase);
+      float m = -INFINITY;        // running max used for P (log2 units, lazily updated)
+      float mraw = -INFINITY;     // true max of the raw scores q.k
+      float l = 0.f;
+      bool ok = true;
+      if (q == 0 || has1) {
+        for (int j = j0; j < n; ++j) {
+          ok = __all_sync(0xffffffffu, wait_bar(bar_addr(&bars->s_full[q]), sfc & 1, abort, a.status));
+          ++sfc;
+          if (!ok) break;
+          tc_fence_after();
+          const int kbase = (jlo + j) * kBN;
+          uint4 mk[EXT == 2 ? 8 : 1];
+          if constexpr (EXT == 2) {
+            // the mask bytes of this row's 128 keys (16 at a time when aligned and whole);
+            // issued before the TMEM loads so the two latencies overlap
+            if (mrow == nullptr) {
+              // band only, or a row past the sequence: nothing to read
+            } else if (a.mask_vec && kbase + kBN <= w.sk) {
+              const uint4* src = reinterpret_cast<const uint4*>(mrow + kbase);
 #pragma unroll
-            for (int x = 0; x < 8; ++x) mk[x] = __ldg(src + x);
-          } else {
+              for (int x = 0; x < 8; ++x) mk[x] = __ldg(src + x);
+            } else {
 #pragma unroll
-            for (int x = 0; x < 8; ++x) {
-              uint32_t wd[4];
+              for (int x = 0; x < 8; ++x) {
+                uint32_t wd[4];
 #pragma unroll
-              for (int y = 0; y < 4; ++y) {
-                uint32_t word = 0;
+                for (int y = 0; y < 4; ++y) {
+                  uint32_t word = 0;
 #pragma unroll
-                for (int z = 0; z < 4; ++z) {
-                  const int c = x * 16 + y * 4 + z;
-                  const uint32_t byte = kbase + c < w.sk ? mrow[kbase + c] : 0u;
-                  word |= (byte != 0u ? 1u : 0u) << (8 * z);
+                  for (int z = 0; z < 4; ++z) {
+                    const int c = x * 16 + y * 4 + z;
+                    const uint32_t byte = kbase + c < w.sk ? mrow[kbase + c] : 0u;
+                    word |= (byte != 0u ? 1u : 0u) << (8 * z);
+                  }
+                  wd[y] = word;
                 }
-                wd[y] = word;
+                mk[x] = make_uint4(wd[0], wd[1], wd[2], wd[3]);
               }
-              mk[x] = make_uint4(wd[0], wd[1], wd[2], wd[3]);
             }
           }
-        }
-        float s[4][32];
+          float s[4][32];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_ld32f(S + c * 32, s[c]);
-        tmem_wait_ld();
-        if constexpr (EXT == 0) {
-          if (kbase + kBN > lim) {
-#pragma unroll
-            for (int c = 0; c < kBN; ++c)
-              if (kbase + c >= lim) s[c >> 5][c & 31] = -INFINITY;
-          }
-        } else {
-          if (kbase + kBN > lim || kbase < lo) {
-#pragma unroll
-            for (int c = 0; c < kBN; ++c)
-              if (kbase + c >= lim || kbase + c < lo) s[c >> 5][c & 31] = -INFINITY;
-          }
-          if (EXT == 2 && mrow != nullptr) {
-#pragma unroll
-          for (int c = 0; c < kBN; ++c) {
-            const uint4 v4 = mk[c >> 4];
-            const uint32_t wd = ((c >> 2) & 3) == 0 ? v4.x : ((c >> 2) & 3) == 1 ? v4.y
-                              : ((c >> 2) & 3) == 2 ? v4.z : v4.w;
-            if ((wd >> (8 * (c & 3))) & 0xffu) s[c >> 5][c & 31] = -INFINITY;
-          }
-          }
-        }
-        // row max: a tree of 3-input maxima over the 128 scores
-        float mx[8];
-#pragma unroll
-        for (int x = 0; x < 8; ++x) {
-          const float* v = &s[x >> 1][(x & 1) * 16];
-          const float a0 = fmax3(v[0], v[1], v[2]), a1 = fmax3(v[3], v[4], v[5]);
-          const float a2 = fmax3(v[6], v[7], v[8]), a3 = fmax3(v[9], v[10], v[11]);
-          const float a4 = fmax3(v[12], v[13], v[14]);
-          mx[x] = fmax3(fmax3(a0, a1, a2), fmax3(a3, a4, v[15]), a0);
-        }
-        const float tmax = fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]),
-                                 fmaxf(mx[6], mx[7]));
-        mraw = fmaxf(mraw, tmax);
-        const float tmax2 = tmax * scale_log2;
-        bool bump = tmax2 > m + kRescaleThreshold;  // also true for the first finite max
-        float corr = 1.f;
-        if (bump) {
-          corr = (m == -INFINITY) ? 0.f : ex2(m - tmax2);
-          m = tmax2;
-          l *= corr;
-        }
-        const float muse = m == -INFINITY ? 0.f : m;
-        // P = 2^(s * scale_log2 - m) with packed (two-lane) FMA and add; exp2 on the MUFU unit
-        // (and, for one pair in kEmuEvery, on the FMA pipe).
-        float2 rs[4] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
-        const float2 sc2 = make_float2(scale_log2, scale_log2), nm2 = make_float2(-muse, -muse);
-        uint32_t pk[2][32];
-#pragma unroll
-        for (int c = 0; c < kBN; c += 2) {
-          const float2 x = __ffma2_rn(make_float2(s[c >> 5][c & 31], s[c >> 5][(c + 1) & 31]), sc2, nm2);
-          float p0, p1;
-          if (kEmuEvery > 0 && ((c >> 1) % (kEmuEvery > 0 ? kEmuEvery : 1)) == kEmuEvery - 1) {
-            exp2_poly2(x.x, x.y, p0, p1);
-          } else {
-            p0 = ex2(x.x);
-            p1 = ex2(x.y);
-          }
-          rs[(c >> 1) & 3] = __fadd2_rn(rs[(c >> 1) & 3], make_float2(p0, p1));
-          pk[c >> 6][(c >> 1) & 31] = pack16x2<F16>(p0, p1);
-        }
-        l += ((rs[0].x + rs[0].y) + (rs[1].x + rs[1].y)) + ((rs[2].x + rs[2].y) + (rs[3].x + rs[3].y));
-        // rescale O (complete up to tile j-1: the S_j commit covers every earlier MMA)
-        if (__any_sync(0xffffffffu, bump && j > j0)) {
-          const float f = (bump && j > j0) ? corr : 1.f;
-#pragma unroll
-          for (int c = 0; c < HDV / 32; ++c) {
-            uint32_t o[32];
-            tmem_ld32(O + c * 32, o);
-            tmem_wait_ld();
-#pragma unroll
-            for (int x = 0; x < 32; ++x) o[x] = __float_as_uint(__uint_as_float(o[x]) * f);
-            tmem_st32(O + c * 32, o);
-          }
-        }
-        tmem_st32(S, pk[0]);
-        tmem_st32(S + 32, pk[1]);
-        tmem_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar_addr(&bars->p_ready[q]));
-      }
-    }
-    // ---- epilogue: O / l -> bf16, statistics ------------------------------------------------
-    const bool have_o = ok && n > j0 && (q == 0 || has1);
-    if (have_o) ok = __all_sync(0xffffffffu, wait_bar(bar_addr(&bars->o_done[q]), 0, abort, a.status));
-    tc_fence_after();
-    if (q == 0 || has1) {
-      const bool store = r < rows;
-      const bool bhsd = a.layout == ATTN_BHSD;
-      uint16_t* out = static_cast<uint16_t*>(a.out);  // bf16 or f16 bit patterns
-      // this row's own result: o = O / l, max and sum in natural-log units
-      // a row that saw no key keeps mraw = -inf (its sum holds only the polynomial's tiny
-      // values for masked scores) and gives a zero output, max -inf and sum 0
-      const bool any = mraw > -INFINITY && l > 0.f && ok;
-      const float m_loc = any ? mraw * a.scale : -INFINITY;
-      const float l_loc = any ? l * ex2(m - mraw * scale_log2) : 0.f;
-      float f_o = any ? 1.f / l : 0.f;  // factor on the unnormalised O in TMEM
-      float f_prev = 0.f;               // factor on the accumulator's previous output row
-      int64_t orow, so;
-      if (a.acc_mode == kAccNone) {
-        orow = bhsd ? (((int64_t)w.b * a.Nq + w.h) * a.Sq + i) * HDV : ((int64_t)(w.q0 + i) * a.Nq + w.h) * HDV;
-        so = bhsd ? ((int64_t)w.b * a.Nq + w.h) * a.Sq + i : (int64_t)(w.q0 + i) * a.Nq + w.h;
-        if (store && a.smax != nullptr) {
-          a.smax[so] = m_loc;
-          a.ssum[so] = l_loc;
-        }
-      } else {
-        // accumulator in the merge layouts: BHSD -> output [Sq, B, Nq*D] (SBH), statistics
-        // [B, Nq, Sq, 8]; TND -> output [T, Nq*D], statistics [T, Nq, 8]
-        orow = bhsd ? (((int64_t)i * a.B + w.b) * a.Nq + w.h) * HDV : ((int64_t)(w.q0 + i) * a.Nq + w.h) * HDV;
-        so = (bhsd ? ((int64_t)w.b * a.Nq + w.h) * a.Sq + i : (int64_t)(w.q0 + i) * a.Nq + w.h) * 8;
-        if (store) merge_into_stats(a, so, m_loc, l_loc, &f_prev, &f_o);
-      }
-#pragma unroll
-      for (int c = 0; c < HDV / 32; ++c) {
-        uint32_t o[32];
-        if (have_o && ok) {
-          tmem_ld32(O + c * 32, o);
+          for (int c = 0; c < 4; ++c) tmem_ld32f(S + c * 32, s[c]);
           tmem_wait_ld();
-        } else {
+          if constexpr (EXT == 0) {
+            if (kbase + kBN > lim) {
 #pragma unroll
-          for (int x = 0; x < 32; ++x) o[x] = 0u;
-        }
-        if (store) {
-          uint4* dst = reinterpret_cast<uint4*>(out + orow + c * 32);
-          uint32_t prev[16];
-          if (a.acc_mode == kAccMerge) {
+              for (int c = 0; c < kBN; ++c)
+                if (kbase + c >= lim) s[c >> 5][c & 31] = -INFINITY;
+            }
+          } else {
+            if (kbase + kBN > lim || kbase < lo) {
 #pragma unroll
-            for (int x = 0; x < 4; ++x) {
-              const uint4 t = dst[x];
-              prev[4 * x] = t.x;
-              prev[4 * x + 1] = t.y;
-              prev[4 * x + 2] = t.z;
-              prev[4 * x + 3] = t.w;
+              for (int c = 0; c < kBN; ++c)
+                if (kbase + c >= lim || kbase + c < lo) s[c >> 5][c & 31] = -INFINITY;
+            }
+            if (EXT == 2 && mrow != nullptr) {
+#pragma unroll
+            for (int c = 0; c < kBN; ++c) {
+              const uint4 v4 = mk[c >> 4];
+              const uint32_t wd = ((c >> 2) & 3) == 0 ? v4.x : ((c >> 2) & 3) == 1 ? v4.y
+                                : ((c >> 2) & 3) == 2 ? v4.z : v4.w;
+              if ((wd >> (8 * (c & 3))) & 0xffu) s[c >> 5][c & 31] = -INFINITY;
+            }
             }
           }
-          uint32_t pkd[16];
+          // row max: a tree of 3-input maxima over the 128 scores
+          float mx[8];
 #pragma unroll
-          for (int x = 0; x < 16; ++x) {
-            float v0 = f_o == 0.f ? 0.f : __uint_as_float(o[2 * x]) * f_o;
-            float v1 = f_o == 0.f ? 0.f : __uint_as_float(o[2 * x + 1]) * f_o;
-            if (a.acc_mode == kAccMerge) {
-              const float2 pv = unpack16x2<F16>(prev[x]);
-              v0 = fmaf(pv.x, f_prev, v0);
-              v1 = fmaf(pv.y, f_prev, v1);
-            }
-            pkd[x] = pack16x2<F16>(v0, v1);
+          for (int x = 0; x < 8; ++x) {
+            const float* v = &s[x >> 1][(x & 1) * 16];
+            const float a0 = fmax3(v[0], v[1], v[2]), a1 = fmax3(v[3], v[4], v[5]);
+            const float a2 = fmax3(v[6], v[7], v[8]), a3 = fmax3(v[9], v[10], v[11]);
+            const float a4 = fmax3(v[12], v[13], v[14]);
+            mx[x] = fmax3(fmax3(a0, a1, a2), fmax3(a3, a4, v[15]), a0);
           }
+          const float tmax = fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]),
+                                   fmaxf(mx[6], mx[7]));
+          mraw = fmaxf(mraw, tmax);
+          const float tmax2 = tmax * scale_log2;
+          bool bump = tmax2 > m + kRescaleThreshold;  // also true for the first finite max
+          float corr = 1.f;
+          if (bump) {
+            corr = (m == -INFINITY) ? 0.f : ex2(m - tmax2);
+            m = tmax2;
+            l *= corr;
+          }
+          const float muse = m == -INFINITY ? 0.f : m;
+          // P = 2^(s * scale_log2 - m) with packed (two-lane) FMA and add; exp2 on the MUFU unit
+          // (and, for one pair in kEmuEvery, on the FMA pipe).
+          float2 rs[4] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
+          const float2 sc2 = make_float2(scale_log2, scale_log2), nm2 = make_float2(-muse, -muse);
+          uint32_t pk[2][32];
 #pragma unroll
-          for (int x = 0; x < 4; ++x)
-            dst[x] = make_uint4(pkd[4 * x], pkd[4 * x + 1], pkd[4 * x + 2], pkd[4 * x + 3]);
+          for (int c = 0; c < kBN; c += 2) {
+            const float2 x = __ffma2_rn(make_float2(s[c >> 5][c & 31], s[c >> 5][(c + 1) & 31]), sc2, nm2);
+            float p0, p1;
+            if (kEmuEvery > 0 && ((c >> 1) % (kEmuEvery > 0 ? kEmuEvery : 1)) == kEmuEvery - 1) {
+              exp2_poly2(x.x, x.y, p0, p1);
+            } else {
+              p0 = ex2(x.x);
+              p1 = ex2(x.y);
+            }
+            rs[(c >> 1) & 3] = __fadd2_rn(rs[(c >> 1) & 3], make_float2(p0, p1));
+            pk[c >> 6][(c >> 1) & 31] = pack16x2<F16>(p0, p1);
+            // the first 64 keys' P go to TMEM (over S columns already read) as soon as they
+            // are packed, so that half of P need not stay in registers
+            if (c == 62) tmem_st32(S, pk[0]);
+          }
+          l += ((rs[0].x + rs[0].y) + (rs[1].x + rs[1].y)) + ((rs[2].x + rs[2].y) + (rs[3].x + rs[3].y));
+          // rescale O (complete up to tile j-1: the S_j commit covers every earlier MMA)
+          if (__any_sync(0xffffffffu, bump && j > j0)) {
+            const float f = (bump && j > j0) ? corr : 1.f;
+#pragma unroll
+            for (int c = 0; c < HDV / 32; ++c) {
+              uint32_t o[32];
+              tmem_ld32(O + c * 32, o);
+              tmem_wait_ld();
+#pragma unroll
+              for (int x = 0; x < 32; ++x) o[x] = __float_as_uint(__uint_as_float(o[x]) * f);
+              tmem_st32(O + c * 32, o);
+            }
+          }
+          tmem_st32(S + 32, pk[1]);
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar_addr(&bars->p_ready[q]));
         }
       }
+      // ---- epilogue: O / l -> bf16, statistics ------------------------------------------------
+      const bool have_o = ok && n > j0 && (q == 0 || has1);
+      if (have_o) {
+        ok = __all_sync(0xffffffffu, wait_bar(bar_addr(&bars->o_done[q]), odc & 1, abort, a.status));
+        ++odc;
+      }
+      tc_fence_after();
+      if (q == 0 || has1) {
+        const bool store = r < (q == 0 ? w.rows0 : w.rows1);
+        const bool bhsd = a.layout == ATTN_BHSD;
+        uint16_t* out = static_cast<uint16_t*>(a.out);  // bf16 or f16 bit patterns
+        // this row's own result: o = O / l, max and sum in natural-log units
+        // a row that saw no key keeps mraw = -inf (its sum holds only the polynomial's tiny
+        // values for masked scores) and gives a zero output, max -inf and sum 0
+        const bool any = mraw > -INFINITY && l > 0.f && ok;
+        const float m_loc = any ? mraw * a.scale : -INFINITY;
+        const float l_loc = any ? l * ex2(m - mraw * scale_log2) : 0.f;
+        float f_o = any ? 1.f / l : 0.f;  // factor on the unnormalised O in TMEM
+        float f_prev = 0.f;               // factor on the accumulator's previous output row
+        int64_t orow, so;
+        if (a.acc_mode == kAccNone) {
+          orow = bhsd ? (((int64_t)w.b * a.Nq + w.h) * a.Sq + i) * HDV : ((int64_t)(w.q0 + i) * a.Nq + w.h) * HDV;
+          so = bhsd ? ((int64_t)w.b * a.Nq + w.h) * a.Sq + i : (int64_t)(w.q0 + i) * a.Nq + w.h;
+          if (store && a.smax != nullptr) {
+            a.smax[so] = m_loc;
+            a.ssum[so] = l_loc;
+          }
+        } else {
+          // accumulator in the merge layouts: BHSD -> output [Sq, B, Nq*D] (SBH), statistics
+          // [B, Nq, Sq, 8]; TND -> output [T, Nq*D], statistics [T, Nq, 8]
+          orow = bhsd ? (((int64_t)i * a.B + w.b) * a.Nq + w.h) * HDV : ((int64_t)(w.q0 + i) * a.Nq + w.h) * HDV;
+          so = (bhsd ? ((int64_t)w.b * a.Nq + w.h) * a.Sq + i : (int64_t)(w.q0 + i) * a.Nq + w.h) * 8;
+          if (store) merge_into_stats(a, so, m_loc, l_loc, &f_prev, &f_o);
+        }
+        // the output row leaves TMEM 64 columns per round trip (two loads, then one wait)
+        uint32_t oc[2][32];
+#pragma unroll
+        for (int c = 0; c < HDV / 32; ++c) {
+          if ((c & 1) == 0) {
+            if (have_o && ok) {
+              tmem_ld32(O + c * 32, oc[0]);
+              tmem_ld32(O + (c + 1) * 32, oc[1]);
+              tmem_wait_ld();
+            } else {
+#pragma unroll
+              for (int x = 0; x < 32; ++x) oc[0][x] = oc[1][x] = 0u;
+            }
+          }
+          const uint32_t (&o)[32] = oc[c & 1];
+          if (store) {
+            uint4* dst = reinterpret_cast<uint4*>(out + orow + c * 32);
+            uint32_t prev[16];
+            if (a.acc_mode == kAccMerge) {
+#pragma unroll
+              for (int x = 0; x < 4; ++x) {
+                const uint4 t = dst[x];
+                prev[4 * x] = t.x;
+                prev[4 * x + 1] = t.y;
+                prev[4 * x + 2] = t.z;
+                prev[4 * x + 3] = t.w;
+              }
+            }
+            uint32_t pkd[16];
+#pragma unroll
+            for (int x = 0; x < 16; ++x) {
+              float v0 = f_o == 0.f ? 0.f : __uint_as_float(o[2 * x]) * f_o;
+              float v1 = f_o == 0.f ? 0.f : __uint_as_float(o[2 * x + 1]) * f_o;
+              if (a.acc_mode == kAccMerge) {
+                const float2 pv = unpack16x2<F16>(prev[x]);
+                v0 = fmaf(pv.x, f_prev, v0);
+                v1 = fmaf(pv.y, f_prev, v1);
+              }
+              pkd[x] = pack16x2<F16>(v0, v1);
+            }
+#pragma unroll
+            for (int x = 0; x < 4; ++x)
+              dst[x] = make_uint4(pkd[4 * x], pkd[4 * x + 1], pkd[4 * x + 2], pkd[4 * x + 3]);
+          }
+        }
+      }
+      if (!ok) break;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_addr(&bars->unit_empty[slot]));
+      }
     }
-  }
 
   // ---- teardown ----------------------------------------------------------------------------
   tc_fence_before();
@@ -674,6 +803,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
+  }
+  if (sched != nullptr && threadIdx.x == 0) {
+    // the last block to finish puts the slot's counters back to 0 for the next launch using it
+    __threadfence();
+    if (atomicAdd(sched + 1, 1) == (int)gridDim.x - 1) {
+      atomicExch(sched, 0);
+      atomicExch(sched + 1, 0);
+    }
   }
 }
 
@@ -715,6 +852,49 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t D, uint64_t dim1, uint6
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// The scheduler slot (g_sched) for a launch on stream `st`, or null: static division of the
+// items. Every stream of every device gets a slot of its own on first use (launches on one
+// stream run one after another, so they can share it). A launch gets none when its stream is
+// being captured into a graph (a graph may be replayed on any stream, next to other launches),
+// for the per-thread default stream (one handle, a different stream in every thread), and once
+// all slots of the device are taken.
+cudaError_t sched_slot(cudaStream_t st, int** out) {
+  *out = nullptr;
+  if (st == cudaStreamPerThread) return cudaSuccess;
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  cudaError_t e = cudaStreamIsCapturing(st, &cap);
+  if (e != cudaSuccess) return e;
+  if (cap != cudaStreamCaptureStatusNone) return cudaSuccess;
+  int dev = 0;
+  e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  constexpr int kMaxDevices = 64;
+  if (dev < 0 || dev >= kMaxDevices) return cudaSuccess;
+  static std::mutex mu;
+  static int* base[kMaxDevices] = {};
+  static int used[kMaxDevices] = {};
+  static std::map<std::pair<int, cudaStream_t>, int> slot_of;
+  std::lock_guard<std::mutex> lk(mu);
+  if (base[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_sched);
+    if (e != cudaSuccess) return e;
+    base[dev] = static_cast<int*>(p);
+  }
+  const auto key = std::make_pair(dev, st);
+  auto f = slot_of.find(key);
+  int slot;
+  if (f != slot_of.end()) {
+    slot = f->second;
+  } else {
+    if (used[dev] >= kSchedSlots) return cudaSuccess;
+    slot = used[dev]++;
+    slot_of.emplace(key, slot);
+  }
+  *out = base[dev] + 2 * slot;
+  return cudaSuccess;
+}
+
 template <int HD, int HDV, bool F16>
 cudaError_t launch_hd(const FwdArgs& a, cudaStream_t st) {
   using C = Cfg<HD, HDV, F16>;
@@ -739,6 +919,20 @@ cudaError_t launch_hd(const FwdArgs& a, cudaStream_t st) {
                                                 : fwd_bf16_kernel<HD, HDV, F16, 0>;
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return e;
+  // The register split inside the kernel (softmax warpgroups up to kRegsSoftmax, the producer
+  // warpgroup down to kRegsProducer) waits for registers the block must have been launched with:
+  // refuse to launch a build whose kernel holds fewer than kRegsLaunch a thread.
+  {
+    static std::atomic<int> checked[3] = {};
+    const int which = kernel == fwd_bf16_kernel<HD, HDV, F16, 2> ? 2 : kernel == fwd_bf16_kernel<HD, HDV, F16, 1> ? 1 : 0;
+    if (checked[which].load(std::memory_order_acquire) == 0) {
+      cudaFuncAttributes fa;
+      e = cudaFuncGetAttributes(&fa, kernel);
+      if (e != cudaSuccess) return e;
+      if (fa.numRegs < kRegsLaunch || fa.maxThreadsPerBlock < kThreads) return cudaErrorInvalidConfiguration;
+      checked[which].store(1, std::memory_order_release);
+    }
+  }
   int units_per_seq = 0;
   int64_t units;
   if (a.layout == ATTN_BHSD) {
@@ -747,11 +941,17 @@ cudaError_t launch_hd(const FwdArgs& a, cudaStream_t st) {
   } else {
     units = (a.Sq + kRowsPerBlock - 1) / kRowsPerBlock + a.B;
   }
-  const int64_t blocks = units * a.Nq;
-  if (blocks <= 0) return cudaSuccess;
-  if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+  const int64_t items = units * a.Nq;
+  if (items <= 0) return cudaSuccess;
+  if (items > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
   const float scale_log2 = a.scale * 1.4426950408889634f;
-  kernel<<<(unsigned)blocks, kThreads, C::kSmemBytes, st>>>(tq, tk, tv, a, units_per_seq, scale_log2);
+  // one persistent block per SM (fewer when there are fewer items)
+  const int64_t grid = items < a.num_sms ? items : (a.num_sms > 0 ? a.num_sms : 1);
+  int* sched = nullptr;
+  cudaError_t se = sched_slot(st, &sched);
+  if (se != cudaSuccess) return se;
+  kernel<<<(unsigned)grid, kThreads, C::kSmemBytes, st>>>(tq, tk, tv, a, units_per_seq, scale_log2, (int)items,
+                                                           sched);
   return cudaGetLastError();
 }
 
