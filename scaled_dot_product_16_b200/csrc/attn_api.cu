@@ -235,8 +235,7 @@ int attn_sparse_csr(const float* q, const float* k, const float* v, const int32_
   a.nnz_cap = nnz_cap;
   a.cols_vec = csr_columns != nullptr && aligned16(csr_columns) && nnz_cap % 4 == 0;
   a.out = out;
-  int sms = 0;
-  int rc = device_state(&a.status, &sms);
+  int rc = device_state(&a.status, &a.num_sms);
   if (rc != ATTN_OK) return rc;
   // D = 64 or 128 with 16-byte aligned tensors: tiled over each block's union of columns;
   // otherwise a warp per row gathering its own entries

@@ -28,6 +28,8 @@
 // by a row-per-warp pass at the end.
 #include <math.h>
 
+#include <atomic>
+
 #include "common.cuh"
 #include "csr_union.cuh"
 #include "launch.h"
@@ -35,18 +37,21 @@
 namespace sdpa {
 namespace {
 
-constexpr int kRows = 128;                   // query rows per block
 constexpr int kKeys = 32;                    // union keys per tile
-constexpr int kThreads = 256;
 constexpr int kWin = 512;                    // union columns whose row marks are held at once
 constexpr int kWinTiles = kWin / kKeys;
 constexpr int kWinWords = kWin / 32;         // mark words per row
 constexpr int kMaskStride = kWinWords + 1;   // padded row of the marks: a warp's 4 rows, 4 banks apart
 constexpr int kMaxS = 32768;
-constexpr int kPtStride = kRows + 4;         // padded key row of P^T: a warp's 16-byte stores spread over banks
 
-template <int D>
+// A block owns ROWS query rows (a multiple of 16: a warp per 16 rows, two threads per row);
+// the host picks ROWS per call so that the blocks fill whole rounds of the GPU's block slots.
+template <int D, int ROWS>
 struct F32Cfg {
+  static constexpr int kRows = ROWS;
+  static constexpr int kThreads = 2 * ROWS;
+  static constexpr int kPtStride = ROWS + 4;  // padded key row of P^T: a warp's 16-byte stores spread over banks
+  static_assert(ROWS % 16 == 0 && ROWS <= 128, "a warp per 16 rows, at most 8 warps");
   static constexpr int kKStride = D + 4;  // floats per staged key row (16-byte groups: key k -> k mod 8)
   static constexpr int kQsOff = 0;                                    // float Qt[D][kRows], scaled
   static constexpr int kKsOff = kQsOff + kRows * D * 4;               // float Ks[2][kKeys][kKStride]
@@ -63,6 +68,7 @@ struct F32Cfg {
   static_assert(kPsOff - kKsOff >= kMaxS, "the union's column bytes fit the K/V buffers");
   static_assert(kSmemBytes <= 232448, "227 KB of shared memory per block");
   static_assert(D != 64 || kSmemBytes <= 112 * 1024, "two blocks per SM at D = 64");
+  static_assert((kPtStride % 32) % 8 == 4, "16-byte P^T stores of 8 consecutive keys on distinct banks");
 };
 
 __device__ __forceinline__ float ex2_approx(float x) {
@@ -82,15 +88,16 @@ __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wai
 
 // Starts the copies of the key and value rows of kcol[0 .. nk) into one buffer pair (key row k
 // at ks + k * kKStride floats, value row k at vs + k * D floats); rows nk .. kKeys-1 are zeroed.
-template <int D>
+template <int D, int ROWS>
 __device__ __forceinline__ void stage_tile(uint32_t ks, uint32_t vs, const int* kcol, int nk, const float* Kb,
                                            const float* Vb) {
+  using C = F32Cfg<D, ROWS>;
   constexpr int kChunks = D / 4;  // 16-byte chunks per row
-  for (int x = threadIdx.x; x < kKeys * kChunks; x += kThreads) {
+  for (int x = threadIdx.x; x < kKeys * kChunks; x += C::kThreads) {
     const int k = x / kChunks, c = x % kChunks;
     const bool valid = k < nk;
     const int64_t col = valid ? kcol[k] : 0;  // row 0 is a readable address for a zero fill
-    cp_async16(ks + (uint32_t)(k * F32Cfg<D>::kKStride + 4 * c) * 4u, Kb + col * D + 4 * c, valid);
+    cp_async16(ks + (uint32_t)(k * C::kKStride + 4 * c) * 4u, Kb + col * D + 4 * c, valid);
     cp_async16(vs + (uint32_t)(k * D + 4 * c) * 4u, Vb + col * D + 4 * c, valid);
   }
 }
@@ -99,18 +106,20 @@ __device__ __forceinline__ void stage_tile(uint32_t ks, uint32_t vs, const int* 
 // u (W0 <= u < W0 + kWin), built a warp per row (csr_mark_row in csr_union.cuh). A row that
 // stores some column twice sets fewer bits than it has entries in the window: it is marked heavy.
 // Every thread of the block calls this; it ends with the marks complete.
+template <int ROWS>
 __device__ __forceinline__ void build_marks(uint32_t* marks, const CsrUnion& un, int* row_heavy,
                                             int* row_cnt, const int32_t* cols, int S, int W0) {
+  constexpr int kThreads = 2 * ROWS;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int x = threadIdx.x; x < kRows * kMaskStride; x += kThreads) marks[x] = 0u;
+  for (int x = threadIdx.x; x < ROWS * kMaskStride; x += kThreads) marks[x] = 0u;
   __syncthreads();
-  for (int rr = warp; rr < kRows; rr += kThreads / 32) {
+  for (int rr = warp; rr < ROWS; rr += kThreads / 32) {
     const int n = csr_mark_row(marks + rr * kMaskStride, un.bitmap, un.wpre, cols, un.row_c0[rr], un.row_c1[rr],
                                S, W0, kWin);
     if (lane == 0) row_cnt[rr] = n;
   }
   __syncthreads();
-  if (threadIdx.x < kRows) {
+  if (threadIdx.x < ROWS) {
     const int x = threadIdx.x;
     int set = 0;
 #pragma unroll
@@ -121,8 +130,9 @@ __device__ __forceinline__ void build_marks(uint32_t* marks, const CsrUnion& un,
 
 // kcol[u - W0] = the column of union index u, for W0 <= u < min(U, W0 + kWin): a thread per
 // bitmap word walks its set bits.
+template <int THREADS>
 __device__ __forceinline__ void list_window_columns(int* kcol, const CsrUnion& un, int nw, int W0) {
-  for (int w = threadIdx.x; w < nw; w += kThreads) {
+  for (int w = threadIdx.x; w < nw; w += THREADS) {
     uint32_t bits = un.bitmap[w];
     int u = (int)un.wpre[w];
     if (u >= W0 + kWin || u + __popc(bits) <= W0) continue;
@@ -135,9 +145,10 @@ __device__ __forceinline__ void list_window_columns(int* kcol, const CsrUnion& u
   }
 }
 
-template <int D>
-__global__ void __launch_bounds__(kThreads, D == 64 ? 2 : 1) csr_f32_tiled_kernel(CsrArgs a) {
-  using C = F32Cfg<D>;
+template <int D, int ROWS>
+__global__ void __launch_bounds__(2 * ROWS, D == 64 ? 2 : 1) csr_f32_tiled_kernel(CsrArgs a) {
+  using C = F32Cfg<D, ROWS>;
+  constexpr int kRows = C::kRows, kThreads = C::kThreads, kPtStride = C::kPtStride;
   extern __shared__ __align__(16) uint8_t smem[];
   float* Qt = reinterpret_cast<float*>(smem + C::kQsOff);
   float* Ks = reinterpret_cast<float*>(smem + C::kKsOff);
@@ -212,15 +223,15 @@ __global__ void __launch_bounds__(kThreads, D == 64 ? 2 : 1) csr_f32_tiled_kerne
     if (t % kWinTiles == 0) {
       __syncthreads();  // the last window's marks, columns and buffers are read no more
       W0 = t * kKeys;
-      build_marks(marks, un, row_heavy, row_cnt, cols, S, W0);
-      list_window_columns(kcol, un, nw, W0);
+      build_marks<ROWS>(marks, un, row_heavy, row_cnt, cols, S, W0);
+      list_window_columns<kThreads>(kcol, un, nw, W0);
       __syncthreads();
-      stage_tile<D>(ks0 + b * kKsBuf, vs0 + b * kVsBuf, kcol, min(kKeys, U - W0), Kb, Vb);
+      stage_tile<D, ROWS>(ks0 + b * kKsBuf, vs0 + b * kVsBuf, kcol, min(kKeys, U - W0), Kb, Vb);
     }
     cp_async_wait_all();
     __syncthreads();  // tile t has landed for every thread; tile t-1's reads of K, V and P are done
     if (t + 1 < T && (t + 1) % kWinTiles != 0)
-      stage_tile<D>(ks0 + (b ^ 1) * kKsBuf, vs0 + (b ^ 1) * kVsBuf, kcol + (t + 1) * kKeys - W0,
+      stage_tile<D, ROWS>(ks0 + (b ^ 1) * kKsBuf, vs0 + (b ^ 1) * kVsBuf, kcol + (t + 1) * kKeys - W0,
                     min(kKeys, U - (t + 1) * kKeys), Kb, Vb);
     const float* Kt = Ks + b * (kKeys * C::kKStride);
     const float* Vt = Vs + b * (kKeys * D);
@@ -373,17 +384,78 @@ __global__ void __launch_bounds__(kThreads, D == 64 ? 2 : 1) csr_f32_tiled_kerne
   }
 }
 
-template <int D>
-cudaError_t launch_d(const CsrArgs& a, cudaStream_t st) {
-  using C = F32Cfg<D>;
-  cudaError_t e = cudaFuncSetAttribute(csr_f32_tiled_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       C::kSmemBytes);
-  if (e != cudaSuccess) return e;
-  const int64_t blocks = (int64_t)a.B * a.H * ((a.S + kRows - 1) / kRows);
+template <int D, int ROWS>
+cudaError_t launch_rows(const CsrArgs& a, cudaStream_t st) {
+  using C = F32Cfg<D, ROWS>;
+  const int64_t blocks = (int64_t)a.B * a.H * ((a.S + ROWS - 1) / ROWS);
   if (blocks <= 0) return cudaSuccess;
   if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-  csr_f32_tiled_kernel<D><<<(unsigned)blocks, kThreads, C::kSmemBytes, st>>>(a);
+  csr_f32_tiled_kernel<D, ROWS><<<(unsigned)blocks, C::kThreads, C::kSmemBytes, st>>>(a);
   return cudaGetLastError();
+}
+
+// Blocks of one instantiation resident on an SM at once (0 on error), looked up once per device.
+template <int D, int ROWS>
+int resident_blocks() {
+  constexpr int kMaxDevices = 64;
+  static std::atomic<int> cached[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 0;
+  int n = cached[dev].load(std::memory_order_acquire);
+  if (n > 0) return n;
+  using C = F32Cfg<D, ROWS>;
+  if (cudaFuncSetAttribute(csr_f32_tiled_kernel<D, ROWS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           C::kSmemBytes) != cudaSuccess)
+    return 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, csr_f32_tiled_kernel<D, ROWS>, C::kThreads,
+                                                    C::kSmemBytes) != cudaSuccess || n <= 0)
+    return 0;
+  cached[dev].store(n, std::memory_order_release);
+  return n;
+}
+
+// Rows per block: the blocks of a call run in rounds of (resident blocks per SM x SMs), and a
+// round takes about as long as one block. A block's time is a fixed part (taking the union of its
+// rows' columns and their marks: latency-bound, a warp per 16 rows, about as long as the tile
+// loop of kFixedRows rows on the window-and-stride pattern of 4,096 keys) plus its tile loop, in
+// proportion to its rows. The choice minimises rounds x (kFixedRows + ROWS) among the block sizes
+// that fit as many blocks on an SM as 128-row blocks do (fewer rows per block with more blocks per
+// SM would change the sharing the estimate assumes); on a tie the larger blocks win. On the
+// 148-SM B200 and 2 x 8 heads of 4,096 rows this picks 112 rows: 592 blocks, exactly two rounds of
+// 2 x 148, where 128-row blocks make 512 and leave 68 SMs with a fourth block after the others
+// are done (0.2936 -> 0.2875 ms measured).
+constexpr int kFixedRows = 74;
+
+template <int D>
+cudaError_t launch_d(const CsrArgs& a, cudaStream_t st, int num_sms) {
+  struct Cand {
+    int rows;
+    int resident;
+  };
+  const Cand cands[] = {{128, resident_blocks<D, 128>()}, {112, resident_blocks<D, 112>()},
+                        {96, resident_blocks<D, 96>()},   {80, resident_blocks<D, 80>()},
+                        {64, resident_blocks<D, 64>()}};
+  int best = 0;
+  int64_t best_cost = 0;
+  for (int c = 0; c < 5; ++c) {
+    if (cands[c].resident <= 0) return cudaErrorInvalidConfiguration;
+    if (cands[c].resident != cands[0].resident) continue;
+    const int64_t blocks = (int64_t)a.B * a.H * ((a.S + cands[c].rows - 1) / cands[c].rows);
+    const int64_t slots = (int64_t)cands[c].resident * (num_sms > 0 ? num_sms : 1);
+    const int64_t rounds = (blocks + slots - 1) / slots;
+    const int64_t cost = rounds * (kFixedRows + cands[c].rows);
+    if (c == 0 || cost < best_cost) {
+      best = c;
+      best_cost = cost;
+    }
+  }
+  switch (cands[best].rows) {
+    case 128: return launch_rows<D, 128>(a, st);
+    case 112: return launch_rows<D, 112>(a, st);
+    case 96: return launch_rows<D, 96>(a, st);
+    case 80: return launch_rows<D, 80>(a, st);
+    default: return launch_rows<D, 64>(a, st);
+  }
 }
 
 }  // namespace
@@ -395,7 +467,7 @@ bool sparse_csr_tiled_supported(const CsrArgs& a) {
 }
 
 cudaError_t launch_sparse_csr_tiled(const CsrArgs& a, cudaStream_t st) {
-  return a.D == 128 ? launch_d<128>(a, st) : launch_d<64>(a, st);
+  return a.D == 128 ? launch_d<128>(a, st, a.num_sms) : launch_d<64>(a, st, a.num_sms);
 }
 
 }  // namespace sdpa

@@ -39,6 +39,7 @@ struct CsrArgs {
   bool cols_vec;  // columns 16-byte aligned and nnz_cap % 4 == 0: read 4 indices at a time
   float* out;
   int* status;
+  int num_sms;   // SMs of the device (the tiled kernel sizes its blocks to fill whole rounds)
 };
 
 struct CsrTcArgs {  // attn_sparse_csr_tc: 16-bit q, k, v, out [B, H, S, D]
