@@ -113,10 +113,17 @@ __device__ __forceinline__ void build_marks(uint32_t* marks, const CsrUnion& un,
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int x = threadIdx.x; x < ROWS * kMaskStride; x += kThreads) marks[x] = 0u;
   __syncthreads();
-  for (int rr = warp; rr < ROWS; rr += kThreads / 32) {
-    const int n = csr_mark_row(marks + rr * kMaskStride, un.bitmap, un.wpre, cols, un.row_c0[rr], un.row_c1[rr],
-                               S, W0, kWin);
-    if (lane == 0) row_cnt[rr] = n;
+  // a warp takes its rows two at a time (the rows are a multiple of 16, the warps ROWS / 16)
+  constexpr int kWarps = kThreads / 32;
+  for (int rr = warp; rr < ROWS; rr += 2 * kWarps) {
+    const int r2 = rr + kWarps;
+    int na, nb;
+    csr_mark_row2(marks + rr * kMaskStride, marks + r2 * kMaskStride, un.bitmap, un.wpre, cols, un.row_c0[rr],
+                  un.row_c1[rr], un.row_c0[r2], un.row_c1[r2], S, W0, kWin, na, nb);
+    if (lane == 0) {
+      row_cnt[rr] = na;
+      row_cnt[r2] = nb;
+    }
   }
   __syncthreads();
   if (threadIdx.x < ROWS) {
