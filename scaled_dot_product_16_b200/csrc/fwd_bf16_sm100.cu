@@ -6,7 +6,9 @@
 // The pages name the FlashAttention algorithm (tiles of Q against streamed K/V tiles with an
 // online softmax) but give no kernel; this is a from-scratch sm_100a design:
 //
-//   * one block owns 256 query rows of one (sequence, head), as two 128-row tiles Q0 and Q1;
+//   * one block per SM takes work items one after another; an item is two 128-row tiles Q0 and
+//     Q1: the same rows of two query heads that share a KV head (GQA with an even group), else
+//     256 consecutive rows of one head;
 //   * K and V tiles (128 keys x D) stream through a ring of shared-memory stages, loaded by
 //     TMA with 128-byte swizzle (one issuing thread, no multicast);
 //   * one thread issues every tcgen05.mma: S_q = Q_q K_j^T (both operands in shared memory,
@@ -138,11 +140,12 @@ struct Cfg {
 constexpr int kSchedSlots = 256;
 __device__ int g_sched[kSchedSlots * 2];
 
-// One work item decoded: 256 query rows (two 128-row tiles) of query head h of sequence b.
+// One work item decoded: two 128-row Q tiles of sequence b (see pair_heads: the same rows of
+// query heads h and h + 1, or 256 consecutive rows of head h).
 struct Unit {
-  int b, h;          // sequence and query head; b < 0 marks the end of the block's work
+  int b, h;          // sequence and (first) query head; b < 0 marks the end of the block's work
   int q0, sq, sk;    // first query token and query length of the sequence; its key length
-  int row0;          // first row (within the sequence) of the 256 rows
+  int row0;          // first row (within the sequence) of Q0
   int rows0, rows1;  // rows of Q0 and Q1 (rows1 <= 0: no second tile)
   int jlo;           // first key tile (the band's first tile for row0; 0 otherwise)
   int n0, n1;        // key tiles from jlo up to Q0's / Q1's last visible key (n1 >= n0)
@@ -237,7 +240,17 @@ __device__ __forceinline__ void merge_into_stats(const FwdArgs& a, int64_t so, f
   *f_o *= cs0 * inv;
 }
 
-// Decodes item x. Items run query-head fastest; for BHSD the 256-row blocks go by level (the
+// The two Q tiles of an item: with an even number of query heads per KV head (GQA), the same 128
+// rows of two query heads of one group (h, h + 1), which need exactly the same key tiles and read
+// the same K/V; otherwise 256 consecutive rows of one head (Q1 the second 128).
+__host__ __device__ __forceinline__ bool pair_heads(const FwdArgs& a) {
+  return a.Nkv > 0 && (a.Nq / a.Nkv) % 2 == 0;
+}
+__host__ __device__ __forceinline__ int rows_per_item(const FwdArgs& a) {
+  return pair_heads(a) ? kBM : kRowsPerBlock;
+}
+
+// Decodes item x. Items run query-head (pair) fastest; for BHSD the row blocks go by level (the
 // last row block of every sequence first), for TND sequence by sequence with each sequence's last
 // row block first, so that the heaviest items of a sequence come first. Run by one full warp;
 // every lane gets the result. Returns false for an item past the last row block (an item there
@@ -246,8 +259,11 @@ __device__ __forceinline__ void merge_into_stats(const FwdArgs& a, int64_t so, f
 template <int EXT>
 __device__ __forceinline__ bool decode_unit(const FwdArgs& a, int units_per_seq, int x, Unit& U, int& k0) {
   const int lane = threadIdx.x & 31;
-  const int h = x % a.Nq;
-  const int y = x / a.Nq;
+  const bool pair = pair_heads(a);
+  const int rows = rows_per_item(a);
+  const int heads = pair ? a.Nq / 2 : a.Nq;  // items per row block
+  const int h = pair ? 2 * (x % heads) : x % heads;
+  const int y = x / heads;
   int b = 0, u = 0;
   bool ok = true;
   if (a.layout == ATTN_BHSD) {
@@ -258,11 +274,11 @@ __device__ __forceinline__ bool decode_unit(const FwdArgs& a, int units_per_seq,
   } else {
     bool bad;
     int t;
-    ok = warp_find_tile(a.cu_q, a.B, a.Sq, kRowsPerBlock, y, &b, &t, a.status, &bad);
+    ok = warp_find_tile(a.cu_q, a.B, a.Sq, rows, y, &b, &t, a.status, &bad);
     if (ok) {
       int qs, ql;
       seq_span(a.cu_q, b, &qs, &ql);
-      u = (ql + kRowsPerBlock - 1) / kRowsPerBlock - 1 - t;
+      u = (ql + rows - 1) / rows - 1 - t;
     } else if (!bad && h == 0) {
       int sb, st;
       bool bad2;
@@ -272,7 +288,7 @@ __device__ __forceinline__ bool decode_unit(const FwdArgs& a, int units_per_seq,
   if (!ok) return false;
   U.b = b;
   U.h = h;
-  U.row0 = u * kRowsPerBlock;
+  U.row0 = u * rows;
   if (a.layout == ATTN_BHSD) {
     U.q0 = 0;
     U.sq = a.Sq;
@@ -287,16 +303,17 @@ __device__ __forceinline__ bool decode_unit(const FwdArgs& a, int units_per_seq,
     }
   }
   U.rows0 = min(kBM, U.sq - U.row0);
-  U.rows1 = min(kBM, U.sq - U.row0 - kBM);
+  U.rows1 = pair ? U.rows0 : min(kBM, U.sq - U.row0 - kBM);
   const bool has1 = U.rows1 > 0;
+  const int r1 = pair ? U.row0 : U.row0 + kBM;  // Q1's first row
   // Key tiles run from jlo to the tile holding each Q tile's last visible key; n0 and n1 count
   // tiles from jlo. With the band, Q1 starts at its own first tile: s1 tiles after jlo.
   U.jlo = EXT >= 1 ? visible_begin(a.mask_mode, U.row0, a.pre) / kBN : 0;
   const int kv_end0 = visible_end(a.mask_mode, U.row0 + U.rows0 - 1, U.sq, U.sk, a.next);
-  const int kv_end1 = has1 ? visible_end(a.mask_mode, U.row0 + kBM + U.rows1 - 1, U.sq, U.sk, a.next) : 0;
+  const int kv_end1 = has1 ? visible_end(a.mask_mode, r1 + U.rows1 - 1, U.sq, U.sk, a.next) : 0;
   U.n0 = max((kv_end0 + kBN - 1) / kBN, U.jlo) - U.jlo;
   U.n1 = has1 ? max((kv_end1 + kBN - 1) / kBN, U.jlo) - U.jlo : U.n0;
-  U.s1 = EXT >= 1 && has1 ? visible_begin(a.mask_mode, U.row0 + kBM, a.pre) / kBN - U.jlo : 0;
+  U.s1 = EXT >= 1 && has1 ? visible_begin(a.mask_mode, r1, a.pre) / kBN - U.jlo : 0;
   return true;
 }
 
@@ -426,7 +443,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t qbar = bar_addr(&bars->q_full);
             mbar_arrive_expect_tx(qbar, (has1 ? 2 : 1) * C::kTileBytes);
             load_tile(&tm_q, sQ, qbar, U.q0 + U.row0, qhead, C::kBoxes);
-            if (has1) load_tile(&tm_q, sQ + C::kTileBytes, qbar, U.q0 + U.row0 + kBM, qhead, C::kBoxes);
+            if (has1) {
+              if (pair_heads(a))
+                load_tile(&tm_q, sQ + C::kTileBytes, qbar, U.q0 + U.row0, qhead + 1, C::kBoxes);
+              else
+                load_tile(&tm_q, sQ + C::kTileBytes, qbar, U.q0 + U.row0 + kBM, qhead, C::kBoxes);
+            }
             ++qn;
           }
           for (int i = first; ok && i < nl; ++i) ok = load_kv(i);
@@ -573,7 +595,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int jlo = w.jlo;
       const int j0 = q == 0 ? 0 : w.s1;              // this Q tile's key tiles: j0 .. n-1
       const int n = q == 0 ? w.n0 : (has1 ? w.n1 : 0);
-      const int i = w.row0 + q * kBM + r;            // row within the sequence
+      const bool pair = pair_heads(a);
+      const int i = w.row0 + (pair ? 0 : q * kBM) + r;  // row within the sequence
+      const int hq = w.h + (pair ? q : 0);              // query head of this Q tile
       const int lim = i < w.sq ? visible_end(a.mask_mode, i, w.sq, w.sk, a.next) : w.sk;
       const int lo = EXT >= 1 && i < w.sq ? visible_begin(a.mask_mode, i, a.pre) : 0;
       // explicit mask row of this query (rows past the sequence read none)
@@ -732,8 +756,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         float f_prev = 0.f;               // factor on the accumulator's previous output row
         int64_t orow, so;
         if (a.acc_mode == kAccNone) {
-          orow = bhsd ? (((int64_t)w.b * a.Nq + w.h) * a.Sq + i) * HDV : ((int64_t)(w.q0 + i) * a.Nq + w.h) * HDV;
-          so = bhsd ? ((int64_t)w.b * a.Nq + w.h) * a.Sq + i : (int64_t)(w.q0 + i) * a.Nq + w.h;
+          orow = bhsd ? (((int64_t)w.b * a.Nq + hq) * a.Sq + i) * HDV : ((int64_t)(w.q0 + i) * a.Nq + hq) * HDV;
+          so = bhsd ? ((int64_t)w.b * a.Nq + hq) * a.Sq + i : (int64_t)(w.q0 + i) * a.Nq + hq;
           if (store && a.smax != nullptr) {
             a.smax[so] = m_loc;
             a.ssum[so] = l_loc;
@@ -741,8 +765,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         } else {
           // accumulator in the merge layouts: BHSD -> output [Sq, B, Nq*D] (SBH), statistics
           // [B, Nq, Sq, 8]; TND -> output [T, Nq*D], statistics [T, Nq, 8]
-          orow = bhsd ? (((int64_t)i * a.B + w.b) * a.Nq + w.h) * HDV : ((int64_t)(w.q0 + i) * a.Nq + w.h) * HDV;
-          so = (bhsd ? ((int64_t)w.b * a.Nq + w.h) * a.Sq + i : (int64_t)(w.q0 + i) * a.Nq + w.h) * 8;
+          orow = bhsd ? (((int64_t)i * a.B + w.b) * a.Nq + hq) * HDV : ((int64_t)(w.q0 + i) * a.Nq + hq) * HDV;
+          so = (bhsd ? ((int64_t)w.b * a.Nq + hq) * a.Sq + i : (int64_t)(w.q0 + i) * a.Nq + hq) * 8;
           if (store) merge_into_stats(a, so, m_loc, l_loc, &f_prev, &f_o);
         }
         // the output row leaves TMEM 64 columns per round trip (two loads, then one wait)
@@ -936,12 +960,12 @@ cudaError_t launch_hd(const FwdArgs& a, cudaStream_t st) {
   int units_per_seq = 0;
   int64_t units;
   if (a.layout == ATTN_BHSD) {
-    units_per_seq = (a.Sq + kRowsPerBlock - 1) / kRowsPerBlock;
+    units_per_seq = (a.Sq + rows_per_item(a) - 1) / rows_per_item(a);
     units = (int64_t)a.B * units_per_seq;
   } else {
-    units = (a.Sq + kRowsPerBlock - 1) / kRowsPerBlock + a.B;
+    units = (a.Sq + rows_per_item(a) - 1) / rows_per_item(a) + a.B;
   }
-  const int64_t items = units * a.Nq;
+  const int64_t items = units * (pair_heads(a) ? a.Nq / 2 : a.Nq);
   if (items <= 0) return cudaSuccess;
   if (items > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
   const float scale_log2 = a.scale * 1.4426950408889634f;
