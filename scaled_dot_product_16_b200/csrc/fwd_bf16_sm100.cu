@@ -122,7 +122,9 @@ struct Cfg {
   static constexpr int kQOff = 0;
   static constexpr int kKVOff = 2 * kTileBytes;
   static constexpr int kBarOff = kKVOff + kStages * kTileBytes;
-  static constexpr int kSmemBytes = kBarOff + 512 + 1024;  // barriers + 1 KB for alignment
+  // output staging for the TMA stores: 4 KB (32 rows x 64 columns, 128-byte swizzle) per softmax warp
+  static constexpr int kStageOff = kBarOff + 1024;
+  static constexpr int kSmemBytes = kStageOff + 8 * 4096 + 1024;  // + 1 KB for alignment
   static_assert(kStages >= 2 && kStages <= 8, "barrier arrays hold 8 stages");
   static_assert(kSmemBytes <= 232448, "227 KB of shared memory per block");
   static constexpr uint32_t kFmt = F16 ? 0u : 1u;  // instruction-descriptor operand format
@@ -329,7 +331,8 @@ __device__ __forceinline__ bool decode_unit(const FwdArgs& a, int units_per_seq,
 template <int HD, int HDV, bool F16, int EXT>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                    const __grid_constant__ CUtensorMap tm_v, FwdArgs a, int units_per_seq,
+                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+                    FwdArgs a, int units_per_seq,
                     float scale_log2, int n_items, int* sched) {
   using C = Cfg<HD, HDV, F16>;
   extern __shared__ uint8_t smem_raw[];
@@ -769,6 +772,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           so = (bhsd ? ((int64_t)w.b * a.Nq + hq) * a.Sq + i : (int64_t)(w.q0 + i) * a.Nq + hq) * 8;
           if (store) merge_into_stats(a, so, m_loc, l_loc, &f_prev, &f_o);
         }
+        // A warp whose 32 rows all lie in the sequence writes its plain output through its
+        // shared-memory slot, 64 columns at a time, with a TMA store of the 32 x 64 box (the
+        // layout the tensor map's 128-byte swizzle expects); otherwise each thread stores its row.
+        const bool tma_out = a.acc_mode == kAccNone && __all_sync(0xffffffffu, store);
+        const uint32_t stg = smem_u32(smem + C::kStageOff) + (uint32_t)warp * 4096u;
+        const int wrow0 = i - lane;  // the warp's first row within the sequence
         // the output row leaves TMEM 64 columns per round trip (two loads, then one wait)
         uint32_t oc[2][32];
 #pragma unroll
@@ -781,6 +790,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             } else {
 #pragma unroll
               for (int x = 0; x < 32; ++x) oc[0][x] = oc[1][x] = 0u;
+            }
+            if (tma_out) {
+              // the slot's previous TMA store (the last 64 columns, or the previous item's) must
+              // have read it; that wait overlaps the TMEM loads above
+              if (lane == 0) bulk_wait_read0();
+              __syncwarp();
             }
           }
           const uint32_t (&o)[32] = oc[c & 1];
@@ -809,9 +824,29 @@ __global__ void __launch_bounds__(kThreads, 1)
               }
               pkd[x] = pack16x2<F16>(v0, v1);
             }
+            if (tma_out) {
 #pragma unroll
-            for (int x = 0; x < 4; ++x)
-              dst[x] = make_uint4(pkd[4 * x], pkd[4 * x + 1], pkd[4 * x + 2], pkd[4 * x + 3]);
+              for (int x = 0; x < 4; ++x) {
+                const uint32_t chunk = (uint32_t)(((c & 1) * 4 + x) ^ (lane & 7));
+                st_shared_v4(stg + (uint32_t)lane * 128u + chunk * 16u, pkd[4 * x], pkd[4 * x + 1], pkd[4 * x + 2],
+                             pkd[4 * x + 3]);
+              }
+            } else {
+#pragma unroll
+              for (int x = 0; x < 4; ++x)
+                dst[x] = make_uint4(pkd[4 * x], pkd[4 * x + 1], pkd[4 * x + 2], pkd[4 * x + 3]);
+            }
+          }
+          if (tma_out && (c & 1) == 1) {
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              if (bhsd)
+                tma_store_3d(&tm_o, stg, 64 * (c >> 1), wrow0, w.b * a.Nq + hq);
+              else
+                tma_store_3d(&tm_o, stg, 64 * (c >> 1), hq, w.q0 + wrow0);
+              bulk_commit();
+            }
           }
         }
       }
@@ -819,6 +854,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(bar_addr(&bars->unit_empty[slot]));
       }
+      if (lane == 0) bulk_wait0();  // this warp's output stores are complete before it exits
     }
 
   // ---- teardown ----------------------------------------------------------------------------
@@ -937,6 +973,14 @@ cudaError_t launch_hd(const FwdArgs& a, cudaStream_t st) {
          make_map(&tk, a.k, D, a.Nkv, tk_rows, D * 2, (uint64_t)a.Nkv * D * 2, 1, kBN, F16) &&
          make_map(&tv, a.v, Dv, a.Nkv, tk_rows, Dv * 2, (uint64_t)a.Nkv * Dv * 2, 1, kBN, F16);
   }
+  // the plain output has Q's layout with the value head size; the TMA stores write 32-row boxes
+  CUtensorMap to = tq;  // not read by the kernel when the output is an accumulator
+  if (ok && a.acc_mode == 0) {
+    if (a.layout == ATTN_BHSD)
+      ok = make_map(&to, a.out, Dv, a.Sq, (uint64_t)a.B * a.Nq, Dv * 2, (uint64_t)a.Sq * Dv * 2, 32, 1, F16);
+    else
+      ok = make_map(&to, a.out, Dv, a.Nq, a.Sq > 0 ? a.Sq : 1, Dv * 2, (uint64_t)a.Nq * Dv * 2, 1, 32, F16);
+  }
   if (!ok) return cudaErrorInvalidValue;
   auto kernel = a.mask != nullptr                 ? fwd_bf16_kernel<HD, HDV, F16, 2>
                 : a.mask_mode == ATTN_MASK_BAND ? fwd_bf16_kernel<HD, HDV, F16, 1>
@@ -974,7 +1018,7 @@ cudaError_t launch_hd(const FwdArgs& a, cudaStream_t st) {
   int* sched = nullptr;
   cudaError_t se = sched_slot(st, &sched);
   if (se != cudaSuccess) return se;
-  kernel<<<(unsigned)grid, kThreads, C::kSmemBytes, st>>>(tq, tk, tv, a, units_per_seq, scale_log2, (int)items,
+  kernel<<<(unsigned)grid, kThreads, C::kSmemBytes, st>>>(tq, tk, tv, to, a, units_per_seq, scale_log2, (int)items,
                                                            sched);
   return cudaGetLastError();
 }
