@@ -29,6 +29,11 @@
  *   - Results are deterministic: the same inputs give bitwise-identical outputs (no atomics
  *     take part in any result).
  *   - Every function is thread-safe; calls on different streams may overlap.
+ *   - No call allocates device memory. The library's own device memory, per device: the status
+ *     word, the work counters of attn_fwd's persistent grid (one pair for each of the first 256
+ *     streams that call it; launches on further streams, and launches being captured into a CUDA
+ *     graph, divide their work statically instead, with the same results) and the fixed scratch
+ *     of attn_sparse_csr_tc_noalloc.
  *
  * Softmax statistics (all calls): softmax_max is max_j s_ij, with s_ij = scale * q_i . k_j, in
  * natural-log units; softmax_sum is sum_j exp(s_ij - softmax_max). A row that sees no key has
