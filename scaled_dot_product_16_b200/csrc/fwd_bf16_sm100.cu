@@ -378,204 +378,204 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t sKV = smem_u32(smem + C::kKVOff);
 
   if (warp >= 8) {
-  // the producer warpgroup gives registers to the softmax warpgroups (each branch sets its own
-  // count first, so that the code after it is compiled for that count)
-  setmaxnreg_dec<kRegsProducer>();
-  if (warp == kTmaWarp) {
-    // =============================== TMA producer (and item decoder) ===========================
-    const bool bhsd = a.layout == ATTN_BHSD;
-    if (lane == 0) {
-      tma_prefetch_desc(&tm_q);
-      tma_prefetch_desc(&tm_k);
-      tma_prefetch_desc(&tm_v);
-    }
-    auto load_tile = [&](const CUtensorMap* map, uint32_t dst, uint32_t bar, int tok, int head, int boxes) {
-      for (int x = 0; x < boxes; ++x) {
-        if (bhsd)
-          tma_load_3d(dst + x * (kBM * 128), map, bar, x * 64, tok, head);
-        else
-          tma_load_3d(dst + x * (kBM * 128), map, bar, x * 64, head, tok);
+    // the producer warpgroup gives registers to the softmax warpgroups (each branch sets its own
+    // count first, so that the code after it is compiled for that count)
+    setmaxnreg_dec<kRegsProducer>();
+    if (warp == kTmaWarp) {
+      // =============================== TMA producer (and item decoder) ===========================
+      const bool bhsd = a.layout == ATTN_BHSD;
+      if (lane == 0) {
+        tma_prefetch_desc(&tm_q);
+        tma_prefetch_desc(&tm_k);
+        tma_prefetch_desc(&tm_v);
       }
-    };
-    uint32_t it = 0;  // K/V tiles issued by this block: position in the ring
-    int qn = 0;       // Q loads issued
-    int k = 0;        // items handed out
-    bool ok = true;
-    int64_t x = blockIdx.x;
-    for (;;) {
-      Unit U;
-      int k0 = 0;
-      const bool end = x >= n_items;
-      const bool live = !end && decode_unit<EXT>(a, units_per_seq, (int)x, U, k0);
-      if (end || live) {
-        // hand the item (or the end mark) to the other roles through slot k % kUnitSlots
-        if (lane == 0) {
-          const int slot = k % kUnitSlots;
-          if (k >= kUnitSlots)
-            ok = wait_bar(bar_addr(&bars->unit_empty[slot]), ((k / kUnitSlots) - 1) & 1, abort, a.status);
-          if (ok) {
-            if (end) bars->units[slot].b = -1;
-            else bars->units[slot] = U;
-            mbar_arrive(bar_addr(&bars->unit_full[slot]));  // releases the slot's contents
-          }
+      auto load_tile = [&](const CUtensorMap* map, uint32_t dst, uint32_t bar, int tok, int head, int boxes) {
+        for (int x = 0; x < boxes; ++x) {
+          if (bhsd)
+            tma_load_3d(dst + x * (kBM * 128), map, bar, x * 64, tok, head);
+          else
+            tma_load_3d(dst + x * (kBM * 128), map, bar, x * 64, head, tok);
         }
-        ok = __shfl_sync(0xffffffffu, ok, 0) != 0;
-        ++k;
-        if (!ok || end) break;
-        if (lane == 0 && U.n1 > 0) {
-          const int g = U.h / (a.Nq / a.Nkv);
-          const int qhead = bhsd ? U.b * a.Nq + U.h : U.h;
-          const int khead = bhsd ? U.b * a.Nkv + g : g;
-          const int nl = 2 * U.n1;
-          // K0, V0, K1, V1, ... through the ring; Q once the previous item's last S has run
-          auto load_kv = [&](int i) {
-            const uint32_t s = it % C::kStages, r = it / C::kStages;
-            if (r > 0 && !wait_bar(bar_addr(&bars->kv_empty[s]), (r - 1) & 1, abort, a.status)) return false;
-            const uint32_t fb = bar_addr(&bars->kv_full[s]);
-            mbar_arrive_expect_tx(fb, (i & 1) ? C::kTileBytesV : C::kTileBytes);
-            load_tile((i & 1) ? &tm_v : &tm_k, sKV + s * C::kTileBytes, fb, k0 + (U.jlo + (i >> 1)) * kBN, khead,
-                      (i & 1) ? C::kBoxesV : C::kBoxes);
-            ++it;
-            return true;
-          };
-          const int first = min(2, nl);
-          for (int i = 0; ok && i < first; ++i) ok = load_kv(i);
-          if (ok && qn > 0) ok = wait_bar(bar_addr(&bars->q_empty), (qn - 1) & 1, abort, a.status);
-          if (ok) {
-            const bool has1 = U.rows1 > 0;
-            const uint32_t qbar = bar_addr(&bars->q_full);
-            mbar_arrive_expect_tx(qbar, (has1 ? 2 : 1) * C::kTileBytes);
-            load_tile(&tm_q, sQ, qbar, U.q0 + U.row0, qhead, C::kBoxes);
-            if (has1) {
-              if (pair_heads(a))
-                load_tile(&tm_q, sQ + C::kTileBytes, qbar, U.q0 + U.row0, qhead + 1, C::kBoxes);
-              else
-                load_tile(&tm_q, sQ + C::kTileBytes, qbar, U.q0 + U.row0 + kBM, qhead, C::kBoxes);
-            }
-            ++qn;
-          }
-          for (int i = first; ok && i < nl; ++i) ok = load_kv(i);
-        }
-        ok = __shfl_sync(0xffffffffu, ok, 0) != 0;
-        if (!ok) break;
-      }
-      int64_t nx = 0;
-      if (lane == 0) nx = sched != nullptr ? (int64_t)gridDim.x + atomicAdd(sched, 1) : x + gridDim.x;
-      x = __shfl_sync(0xffffffffu, nx, 0);
-    }
-    if (lane == 0) {
-      // drain: every load this thread issued must have landed before the block exits
-      for (uint32_t i = it > (uint32_t)C::kStages ? it - C::kStages : 0u; i < it; ++i)
-        wait_bar(bar_addr(&bars->kv_full[i % C::kStages]), (i / C::kStages) & 1, abort, a.status, false);
-      if (qn > 0) wait_bar(bar_addr(&bars->q_full), (qn - 1) & 1, abort, a.status, false);
-    }
-  } else if (warp == kMmaWarp) {
-    // =============================== MMA issue ==========================================
-    if (lane == 0) {
-      const uint32_t S0 = tmem, S1 = tmem + 128, O0 = tmem + 256, O1 = tmem + 256 + HDV;
-      // Descriptors are built once. K-step kk of an operand adds a constant to the start
-      // address field (shared-memory addresses stay below 256 KB, so the 14-bit field never
-      // carries), which keeps the issue loop at a few instructions per MMA.
-      const uint64_t dq0 = smem_desc_sw128(sQ, 16, 1024);
-      const uint64_t dq1 = dq0 + (uint64_t)(C::kTileBytes >> 4);
-      const uint64_t dk0 = smem_desc_sw128(sKV, 16, 1024);
-      const uint64_t dv0 = smem_desc_sw128(sKV, kBN * 128, 1024);
-      const uint32_t kvfull0 = bar_addr(&bars->kv_full[0]), kvempty0 = bar_addr(&bars->kv_empty[0]);
-      auto full = [&](uint32_t i) {
-        return wait_bar(kvfull0 + 8 * (i % C::kStages), (i / C::kStages) & 1, abort, a.status);
       };
-      auto release = [&](uint32_t i) { mma_commit(kvempty0 + 8 * (i % C::kStages)); };
-      auto issue_qk = [&](uint32_t d, uint64_t dq, uint32_t i) {
-        const uint64_t dk = dk0 + (uint64_t)(((i % C::kStages) * C::kTileBytes) >> 4);
-        if constexpr (HD == 128)
-          mma_ss_chain8(d, dq, dk, C::kIdescQK, 0u);
-        else
-          mma_ss_chain4(d, dq, dk, C::kIdescQK, 0u);
-      };
-      auto issue_pv = [&](uint32_t d, uint32_t p_tmem, uint32_t i, bool acc) {
-        const uint64_t dv = dv0 + (uint64_t)(((i % C::kStages) * C::kTileBytes) >> 4);
-        mma_ts_chain8(d, p_tmem, dv, C::kIdescPV, acc ? 1u : 0u);
-      };
+      uint32_t it = 0;  // K/V tiles issued by this block: position in the ring
+      int qn = 0;       // Q loads issued
+      int k = 0;        // items handed out
       bool ok = true;
-      if constexpr (SDPA_TEST_STALL != 0) ok = wait_bar(bar_addr(&bars->stall), 0, abort, a.status);
-      uint32_t it = 0;        // K/V tiles consumed (the same sequence the TMA warp issues)
-      int qn = 0;             // Q loads consumed
-      uint32_t pc0 = 0, pc1 = 0;  // P hand-offs taken from each softmax warpgroup
-      for (int k = 0; ok; ++k) {
-        const int slot = k % kUnitSlots;
-        if (!(ok = wait_bar(bar_addr(&bars->unit_full[slot]), (k / kUnitSlots) & 1, abort, a.status))) break;
-        const Unit* us = &bars->units[slot];
-        const int ub = us->b, n0 = us->n0, n1 = us->n1, s1 = us->s1;
-        const bool has1 = us->rows1 > 0;
-        mbar_arrive(bar_addr(&bars->unit_empty[slot]));
-        if (ub < 0) break;
-        if (n1 <= 0) continue;
-        // Q1 works on key tiles s1 .. n1-1 (s1 = 0 except with the band)
-        auto act1 = [&](int j) { return has1 && j >= s1; };
-        // after the S MMAs of the item's last key tile: Q may be overwritten once they have run
-        auto after_s = [&](int t) {
-          if (t == n1 - 1) mma_commit(bar_addr(&bars->q_empty));
-        };
-        ok = wait_bar(bar_addr(&bars->q_full), qn & 1, abort, a.status);
-        ++qn;
-        if (ok) ok = full(it);
-        if (!ok) break;
-        tc_fence_after();
-        if (n0 > 0) {
-          issue_qk(S0, dq0, it);
-          mma_commit(bar_addr(&bars->s_full[0]));
-        }
-        if (act1(0)) {
-          issue_qk(S1, dq1, it);
-          mma_commit(bar_addr(&bars->s_full[1]));
-        }
-        after_s(0);
-        release(it);
-        for (int j = 0; ok && j < n1; ++j) {
-          const uint32_t iv = it + 2 * j + 1, ik = it + 2 * j + 2;
-          if (!(ok = full(iv))) break;
-          tc_fence_after();
-          if (j < n0) {
-            if (!(ok = wait_bar(bar_addr(&bars->p_ready[0]), pc0 & 1, abort, a.status))) break;
-            ++pc0;
-            tc_fence_after();
-            issue_pv(O0, S0, iv, j > 0);
-            if (j == n0 - 1) mma_commit(bar_addr(&bars->o_done[0]));
-          }
-          const bool next = j + 1 < n1;
-          if (next) {
-            if (!(ok = full(ik))) break;
-            tc_fence_after();
-            if (j + 1 < n0) {
-              issue_qk(S0, dq0, ik);
-              mma_commit(bar_addr(&bars->s_full[0]));
+      int64_t x = blockIdx.x;
+      for (;;) {
+        Unit U;
+        int k0 = 0;
+        const bool end = x >= n_items;
+        const bool live = !end && decode_unit<EXT>(a, units_per_seq, (int)x, U, k0);
+        if (end || live) {
+          // hand the item (or the end mark) to the other roles through slot k % kUnitSlots
+          if (lane == 0) {
+            const int slot = k % kUnitSlots;
+            if (k >= kUnitSlots)
+              ok = wait_bar(bar_addr(&bars->unit_empty[slot]), ((k / kUnitSlots) - 1) & 1, abort, a.status);
+            if (ok) {
+              if (end) bars->units[slot].b = -1;
+              else bars->units[slot] = U;
+              mbar_arrive(bar_addr(&bars->unit_full[slot]));  // releases the slot's contents
             }
           }
-          if (act1(j)) {
-            if (!(ok = wait_bar(bar_addr(&bars->p_ready[1]), pc1 & 1, abort, a.status))) break;
-            ++pc1;
-            tc_fence_after();
-            issue_pv(O1, S1, iv, j > s1);
-            if (j == n1 - 1) mma_commit(bar_addr(&bars->o_done[1]));
-          }
-          release(iv);
-          if (next) {
-            if (act1(j + 1)) {
-              issue_qk(S1, dq1, ik);
-              mma_commit(bar_addr(&bars->s_full[1]));
+          ok = __shfl_sync(0xffffffffu, ok, 0) != 0;
+          ++k;
+          if (!ok || end) break;
+          if (lane == 0 && U.n1 > 0) {
+            const int g = U.h / (a.Nq / a.Nkv);
+            const int qhead = bhsd ? U.b * a.Nq + U.h : U.h;
+            const int khead = bhsd ? U.b * a.Nkv + g : g;
+            const int nl = 2 * U.n1;
+            // K0, V0, K1, V1, ... through the ring; Q once the previous item's last S has run
+            auto load_kv = [&](int i) {
+              const uint32_t s = it % C::kStages, r = it / C::kStages;
+              if (r > 0 && !wait_bar(bar_addr(&bars->kv_empty[s]), (r - 1) & 1, abort, a.status)) return false;
+              const uint32_t fb = bar_addr(&bars->kv_full[s]);
+              mbar_arrive_expect_tx(fb, (i & 1) ? C::kTileBytesV : C::kTileBytes);
+              load_tile((i & 1) ? &tm_v : &tm_k, sKV + s * C::kTileBytes, fb, k0 + (U.jlo + (i >> 1)) * kBN, khead,
+                        (i & 1) ? C::kBoxesV : C::kBoxes);
+              ++it;
+              return true;
+            };
+            const int first = min(2, nl);
+            for (int i = 0; ok && i < first; ++i) ok = load_kv(i);
+            if (ok && qn > 0) ok = wait_bar(bar_addr(&bars->q_empty), (qn - 1) & 1, abort, a.status);
+            if (ok) {
+              const bool has1 = U.rows1 > 0;
+              const uint32_t qbar = bar_addr(&bars->q_full);
+              mbar_arrive_expect_tx(qbar, (has1 ? 2 : 1) * C::kTileBytes);
+              load_tile(&tm_q, sQ, qbar, U.q0 + U.row0, qhead, C::kBoxes);
+              if (has1) {
+                if (pair_heads(a))
+                  load_tile(&tm_q, sQ + C::kTileBytes, qbar, U.q0 + U.row0, qhead + 1, C::kBoxes);
+                else
+                  load_tile(&tm_q, sQ + C::kTileBytes, qbar, U.q0 + U.row0 + kBM, qhead, C::kBoxes);
+              }
+              ++qn;
             }
-            after_s(j + 1);
-            release(ik);
+            for (int i = first; ok && i < nl; ++i) ok = load_kv(i);
           }
+          ok = __shfl_sync(0xffffffffu, ok, 0) != 0;
+          if (!ok) break;
         }
-        it += 2 * n1;
+        int64_t nx = 0;
+        if (lane == 0) nx = sched != nullptr ? (int64_t)gridDim.x + atomicAdd(sched, 1) : x + gridDim.x;
+        x = __shfl_sync(0xffffffffu, nx, 0);
       }
-      if (!ok) *abort = 1;
-      // every MMA and commit issued above must have completed before TMEM is freed
-      mma_commit(bar_addr(&bars->drain));
-      wait_bar(bar_addr(&bars->drain), 0, abort, a.status, false);
+      if (lane == 0) {
+        // drain: every load this thread issued must have landed before the block exits
+        for (uint32_t i = it > (uint32_t)C::kStages ? it - C::kStages : 0u; i < it; ++i)
+          wait_bar(bar_addr(&bars->kv_full[i % C::kStages]), (i / C::kStages) & 1, abort, a.status, false);
+        if (qn > 0) wait_bar(bar_addr(&bars->q_full), (qn - 1) & 1, abort, a.status, false);
+      }
+    } else if (warp == kMmaWarp) {
+      // =============================== MMA issue ==========================================
+      if (lane == 0) {
+        const uint32_t S0 = tmem, S1 = tmem + 128, O0 = tmem + 256, O1 = tmem + 256 + HDV;
+        // Descriptors are built once. K-step kk of an operand adds a constant to the start
+        // address field (shared-memory addresses stay below 256 KB, so the 14-bit field never
+        // carries), which keeps the issue loop at a few instructions per MMA.
+        const uint64_t dq0 = smem_desc_sw128(sQ, 16, 1024);
+        const uint64_t dq1 = dq0 + (uint64_t)(C::kTileBytes >> 4);
+        const uint64_t dk0 = smem_desc_sw128(sKV, 16, 1024);
+        const uint64_t dv0 = smem_desc_sw128(sKV, kBN * 128, 1024);
+        const uint32_t kvfull0 = bar_addr(&bars->kv_full[0]), kvempty0 = bar_addr(&bars->kv_empty[0]);
+        auto full = [&](uint32_t i) {
+          return wait_bar(kvfull0 + 8 * (i % C::kStages), (i / C::kStages) & 1, abort, a.status);
+        };
+        auto release = [&](uint32_t i) { mma_commit(kvempty0 + 8 * (i % C::kStages)); };
+        auto issue_qk = [&](uint32_t d, uint64_t dq, uint32_t i) {
+          const uint64_t dk = dk0 + (uint64_t)(((i % C::kStages) * C::kTileBytes) >> 4);
+          if constexpr (HD == 128)
+            mma_ss_chain8(d, dq, dk, C::kIdescQK, 0u);
+          else
+            mma_ss_chain4(d, dq, dk, C::kIdescQK, 0u);
+        };
+        auto issue_pv = [&](uint32_t d, uint32_t p_tmem, uint32_t i, bool acc) {
+          const uint64_t dv = dv0 + (uint64_t)(((i % C::kStages) * C::kTileBytes) >> 4);
+          mma_ts_chain8(d, p_tmem, dv, C::kIdescPV, acc ? 1u : 0u);
+        };
+        bool ok = true;
+        if constexpr (SDPA_TEST_STALL != 0) ok = wait_bar(bar_addr(&bars->stall), 0, abort, a.status);
+        uint32_t it = 0;        // K/V tiles consumed (the same sequence the TMA warp issues)
+        int qn = 0;             // Q loads consumed
+        uint32_t pc0 = 0, pc1 = 0;  // P hand-offs taken from each softmax warpgroup
+        for (int k = 0; ok; ++k) {
+          const int slot = k % kUnitSlots;
+          if (!(ok = wait_bar(bar_addr(&bars->unit_full[slot]), (k / kUnitSlots) & 1, abort, a.status))) break;
+          const Unit* us = &bars->units[slot];
+          const int ub = us->b, n0 = us->n0, n1 = us->n1, s1 = us->s1;
+          const bool has1 = us->rows1 > 0;
+          mbar_arrive(bar_addr(&bars->unit_empty[slot]));
+          if (ub < 0) break;
+          if (n1 <= 0) continue;
+          // Q1 works on key tiles s1 .. n1-1 (s1 = 0 except with the band)
+          auto act1 = [&](int j) { return has1 && j >= s1; };
+          // after the S MMAs of the item's last key tile: Q may be overwritten once they have run
+          auto after_s = [&](int t) {
+            if (t == n1 - 1) mma_commit(bar_addr(&bars->q_empty));
+          };
+          ok = wait_bar(bar_addr(&bars->q_full), qn & 1, abort, a.status);
+          ++qn;
+          if (ok) ok = full(it);
+          if (!ok) break;
+          tc_fence_after();
+          if (n0 > 0) {
+            issue_qk(S0, dq0, it);
+            mma_commit(bar_addr(&bars->s_full[0]));
+          }
+          if (act1(0)) {
+            issue_qk(S1, dq1, it);
+            mma_commit(bar_addr(&bars->s_full[1]));
+          }
+          after_s(0);
+          release(it);
+          for (int j = 0; ok && j < n1; ++j) {
+            const uint32_t iv = it + 2 * j + 1, ik = it + 2 * j + 2;
+            if (!(ok = full(iv))) break;
+            tc_fence_after();
+            if (j < n0) {
+              if (!(ok = wait_bar(bar_addr(&bars->p_ready[0]), pc0 & 1, abort, a.status))) break;
+              ++pc0;
+              tc_fence_after();
+              issue_pv(O0, S0, iv, j > 0);
+              if (j == n0 - 1) mma_commit(bar_addr(&bars->o_done[0]));
+            }
+            const bool next = j + 1 < n1;
+            if (next) {
+              if (!(ok = full(ik))) break;
+              tc_fence_after();
+              if (j + 1 < n0) {
+                issue_qk(S0, dq0, ik);
+                mma_commit(bar_addr(&bars->s_full[0]));
+              }
+            }
+            if (act1(j)) {
+              if (!(ok = wait_bar(bar_addr(&bars->p_ready[1]), pc1 & 1, abort, a.status))) break;
+              ++pc1;
+              tc_fence_after();
+              issue_pv(O1, S1, iv, j > s1);
+              if (j == n1 - 1) mma_commit(bar_addr(&bars->o_done[1]));
+            }
+            release(iv);
+            if (next) {
+              if (act1(j + 1)) {
+                issue_qk(S1, dq1, ik);
+                mma_commit(bar_addr(&bars->s_full[1]));
+              }
+              after_s(j + 1);
+              release(ik);
+            }
+          }
+          it += 2 * n1;
+        }
+        if (!ok) *abort = 1;
+        // every MMA and commit issued above must have completed before TMEM is freed
+        mma_commit(bar_addr(&bars->drain));
+        wait_bar(bar_addr(&bars->drain), 0, abort, a.status, false);
+      }
     }
-  }
   } else {
     setmaxnreg_inc<kRegsSoftmax>();
     // =============================== softmax + epilogue ================================
