@@ -230,3 +230,27 @@ def test_causal_attention_from_band_masked_key_chunks():
     ref, rm, rl = G.oracle_fwd(full)
     G.check_out(G.f64(got), ref, W.BF16, "causal from chunks", abs_ref=lambda: G.oracle_abs_fwd(full))
     G.check_stats(acc[1][..., 0].cpu().numpy(), acc[2][..., 0].cpu().numpy(), rm, rl, "causal stats")
+
+
+# ---- the two forms of a work item of the bf16 kernel, across GQA group sizes --------------------
+# With an even number of query heads per KV head an item is the same 128 rows of two query heads
+# of one group; otherwise it is 256 consecutive rows of one head. Both forms, on a packed batch
+# with ragged and empty sequences, for the plain, causal, band and explicit-mask paths.
+GROUPS = [(2, 1), (6, 2), (8, 2), (16, 2), (5, 5)]
+GROUP_IDS = ["group2", "group3", "group4", "group8", "mha"]
+
+
+@pytest.mark.parametrize("Nq,Nkv", GROUPS, ids=GROUP_IDS)
+@pytest.mark.parametrize("mode", [W.MASK_NONE, W.MASK_CAUSAL_TOPLEFT, BAND], ids=["full", "causal", "band"])
+def test_item_forms_across_groups(Nq, Nkv, mode):
+    inp = W.varlen_tnd([300, 0, 129, 520], Nq, Nkv, 128, causal=False, dtype=BF, seed=Nq * 10 + Nkv, cfg=41)
+    _check(inp, mode=mode, pre=200, nxt=0)
+
+
+@pytest.mark.parametrize("Nq,Nkv", [(8, 2), (6, 2)], ids=["group4", "group3"])
+def test_item_forms_with_explicit_mask(Nq, Nkv):
+    inp = W.varlen_tnd([300, 129, 520], Nq, Nkv, 128, causal=False, dtype=BF, seed=Nq + 7 * Nkv, cfg=42)
+    rng = np.random.default_rng(Nq * Nkv)
+    rs, bs = 528, 528 * 528
+    mask = _random_mask(rng, inp.B, 528, 528, rs, bs, p=0.3, full_row=(1, 7))
+    _check(inp, mode=W.MASK_CAUSAL_TOPLEFT, mask=mask, bs=bs, rs=rs)
