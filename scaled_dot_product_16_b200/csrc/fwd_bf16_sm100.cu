@@ -755,7 +755,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool any = mraw > -INFINITY && l > 0.f && ok;
         const float m_loc = any ? mraw * a.scale : -INFINITY;
         const float l_loc = any ? l * ex2(m - mraw * scale_log2) : 0.f;
-        float f_o = any ? 1.f / l : 0.f;  // factor on the unnormalised O in TMEM
+        float f_o = any ? __frcp_rn(l) : 0.f;  // factor on the unnormalised O in TMEM
         float f_prev = 0.f;               // factor on the accumulator's previous output row
         int64_t orow, so;
         if (a.acc_mode == kAccNone) {
@@ -812,17 +812,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                 prev[4 * x + 3] = t.w;
               }
             }
+            // O is finite, so a row that saw no key (f_o = 0) gives zeros
             uint32_t pkd[16];
+            if (a.acc_mode == kAccMerge) {
 #pragma unroll
-            for (int x = 0; x < 16; ++x) {
-              float v0 = f_o == 0.f ? 0.f : __uint_as_float(o[2 * x]) * f_o;
-              float v1 = f_o == 0.f ? 0.f : __uint_as_float(o[2 * x + 1]) * f_o;
-              if (a.acc_mode == kAccMerge) {
+              for (int x = 0; x < 16; ++x) {
                 const float2 pv = unpack16x2<F16>(prev[x]);
-                v0 = fmaf(pv.x, f_prev, v0);
-                v1 = fmaf(pv.y, f_prev, v1);
+                pkd[x] = pack16x2<F16>(fmaf(pv.x, f_prev, __uint_as_float(o[2 * x]) * f_o),
+                                       fmaf(pv.y, f_prev, __uint_as_float(o[2 * x + 1]) * f_o));
               }
-              pkd[x] = pack16x2<F16>(v0, v1);
+            } else {
+#pragma unroll
+              for (int x = 0; x < 16; ++x)
+                pkd[x] = pack16x2<F16>(__uint_as_float(o[2 * x]) * f_o, __uint_as_float(o[2 * x + 1]) * f_o);
             }
             if (tma_out) {
 #pragma unroll
