@@ -442,20 +442,24 @@ cudaError_t launch_d(const CsrArgs& a, cudaStream_t st, int num_sms) {
   const Cand cands[] = {{128, resident_blocks<D, 128>()}, {112, resident_blocks<D, 112>()},
                         {96, resident_blocks<D, 96>()},   {80, resident_blocks<D, 80>()},
                         {64, resident_blocks<D, 64>()}};
-  int best = 0;
+  // candidates that cannot be resident at all are skipped; the 128-row block's residency is the
+  // reference (if it cannot run, the first size that can sets it)
+  int ref = -1, best = -1;
   int64_t best_cost = 0;
   for (int c = 0; c < 5; ++c) {
-    if (cands[c].resident <= 0) return cudaErrorInvalidConfiguration;
-    if (cands[c].resident != cands[0].resident) continue;
+    if (cands[c].resident <= 0) continue;
+    if (ref < 0) ref = c;
+    if (cands[c].resident != cands[ref].resident) continue;
     const int64_t blocks = (int64_t)a.B * a.H * ((a.S + cands[c].rows - 1) / cands[c].rows);
     const int64_t slots = (int64_t)cands[c].resident * (num_sms > 0 ? num_sms : 1);
     const int64_t rounds = (blocks + slots - 1) / slots;
     const int64_t cost = rounds * (kFixedRows + cands[c].rows);
-    if (c == 0 || cost < best_cost) {
+    if (best < 0 || cost < best_cost) {
       best = c;
       best_cost = cost;
     }
   }
+  if (best < 0) return cudaErrorInvalidConfiguration;
   switch (cands[best].rows) {
     case 128: return launch_rows<D, 128>(a, st);
     case 112: return launch_rows<D, 112>(a, st);
