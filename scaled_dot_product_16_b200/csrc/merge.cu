@@ -103,6 +103,18 @@ __device__ __forceinline__ void from_f(float x, __half* p) { *p = __float2half_r
 __device__ __forceinline__ void from_f(float x, __nv_bfloat16* p) { *p = __float2bfloat16_rn(x); }
 __device__ __forceinline__ void from_f(float x, float* p) { *p = x; }
 
+// 32-byte global accesses that do not allocate in L1 (every byte of the merge is touched once).
+__device__ __forceinline__ void ld32_na(const void* p, uint4& lo, uint4& hi) {
+  asm volatile("ld.global.L1::no_allocate.v8.f32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+               : "=r"(lo.x), "=r"(lo.y), "=r"(lo.z), "=r"(lo.w), "=r"(hi.x), "=r"(hi.y), "=r"(hi.z), "=r"(hi.w)
+               : "l"(p));
+}
+__device__ __forceinline__ void st32_na(void* p, const uint4& lo, const uint4& hi) {
+  asm volatile("st.global.L1::no_allocate.v8.f32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(lo.x),
+               "r"(lo.y), "r"(lo.z), "r"(lo.w), "r"(hi.x), "r"(hi.y), "r"(hi.z), "r"(hi.w)
+               : "memory");
+}
+
 // Lane-wise statistics update; returns the lane's scaled partial sums.
 __device__ __forceinline__ void merge_lane(float pm, float ps, float cm, float cs, float* m,
                                            float* ps2, float* cs2) {
@@ -209,13 +221,16 @@ __global__ void __launch_bounds__(kThreads) merge_sbh_kernel(
 // element read and written by the same thread, so the outputs may alias prev_*) and hands
 // the lane-0 output scales through shared memory. The barrier therefore overlaps the bulk
 // loads instead of preceding them.
-template <typename T, int ROWS, int THREADS, int PER, bool FLAT>
+// W32: 32-byte accesses (two 16-byte vectors each) when every row base is 32-byte aligned.
+template <typename T, int ROWS, int THREADS, int PER, bool FLAT, bool W32>
 __global__ void __launch_bounds__(THREADS) merge_sbh_vec_kernel(
     const T* prev_out, const float* prev_max, const float* prev_sum,  // may alias the outputs
     const T* __restrict__ cur_out, const float* __restrict__ cur_max,
     const float* __restrict__ cur_sum, int S, int B, int N, int D, T* out, float* out_max,
     float* out_sum) {
-  constexpr int V = Vec16<T>::n;
+  constexpr int V16 = Vec16<T>::n;        // elements per 16-byte vector
+  constexpr int H = W32 ? 2 : 1;           // 16-byte vectors per access
+  constexpr int V = V16 * H;               // elements per access
   __shared__ float s_po[ROWS], s_co[ROWS];
   // SBH: block (b*N + n, s-block); FLAT (TND): block = ROWS consecutive rows t*N + n
   const int bn = FLAT ? 0 : blockIdx.x;
@@ -229,15 +244,20 @@ __global__ void __launch_bounds__(THREADS) merge_sbh_vec_kernel(
   const int64_t row0 = FLAT ? s0 * D : ((int64_t)s0 * B + b) * N * D + (int64_t)n * D;
 
   // 1. bulk loads of the partial outputs, all in flight at once
-  uint4 pv[PER], cv[PER];
+  uint4 pv[PER][H], cv[PER][H];
 #pragma unroll
   for (int u = 0; u < PER; ++u) {
     const int idx = u * THREADS + threadIdx.x;
     if (idx < total) {
       const int r = idx / vpr, c = idx - r * vpr;
       const int64_t off = row0 + r * row_stride + (int64_t)c * V;
-      pv[u] = *reinterpret_cast<const uint4*>(prev_out + off);
-      cv[u] = *reinterpret_cast<const uint4*>(cur_out + off);
+      if constexpr (W32) {
+        ld32_na(prev_out + off, pv[u][0], pv[u][H - 1]);
+        ld32_na(cur_out + off, cv[u][0], cv[u][H - 1]);
+      } else {
+        pv[u][0] = *reinterpret_cast<const uint4*>(prev_out + off);
+        cv[u][0] = *reinterpret_cast<const uint4*>(cur_out + off);
+      }
     }
   }
   // 2. lane-wise statistics, one (row, lane) element per thread
@@ -264,22 +284,30 @@ __global__ void __launch_bounds__(THREADS) merge_sbh_vec_kernel(
     if (idx < total) {
       const int r = idx / vpr, c = idx - r * vpr;
       const int64_t off = row0 + r * row_stride + (int64_t)c * V;
-      float a[V], bb[V], o[V];
-      unpack(pv[u], a, (T*)nullptr);
-      unpack(cv[u], bb, (T*)nullptr);
       const float po = s_po[r], co = s_co[r];
+      uint4 res[H];
 #pragma unroll
-      for (int i = 0; i < V; ++i) o[i] = fmaf(a[i], po, bb[i] * co);
-      *reinterpret_cast<uint4*>(out + off) = pack(o, (T*)nullptr);
+      for (int h = 0; h < H; ++h) {
+        float a[V16], bb[V16], o[V16];
+        unpack(pv[u][h], a, (T*)nullptr);
+        unpack(cv[u][h], bb, (T*)nullptr);
+#pragma unroll
+        for (int i = 0; i < V16; ++i) o[i] = fmaf(a[i], po, bb[i] * co);
+        res[h] = pack(o, (T*)nullptr);
+      }
+      if constexpr (W32)
+        st32_na(out + off, res[0], res[H - 1]);
+      else
+        *reinterpret_cast<uint4*>(out + off) = res[0];
     }
   }
 }
 
-template <typename T, int ROWS, int THREADS, int PER, bool FLAT>
+template <typename T, int ROWS, int THREADS, int PER, bool FLAT, bool W32 = false>
 void launch_vec(const MergeArgs& a, cudaStream_t st) {
   const dim3 grid = FLAT ? dim3((unsigned)(((int64_t)a.S * a.N + ROWS - 1) / ROWS), 1)
                          : dim3(a.B * a.N, (a.S + ROWS - 1) / ROWS);
-  merge_sbh_vec_kernel<T, ROWS, THREADS, PER, FLAT><<<grid, THREADS, 0, st>>>(
+  merge_sbh_vec_kernel<T, ROWS, THREADS, PER, FLAT, W32><<<grid, THREADS, 0, st>>>(
       (const T*)a.prev_out, a.prev_max, a.prev_sum, (const T*)a.cur_out, a.cur_max, a.cur_sum,
       a.S, a.B, a.N, a.D, (T*)a.out, a.out_max, a.out_sum);
 }
@@ -306,7 +334,13 @@ void launch_layout(const MergeArgs& a, cudaStream_t st) {
   // tiny blocks (8 rows x 64 threads x 2 vectors) measured fastest: many independent blocks
   const int vpr = a.D / V;
   constexpr int R = SDPA_MERGE_ROWS, TH = SDPA_MERGE_THREADS, PR = SDPA_MERGE_PER;
-  if (vec && R * vpr <= PR * TH)
+  // 32-byte accesses: D a multiple of two vectors and every output base 32-byte aligned (row
+  // strides are then multiples of 32 bytes too)
+  const bool w32 = vec && (a.D % (2 * V)) == 0 && ((uintptr_t)a.prev_out % 32) == 0 &&
+                   ((uintptr_t)a.cur_out % 32) == 0 && ((uintptr_t)a.out % 32) == 0;
+  if (w32 && R * (vpr / 2) <= (PR / 2 > 0 ? PR / 2 : 1) * TH)
+    launch_vec<T, R, TH, (PR / 2 > 0 ? PR / 2 : 1), FLAT, true>(a, st);
+  else if (vec && R * vpr <= PR * TH)
     launch_vec<T, R, TH, PR, FLAT>(a, st);
   else if (vec && 16 * vpr <= 4 * 256)
     launch_vec<T, 16, 256, 4, FLAT>(a, st);
