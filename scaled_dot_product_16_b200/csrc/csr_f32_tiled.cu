@@ -253,7 +253,7 @@ __global__ void __launch_bounds__(2 * ROWS, D == 64 ? 2 : 1) csr_f32_tiled_kerne
     for (int i = 0; i < 4; ++i)
 #pragma unroll
       for (int j = 0; j < 4; ++j) sc[i][j] = 0.f;
-#pragma unroll 2
+#pragma unroll 8  // (2, 4 and 16 measured slower)
     for (int d = 0; d < D; d += 4) {
       float4 kk[4];
 #pragma unroll
@@ -320,7 +320,7 @@ __global__ void __launch_bounds__(2 * ROWS, D == 64 ? 2 : 1) csr_f32_tiled_kerne
     for (int i = 0; i < 4; ++i)
 #pragma unroll
       for (int c = 0; c < kV4 * 4; ++c) o[i][c] *= corr[i];
-#pragma unroll 4
+#pragma unroll 8  // (4, 16 and 32 measured slower)
     for (int k = 0; k < kKeys; ++k) {
       const float4 p4 = *reinterpret_cast<const float4*>(Pt + k * kPtStride + 4 * rg);
       const float pk[4] = {p4.x, p4.y, p4.z, p4.w};
