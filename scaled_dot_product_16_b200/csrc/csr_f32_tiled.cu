@@ -305,7 +305,8 @@ __global__ void __launch_bounds__(2 * ROWS, D == 64 ? 2 : 1) csr_f32_tiled_kerne
         }
       }
 #pragma unroll
-      for (int x = 1; x < 8; x <<= 1) rs += __shfl_xor_sync(0xffffffffu, rs, x);
+      // this lane's part of the row sum: the 8 lanes of a row share its max (so its rescale
+      // factor), and their parts are added once, after the last tile
       l[i] = l[i] * corr[i] + rs;
       m[i] = mnew;
     }
@@ -342,6 +343,10 @@ __global__ void __launch_bounds__(2 * ROWS, D == 64 ? 2 : 1) csr_f32_tiled_kerne
     }
   }
   __syncthreads();
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int x = 1; x < 8; x <<= 1) l[i] += __shfl_xor_sync(0xffffffffu, l[i], x);
 
   // ---- epilogue: O / l; bad rows are zeros, heavy rows are redone below -----------------------
 #pragma unroll
