@@ -277,38 +277,48 @@ __global__ void __launch_bounds__(2 * ROWS, D == 64 ? 2 : 1) csr_f32_tiled_kerne
         }
       }
     }
-    // online softmax per row over the 8 threads that share it
-    float corr[4], p[4][4];
+    // Online softmax per row over the 8 lanes that share it. The max in use is raised only when
+    // some stored score of the tile exceeds it by more than 2^kLazyLog2 (log2 units, as the
+    // scores are): only then is the tile's row max reduced over the 8 lanes and O and the sum
+    // rescaled. Otherwise P is taken against the max in use (each P at most 2^kLazyLog2, and
+    // the same max for the row's P, sum and O, so the result is unchanged).
+    constexpr float kLazyLog2 = 8.f;
+    float corr[4], p[4][4], lmax[4];
+    bool has[4][4];
+    bool need = false;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const uint32_t mw = marks[(4 * rg + i) * kMaskStride + t % kWinTiles] >> kg;
-      bool has[4];
-      float tmax = -INFINITY;
+      lmax[i] = -INFINITY;
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        has[j] = ((mw >> (8 * j)) & 1u) != 0u;
-        if (has[j]) tmax = fmaxf(tmax, sc[i][j]);
+        has[i][j] = ((mw >> (8 * j)) & 1u) != 0u;
+        if (has[i][j]) lmax[i] = fmaxf(lmax[i], sc[i][j]);
       }
+      need |= lmax[i] > m[i] + kLazyLog2;  // also true for the first finite score of a row
+    }
+    const bool bump = __any_sync(0xffffffffu, need);
 #pragma unroll
-      for (int x = 1; x < 8; x <<= 1) tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, x));
-      const float mnew = fmaxf(m[i], tmax);
-      float rs = 0.f;
+    for (int i = 0; i < 4; ++i) {
       corr[i] = 1.f;
+      if (bump) {
+        float tmax = lmax[i];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) p[i][j] = 0.f;
-      if (mnew != -INFINITY) {
-        corr[i] = m[i] == -INFINITY ? 0.f : ex2_approx(m[i] - mnew);
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          p[i][j] = has[j] ? ex2_approx(sc[i][j] - mnew) : 0.f;
-          rs += p[i][j];
+        for (int x = 1; x < 8; x <<= 1) tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, x));
+        if (tmax > m[i] + kLazyLog2) {  // the same on the row's 8 lanes
+          corr[i] = m[i] == -INFINITY ? 0.f : ex2_approx(m[i] - tmax);
+          m[i] = tmax;
         }
       }
+      float rs = 0.f;
 #pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        p[i][j] = has[i][j] && m[i] != -INFINITY ? ex2_approx(sc[i][j] - m[i]) : 0.f;
+        rs += p[i][j];
+      }
       // this lane's part of the row sum: the 8 lanes of a row share its max (so its rescale
       // factor), and their parts are added once, after the last tile
       l[i] = l[i] * corr[i] + rs;
-      m[i] = mnew;
     }
     // P transposed: key kg + 8j's 4 rows 4rg.. as one 16-byte store, read back below as one
     // 16-byte load per key by the same 8 lanes of this warp
@@ -316,11 +326,13 @@ __global__ void __launch_bounds__(2 * ROWS, D == 64 ? 2 : 1) csr_f32_tiled_kerne
     for (int j = 0; j < 4; ++j)
       *reinterpret_cast<float4*>(Pt + (kg + 8 * j) * kPtStride + 4 * rg) = make_float4(p[0][j], p[1][j], p[2][j], p[3][j]);
     __syncwarp();
-    // O = O * corr + P V for rows 4rg.. and columns 4kg + 32c ..
+    // O = O * corr + P V for rows 4rg.. and columns 4kg + 32c .. (the rescale only after a bump)
+    if (bump) {
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
+      for (int i = 0; i < 4; ++i)
 #pragma unroll
-      for (int c = 0; c < kV4 * 4; ++c) o[i][c] *= corr[i];
+        for (int c = 0; c < kV4 * 4; ++c) o[i][c] *= corr[i];
+    }
 #pragma unroll 8  // (4, 16 and 32 measured slower)
     for (int k = 0; k < kKeys; ++k) {
       const float4 p4 = *reinterpret_cast<const float4*>(Pt + k * kPtStride + 4 * rg);
