@@ -333,8 +333,13 @@ __global__ void __launch_bounds__(2 * ROWS, D == 64 ? 2 : 1) csr_f32_tiled_kerne
 #pragma unroll
         for (int c = 0; c < kV4 * 4; ++c) o[i][c] *= corr[i];
     }
-#pragma unroll 8  // (4, 16 and 32 measured slower)
-    for (int k = 0; k < kKeys; ++k) {
+    // keys in groups of 8; a group that none of this warp's 16 rows stores is skipped
+    const uint32_t kmask = __reduce_or_sync(0xffffffffu, wmark);
+#pragma unroll 1
+    for (int g = 0; g < kKeys / 8; ++g) {
+    if (((kmask >> (8 * g)) & 0xffu) == 0u) continue;
+#pragma unroll
+    for (int k = 8 * g; k < 8 * g + 8; ++k) {
       const float4 p4 = *reinterpret_cast<const float4*>(Pt + k * kPtStride + 4 * rg);
       const float pk[4] = {p4.x, p4.y, p4.z, p4.w};
 #pragma unroll
@@ -352,6 +357,7 @@ __global__ void __launch_bounds__(2 * ROWS, D == 64 ? 2 : 1) csr_f32_tiled_kerne
           o[i][4 * c + 3] = hi.y;
         }
       }
+    }
     }
   }
   __syncthreads();
