@@ -654,9 +654,24 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_wait_ld();
           if constexpr (EXT == 0) {
             if (kbase + kBN > lim) {
+              const int hi = lim - kbase;  // this row's first masked column of the tile
 #pragma unroll
               for (int c = 0; c < kBN; ++c)
-                if (kbase + c >= lim) s[c >> 5][c & 31] = -INFINITY;
+                if (c >= hi) s[c >> 5][c & 31] = -INFINITY;
+            }
+          } else if constexpr (EXT == 1) {
+            // each edge on its own: a tile of a band wider than a tile holds at most one of them
+            if (kbase + kBN > lim) {
+              const int hi = lim - kbase;
+#pragma unroll
+              for (int c = 0; c < kBN; ++c)
+                if (c >= hi) s[c >> 5][c & 31] = -INFINITY;
+            }
+            if (kbase < lo) {
+              const int first = lo - kbase;  // this row's first visible column of the tile
+#pragma unroll
+              for (int c = 0; c < kBN; ++c)
+                if (c < first) s[c >> 5][c & 31] = -INFINITY;
             }
           } else {
             if (kbase + kBN > lim || kbase < lo) {
